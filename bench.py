@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""Benchmark of the ACE MoE layer forward on B200 through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload: the Qwen3-30B-A3B-shaped layer (hidden 2048, 128 experts of
+FFN 768, top-8, renormalised gates), prefill of 1 x 1024 tokens, 60% of the
+T*k slots skipped.  A "step" is one whole forward (RMSNorm, router, top-k,
+skip mask, compaction, gate/up GEMM + SiLU, down GEMM x gate, combine) over
+the batch.  Inputs are resident in HBM; the weights (1.2 GB) exceed L2, and
+L2 is also flushed (a 256 MiB write) before every timed step, outside the
+timed interval.  Each step is timed with CUDA events on the launching stream.
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank runs an
+independent replica (the layer forward has no exchange step); the time is the
+maximum over ranks and the value counts the tokens of all ranks.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (prefill, decode) at skip rate; % of tensor/HBM roofline"
+KERNELS_PER_FORWARD = 8  # rmsnorm, router GEMM, top-k/mask, scan, scatter, gate/up, down, combine
+
+
+# ----------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm_gbs=float(j["hbm_gbs"]), bf16_tflops=float(j["bf16_tflops"]),
+                    bf16_tflops_sustained=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ----------------------------------------------------------- our workload
+def tau_quantile_host(score, n_skip):
+    """tau = c_(n+1) over the non-top-1 scores sorted ascending (quantile
+    mapping of the target skip count)."""
+    cand = np.sort(score[:, 1:].reshape(-1).astype(np.float64))
+    if n_skip <= 0:
+        return float(cand[0])
+    if n_skip >= cand.size:
+        return float("inf")
+    return float(cand[n_skip])
+
+
+def setup_prefill(w, rate, device):
+    from token_dynamic_expert_b200 import ace
+    layer = workloads.make_layer(w, seed=w.seed, device=device)
+    u = workloads.make_tokens(w, device=device)
+    E = w.E
+    # ACE tables from the GPU table build
+    a_gsp = torch.empty(E, dtype=torch.float32, device=device)
+    a_rcr = torch.empty_like(a_gsp)
+    amax = torch.empty_like(a_gsp)
+    L0 = ace.make_layer(layer["gamma"], layer["wr"], layer["wg"], layer["wu"], layer["wd"], w.k,
+                        router_bias=layer["bias"])
+    tables = "ace_build_tables"
+    try:
+        tws = ace.alloc_workspace(ace.ace_tables_workspace_size(L0), device)
+        ace.ace_build_tables([L0], a_gsp, a_rcr, amax, tws)
+        del tws
+    except ace.AceError:
+        amax.fill_(1.0)
+        tables = "unit table (table build unavailable in this build)"
+    L = ace.make_layer(layer["gamma"], layer["wr"], layer["wg"], layer["wu"], layer["wd"], w.k,
+                       amax=amax, router_bias=layer["bias"])
+    ws = ace.alloc_workspace(ace.ace_workspace_size(L, w.T), device)
+    score = torch.empty(w.T, w.k, dtype=torch.float32, device=device)
+    ace.ace_moe_scores(L, u, score, ws)
+    torch.cuda.synchronize()
+    n_skip = int(np.floor(rate * (w.T * w.k if w.skip_of == "slots" else w.T * (w.k - 1)) + 0.5))
+    tau = tau_quantile_host(score.cpu().numpy(), n_skip)
+    tau32 = float(np.float32(tau)) if np.isfinite(tau) else float("inf")
+    y = torch.empty_like(u)
+    return dict(layer=layer, u=u, L=L, ws=ws, y=y, tau=tau32, amax=amax, tables=tables,
+                n_skip=n_skip)
+
+
+def slot_stats(st, w):
+    """Kept slots and touched experts of one forward (read once, untimed)."""
+    from token_dynamic_expert_b200 import ace
+    dbg = ace.DebugOut(w.T, w.k, w.E, st["u"].device)
+    ace.ace_moe_forward(st["L"], st["u"], st["tau"], st["y"], st["ws"], dbg=dbg.c)
+    code, flags = ace.ace_read_status(st["ws"])
+    if code != ace.ACE_OK:
+        raise RuntimeError("device status %s flags %#x" % (ace.ace_status_str(code), flags))
+    off = dbg.expert_offsets.cpu().numpy()
+    counts = np.diff(off)
+    return dict(S=int(dbg.n_kept.item()), touched=int((counts > 0).sum()),
+                skipped=int((dbg.keep == 0).sum().item()), counts=counts)
+
+
+def run_ours(args, w, rate, ws_n, rank, local):
+    from token_dynamic_expert_b200 import ace
+    dev = torch.device("cuda", local)
+    st = setup_prefill(w, rate, dev)
+    ss = slot_stats(st, w)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    dbgs = [ace.timing_debug(e[1], e[2], e[3]) for e in evs]
+
+    def step(i=None):
+        if i is None:
+            ace.ace_moe_forward(st["L"], st["u"], st["tau"], st["y"], st["ws"], stream=stream)
+        else:
+            e = evs[i]
+            e[0].record(stream)
+            ace.ace_moe_forward(st["L"], st["u"], st["tau"], st["y"], st["ws"], dbg=dbgs[i],
+                                stream=stream)
+            e[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    code, flags = ace.ace_read_status(st["ws"])
+    if code != ace.ACE_OK:
+        raise RuntimeError("device status %s flags %#x" % (ace.ace_status_str(code), flags))
+    barrier(ws_n)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(1)
+            step(i)
+        barrier(ws_n)
+    t_steps = [e[0].elapsed_time(e[4]) for e in evs]
+    t_gu = [e[1].elapsed_time(e[2]) for e in evs]
+    t_dn = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = max_over_ranks(sum(t_steps), ws_n)
+    ms_step = total_ms / args.steps
+    value = ws_n * args.steps * w.T / (total_ms / 1e3)
+
+    # roofline of the dominant kernel (gate/up GEMM + SiLU) and of the down GEMM
+    pk = peaks()
+    d, m, S, touched = w.d, w.m, ss["S"], ss["touched"]
+    gu_bytes = touched * 2 * m * d * 2 + S * d * 2 + S * m * 2
+    dn_bytes = touched * d * m * 2 + S * m * 2 + S * d * 4
+    gu_ms = statistics.mean(t_gu)
+    dn_ms = statistics.mean(t_dn)
+    gu_gbs = gu_bytes / (gu_ms / 1e3) / 1e9
+    dn_gbs = dn_bytes / (dn_ms / 1e3) / 1e9
+    flops = S * 2 * d * 3 * m
+    layer_bytes = touched * 3 * d * m * 2 + w.T * d * 2 * 2 + w.E * d * 2
+    roof_ms = max(flops / (pk["bf16_tflops"] * 1e12), layer_bytes / (pk["hbm_gbs"] * 1e9)) * 1e3
+
+    # end to end through the public API with host buffers
+    u_host = st["u"].cpu().pin_memory()
+    y_host = torch.empty_like(u_host).pin_memory()
+    u_dev, y_dev = st["u"], st["y"]
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    for _ in range(2):
+        u_dev.copy_(u_host, non_blocking=True)
+        step()
+        y_host.copy_(y_dev, non_blocking=True)
+    barrier(ws_n)
+    for i in range(args.steps):
+        flush.fill_(1)
+        e2e_ev[i][0].record(stream)
+        u_dev.copy_(u_host, non_blocking=True)
+        ace.ace_moe_forward(st["L"], u_dev, st["tau"], y_dev, st["ws"], stream=stream)
+        y_host.copy_(y_dev, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    barrier(ws_n)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), ws_n)
+    e2e_value = ws_n * args.steps * w.T / (e2e_ms / 1e3)
+    nbytes = w.T * w.d * u_host.element_size()
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,0.02) weights, N(0,1) tokens)",
+        "config": {"workload": w.name, "tokens": w.T, "hidden": w.d, "experts": w.E,
+                   "expert_ffn": w.m, "top_k": w.k, "skip_rate": rate,
+                   "skip_of": w.skip_of, "router_bias": w.bias, "tau": st["tau"],
+                   "realised_skip": ss["skipped"] / (w.T * w.k), "kept_slots": S,
+                   "touched_experts": touched, "tables": st["tables"],
+                   "parallelism": "replicas" if ws_n > 1 else "single",
+                   "l2": "flushed before each timed step (256 MiB write), flush untimed"},
+        "roofline": {"bound": "hbm", "achieved": gu_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": gu_gbs / pk["hbm_gbs"], "traffic": None,
+                     "kernel": "k_experts<0> (gate/up GEMM + SiLU)",
+                     "algorithmic_bytes": gu_bytes, "kernel_ms": gu_ms,
+                     "peak_source": pk["source"]},
+        "kernels": {
+            "down": {"achieved_gbs": dn_gbs, "frac": dn_gbs / pk["hbm_gbs"], "kernel_ms": dn_ms,
+                     "algorithmic_bytes": dn_bytes},
+            "layer": {"roofline_ms": roof_ms, "frac_of_roofline": roof_ms / ms_step,
+                      "tensor_frac": flops / (ms_step / 1e3) / (pk["bf16_tflops"] * 1e12),
+                      "flops": flops, "bytes": layer_bytes}},
+        "clocks": clk.summary(),
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+                "d2h_bytes_per_step": nbytes},
+        "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+    }
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, st, rate)
+    return out
+
+
+# ---------------------------------------------------------- CPU baselines
+def _oracle_inputs(st):
+    layer = {k: (v.detach().cpu() if torch.is_tensor(v) else v) for k, v in st["layer"].items()}
+    amax = st["amax"].cpu().numpy().astype(np.float32)
+    return layer, st["u"].cpu(), amax
+
+
+def cpu_baseline(w, st, rate, target_s=12.0):
+    """The oracle as it stands on the host cores, on a bounded sample of the
+    same workload (the first tokens of the batch)."""
+    import oracle
+    layer, u, amax = _oracle_inputs(st)
+    t0 = time.perf_counter()
+    oracle.moe_forward(layer, u[:8], st["tau"], amax, amax)
+    per_tok = (time.perf_counter() - t0) / 8
+    n = int(max(8, min(w.T, target_s / max(per_tok, 1e-6))))
+    t0 = time.perf_counter()
+    oracle.moe_forward(layer, u[:n], st["tau"], amax, amax)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": "%d of the %d tokens (fp64 forward incl. routing and mask), %.1f s"
+                      % (n, w.T, dt)}
+
+
+def run_reference(args, w, rate):
+    """The reference arm: the fp64 CPU oracle, each step a bounded sample."""
+    import oracle
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else None
+    if dev is None:
+        layer = workloads.make_layer(w)
+        u = workloads.make_tokens(w)
+        amax = np.ones(w.E, dtype=np.float32)
+        tau = 0.0
+    else:
+        st = setup_prefill(w, rate, dev)
+        layer, u, amax = _oracle_inputs(st)
+        tau = st["tau"]
+    t0 = time.perf_counter()
+    oracle.moe_forward(layer, u[:4], tau, amax, amax)
+    per_tok = (time.perf_counter() - t0) / 4
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    n = int(max(4, min(w.T, budget / max(per_tok, 1e-6))))
+    for _ in range(args.warmup):
+        oracle.moe_forward(layer, u[:n], tau, amax, amax)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.moe_forward(layer, u[:n], tau, amax, amax)
+    dt = time.perf_counter() - t0
+    val = args.steps * n / dt
+    return {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "tokens": w.T, "hidden": w.d, "experts": w.E,
+                       "expert_ffn": w.m, "top_k": w.k, "skip_rate": rate},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "kind": "oracle",
+                             "cores": oracle.threads(),
+                             "sample": "%d of %d tokens per step" % (n, w.T)},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill_1024",
+                    choices=["prefill_1024", "prefill_8192_e256", "sweep_4096"])
+    ap.add_argument("--rate", type=float, default=None, help="override the skip rate")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    w = workloads.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        rate = w.skip if args.rate is None else args.rate
+        print(json.dumps(run_reference(args, w, rate)), flush=True)
+        return
+
+    from token_dynamic_expert_b200 import build as _b  # noqa: F401  (the .so ships prebuilt)
+    ws_n, rank, local = dist_setup(args.gpus)
+    rates = [w.skip if args.rate is None else args.rate]
+    if args.workload == "sweep_4096" and args.rate is None:
+        rates = list(workloads.SWEEP_RATES)
+    for rate in rates:
+        out = run_ours(args, w, rate, ws_n, rank, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    if ws_n > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,226 @@
+/*
+ * ace.h -- C ABI of libace: the forward pass of a routed SwiGLU
+ * mixture-of-experts layer with ACE per-token expert skipping, and the
+ * offline construction of ACE's per-expert tables, on NVIDIA B200 (sm_100a).
+ *
+ * Method: "ACE: Adaptive Calibration-Free Expert Skipping for MoE-based
+ * LLMs" (picx.dev whiteboard summary of arXiv 2609.05228), cited as [ACE]
+ * with its section, and the news article "ACE Skips Low-Contribution MoE
+ * Experts Per Token" (ainews.surl.tw), cited as [NEWS].
+ *
+ * Conventions for every entry point
+ *   - Pointers marked (device) are CUDA device pointers owned by the caller;
+ *     the library never frees, retains or writes through a weight pointer
+ *     (checkpoint preservation, [ACE] "Practical Implications").
+ *   - The library allocates no device memory: scratch space is the caller's
+ *     workspace `ws` of at least the size the matching *_workspace_size
+ *     query returns, 256-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; nothing synchronises the
+ *     host except ace_read_status.  No call allocates or synchronises, so
+ *     the forward can be captured in a CUDA graph.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and return ACE_ERR_INVALID_ARG / ACE_ERR_WORKSPACE /
+ *     ACE_ERR_UNSUPPORTED.  Launch failures return ACE_ERR_CUDA.  Errors a
+ *     kernel detects (an index out of range, a pipeline wait that exceeded
+ *     its time limit) set bits in a status word inside the workspace; read
+ *     them with ace_read_status.
+ *   - Matrices are row-major.  Layouts (with the page's row-vector
+ *     convention: W^gate, W^up are d x m and W^down is m x d):
+ *       gamma      [d]        fp32   RMSNorm scale (diagonal of Gamma_l)
+ *       w_router   [E][d]     dtype  row e is the router vector w_{l,e}
+ *       router_bias[E]        fp32   optional, added to the logits
+ *       w_gate     [E][m][d]  dtype  w_gate[e][j][i] = W^gate_{l,e}[i][j]
+ *       w_up       [E][m][d]  dtype  likewise
+ *       w_down     [E][d][m]  dtype  w_down[e][i][j] = W^down_{l,e}[j][i]
+ *       u, y       [T][d]     dtype  layer input and output rows
+ */
+#ifndef ACE_H_
+#define ACE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ACE_API __attribute__((visibility("default")))
+#else
+#define ACE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ACE_OK = 0,
+  ACE_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer    */
+  ACE_ERR_WORKSPACE = 2,    /* workspace missing, too small or misaligned   */
+  ACE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed         */
+  ACE_ERR_UNSUPPORTED = 4,  /* valid but not implemented (shape, dtype)     */
+  ACE_ERR_DEVICE_FAULT = 5, /* a kernel flagged an out-of-range index       */
+  ACE_ERR_TIMEOUT = 6       /* a kernel's bounded wait ran out              */
+} ace_status;
+
+/* device status bits (ace_read_status) */
+#define ACE_FLAG_BAD_INDEX 0x1u    /* an expert/slot index outside its range */
+#define ACE_FLAG_TIMEOUT 0x2u      /* a pipeline wait exceeded its limit     */
+#define ACE_FLAG_OVERFLOW 0x4u     /* more kept slots than the workspace holds */
+
+typedef enum { ACE_BF16 = 0, ACE_F32 = 1 } ace_dtype;
+
+/* GSP norm: Frobenius exactly as printed in [ACE] "Methodology 1", or the
+ * spectral norm (largest singular value, power iteration). */
+typedef enum { ACE_GSP_FRO = 0, ACE_GSP_SPECTRAL = 1 } ace_gsp_norm;
+
+/* Fusion of the two views into one score ([ACE] "3. Conservative Fusion"). */
+typedef enum { ACE_FUSE_MAX = 0 } ace_fusion;
+
+/* One MoE layer: shapes, weights (device) and its ACE table. */
+typedef struct {
+  int d;                   /* hidden size                                  */
+  int E;                   /* routed experts                               */
+  int m;                   /* expert intermediate size                     */
+  int k;                   /* experts per token (top-k), 1 <= k <= E, <= 16 */
+  ace_dtype dtype;         /* storage and activation type                  */
+  const float* gamma;      /* [d]                                          */
+  const void* w_router;    /* [E][d]                                       */
+  const float* router_bias;/* [E] or NULL                                  */
+  const void* w_gate;      /* [E][m][d]                                    */
+  const void* w_up;        /* [E][m][d]                                    */
+  const void* w_down;      /* [E][d][m]                                    */
+  const float* amax;       /* [E] max(A^GSP, A^RCR) from ace_build_tables;
+                              NULL only for ace_moe_scores callers that want
+                              the raw gates (scores use 1.0 then)           */
+} ace_layer;
+
+/* Forward options. */
+typedef struct {
+  float tau;           /* skip threshold: slot i > 0 is skipped iff
+                          g_i * Amax[e_i] < tau ([ACE] "Conservative
+                          Fusion"; tau comes from the caller, one per layer
+                          and skip budget, [ACE] "Efficiency Results")    */
+  int renorm_topk;     /* 1: gates renormalised over the top-k (the gate of
+                          slot i is p_i / sum_topk p); 0: raw softmax p_i    */
+  ace_fusion fusion;   /* ACE_FUSE_MAX                                    */
+  float eps_rms;       /* RMSNorm epsilon (1e-6 in the shipped workloads)  */
+} ace_fwd_opts;
+
+/* Optional copies of the forward's intermediates (device pointers, each may
+ * be NULL).  Sizes use the call's T, k, E. */
+typedef struct {
+  int32_t* topk_idx;       /* [T][k] expert of slot (t, i); i = 0 is top-1 */
+  float* gate;             /* [T][k] gate g_{t,i}                          */
+  float* score;            /* [T][k] fused score c = g * Amax[e]           */
+  uint8_t* keep;           /* [T][k] 1 = kept, 0 = skipped                 */
+  int32_t* expert_offsets; /* [E+1] first kept slot of each expert         */
+  int32_t* slot_token;     /* [T*k] token of each kept slot (first n_kept)  */
+  int32_t* slot_rank;      /* [T*k] rank i of each kept slot               */
+  int32_t* n_kept;         /* [1]   number of kept slots                   */
+  float* logits;           /* [T][E] router logits (bias included)          */
+  /* Optional cudaEvent_t handles (passed as void*) recorded on the call's
+   * stream right before the gate/up expert GEMM, between it and the down
+   * GEMM, and right after the down GEMM: live kernel timing for profilers
+   * and benchmarks.  NULL = not recorded. */
+  void* ev_experts_begin;
+  void* ev_experts_mid;
+  void* ev_experts_end;
+} ace_debug_out;
+
+/* Table-build options ([ACE] "Methodology 1-2"). */
+typedef struct {
+  ace_gsp_norm gsp_norm; /* ACE_GSP_FRO (default) or ACE_GSP_SPECTRAL       */
+  float eps;             /* epsilon of the layer normalisations and of RCR  */
+  float rho;             /* RCR prototype scale rho_l (1.0 by default)      */
+  int power_iters;       /* power-iteration steps (200 by default)          */
+} ace_table_opts;
+
+/* ------------------------------------------------------------------------
+ * ace_workspace_size
+ *   Bytes of workspace ace_moe_forward / ace_moe_scores need for `layer`
+ *   and up to `max_tokens` tokens per call.  Returns 0 for an invalid
+ *   layer.  The size covers the worst case (no slot skipped).
+ * ---------------------------------------------------------------------- */
+ACE_API size_t ace_workspace_size(const ace_layer* layer, int max_tokens);
+
+/* ------------------------------------------------------------------------
+ * ace_moe_forward -- one MoE layer forward with ACE skipping.
+ *   [ACE] "Theoretical Foundation" (x = xbar Gamma and the SwiGLU expert
+ *   f_{l,e}), "Methodology 1-2" (scores s = g A), "3. Conservative Fusion"
+ *   (max-fusion, top-1 always kept); [NEWS] (online stage: table lookups,
+ *   the token's gate and scalar operations).
+ *   Per token t: x_t = RMSNorm(u_t) * gamma; logits x_t . w_e (+ b_e); the
+ *   top-k experts by logit (ties: lower index first); gates; scores
+ *   c = g * Amax[e]; slot i is kept iff i == 0 or !(c < tau); the kept
+ *   slots are grouped by expert (then token), run through their SwiGLU
+ *   experts, and y_t = sum over kept i, in rank order, of g_i f_{e_i}(x_t).
+ *   Skipped slots drop out without re-normalising the others.
+ *   u (device) [T][d], y (device) [T][d], both layer->dtype; they must not
+ *   overlap.  0 <= T <= max_tokens of the workspace.  T == 0 is a no-op.
+ *   dbg may be NULL.
+ *   bf16 layers run the expert GEMMs on tcgen05 tensor cores and need
+ *   d % 128 == 0 and m % 128 == 0; fp32 layers use CUDA cores.
+ * ---------------------------------------------------------------------- */
+ACE_API ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T,
+                           const ace_fwd_opts* opts, void* y, void* ws,
+                           size_t ws_bytes, ace_debug_out* dbg, void* stream);
+
+/* ------------------------------------------------------------------------
+ * ace_moe_scores -- only the routing half of the forward: fused scores
+ *   c = g * Amax[e] (gate alone when layer->amax is NULL) of every slot,
+ *   for building tau by quantile mapping ([ACE] "Efficiency Results",
+ *   Table 6).  score (device) [T][k] fp32, column 0 = top-1 slot;
+ *   topk_idx (device) [T][k] int32 or NULL.
+ * ---------------------------------------------------------------------- */
+ACE_API ace_status ace_moe_scores(const ace_layer* layer, const void* u, int T,
+                          const ace_fwd_opts* opts, float* score,
+                          int32_t* topk_idx, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* ------------------------------------------------------------------------
+ * ace_tables_workspace_size
+ *   Bytes of workspace ace_build_tables needs for layers shaped like
+ *   `layer` (d, E, m, dtype).
+ * ---------------------------------------------------------------------- */
+ACE_API size_t ace_tables_workspace_size(const ace_layer* layer);
+
+/* ------------------------------------------------------------------------
+ * ace_build_tables -- offline ACE statistics of n_layers layers (all with
+ *   the same d, E, m, dtype), [ACE] "Methodology 1" (GSP) and
+ *   "Methodology 2" (RCR):
+ *     a^up   = ||Gamma W^up|| ||Gamma W^gate W^down||
+ *     a^gate = ||Gamma W^gate|| ||Gamma W^up W^down||
+ *     A^GSP(e) = sqrt(a^up a^gate)_e / (mean_j sqrt(a^up a^gate)_j + eps)
+ *     q_e = (w_e - mean_j w_j) / (RMS(w_e - mean_j w_j) + eps) * rho
+ *     A^RCR(e) = a~_e / (mean_j a~_j + eps), a~_e = ||f_e(q_e)|| / (||q_e|| + eps)
+ *   Outputs (device, fp32, [n_layers][E]): a_gsp, a_rcr, amax = max of the
+ *   two (the table ace_moe_forward reads).  sigma (device, [n_layers][E][3]
+ *   or NULL) receives the largest singular values of Gamma W^gate,
+ *   Gamma W^up and W^down (the constants of the bound on ||f(x)|| in
+ *   [ACE] "Theoretical Foundation"), by power iteration from the all-ones
+ *   vector in R^m for opts->power_iters steps.  Weights are only read.
+ * ---------------------------------------------------------------------- */
+ACE_API ace_status ace_build_tables(const ace_layer* layers, int n_layers,
+                            const ace_table_opts* opts, float* a_gsp,
+                            float* a_rcr, float* amax, float* sigma, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * ace_read_status -- synchronise `stream` and return the device status
+ *   word that the most recent call using `ws` left there (ACE_FLAG_* bits in
+ *   *flags; every forward, scores or tables call clears it when it starts).
+ *   Returns ACE_ERR_TIMEOUT / ACE_ERR_DEVICE_FAULT when the corresponding
+ *   bit is set, else ACE_OK.  flags may be NULL.
+ * ---------------------------------------------------------------------- */
+ACE_API ace_status ace_read_status(void* ws, size_t ws_bytes, uint32_t* flags,
+                           void* stream);
+
+/* Human-readable name of a status code (static storage). */
+ACE_API const char* ace_status_str(ace_status s);
+
+/* Library version, "major.minor.patch" (static storage). */
+ACE_API const char* ace_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ACE_H_ */

@@ -1,0 +1,187 @@
+"""GPU parity of ace_moe_forward (through the C ABI) against the fp64 oracle.
+
+Sizes span several tiles and ragged tails; the full-size cases run in the
+launch configuration the benchmark times and compare every token's routing
+and mask, and a sample of tokens' outputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity_util import compare, midpoint_tau, run_gpu, setup_case
+
+pytestmark = pytest.mark.gpu
+
+W = workloads.Workload
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from token_dynamic_expert_b200 import build
+    build.build()
+
+
+def _check(w, tables="oracle", rate=None, T=None, renorm=True, seed=0, y_tol=2e-2,
+           out_tokens=None):
+    layer, u, A_gsp, A_rcr, amax, tau, n = setup_case(w, seed=seed, T=T, tables=tables, rate=rate)
+    gpu = run_gpu(layer, u, amax, tau, renorm=renorm)
+    res = compare(layer, u, gpu, A_gsp, A_rcr, tau, renorm=renorm, y_tol=y_tol,
+                  out_tokens=out_tokens)
+    skipped = int((gpu["keep"] == 0).sum())
+    if res["band"] == 0 and res["ties"] == 0 and np.isfinite(tau) and tau > 0:
+        assert skipped == n  # the threshold realises exactly the requested count
+    return res, gpu
+
+
+def test_tiny_fp32_layer():
+    """hidden 256, 8 experts of FFN 128, top-2, 64 tokens, fp32; tau skips
+    50% of the non-top-1 slots."""
+    res, gpu = _check(workloads.WORKLOADS["tiny_fp32"], y_tol=1e-4)
+    assert res["compared_tokens"] == 64
+    assert int((gpu["keep"][:, 1] == 0).sum()) == 32
+
+
+@pytest.mark.parametrize("w", [
+    W("multi_tile", T=300, d=256, E=16, m=256, k=4, dtype="bf16", bias=False, skip=0.5,
+      skip_of="slots"),
+    W("wide", T=200, d=512, E=8, m=384, k=2, dtype="bf16", bias=False, skip=0.3, skip_of="slots"),
+])
+def test_bf16_small_layers_oracle_tables(w):
+    res, _ = _check(w)
+    assert res["compared_tokens"] >= w.T - 2
+
+
+def test_bf16_expert_with_several_slot_tiles():
+    """8 experts, top-2, 1100 tokens: ~275 slots per expert, so every expert
+    spans two 256-slot tiles with a ragged second one."""
+    w = W("heavy", T=1100, d=256, E=8, m=128, k=2, dtype="bf16", bias=False, skip=0.1,
+          skip_of="slots")
+    res, gpu = _check(w, tables="spread")
+    counts = np.diff(gpu["expert_offsets"])
+    assert (counts > 256).any()
+
+
+def test_bf16_router_bias_skewed_load():
+    w = W("skewed", T=512, d=384, E=32, m=128, k=4, dtype="bf16", bias=True, skip=0.5,
+          skip_of="slots")
+    res, gpu = _check(w, tables="spread")
+    counts = np.diff(gpu["expert_offsets"])
+    assert counts.max() > 3 * max(1, counts.mean())  # the bias does skew the load
+
+
+@pytest.mark.parametrize("rate", [0.0, 0.75, 0.875])
+def test_skip_extremes(rate):
+    """0%: every slot kept (dense top-k MoE); 87.5% with k = 8: only top-1."""
+    w = W("extremes", T=96, d=256, E=16, m=128, k=8, dtype="bf16", bias=False, skip=rate,
+          skip_of="slots")
+    res, gpu = _check(w, rate=rate)
+    if rate == 0.0:
+        assert (gpu["keep"] == 1).all()
+    if rate == 0.875:
+        assert (gpu["keep"][:, 1:] == 0).all()
+
+
+def test_no_skip_matches_dense_topk_oracle():
+    w = W("dense", T=64, d=256, E=8, m=128, k=3, dtype="bf16", bias=False, skip=0.0,
+          skip_of="slots")
+    layer, u, A_gsp, A_rcr, amax, _, _ = setup_case(w)
+    gpu = run_gpu(layer, u, amax, -1.0)
+    assert (gpu["keep"] == 1).all()
+    ref = oracle.moe_forward(layer, u, -1.0, A_gsp, A_rcr)
+    dense = oracle.combine(ref["x"], ref["idx"], ref["gate"], np.ones_like(ref["keep"]),
+                           layer["wg"], layer["wu"], layer["wd"])
+    rel = np.abs(gpu["y"] - dense).max(1) / np.abs(dense).max(1)
+    assert rel.max() < 2e-2
+
+
+@pytest.mark.parametrize("k", [1, 8])
+def test_k_edge_cases(k):
+    w = W("k%d" % k, T=70, d=256, E=8, m=128, k=k, dtype="bf16", bias=False, skip=0.4,
+          skip_of="slots")
+    _check(w, rate=0.4 if k > 1 else 0.0)
+
+
+def test_raw_softmax_gates():
+    w = W("raw", T=128, d=256, E=16, m=128, k=4, dtype="bf16", bias=False, skip=0.5,
+          skip_of="slots")
+    _check(w, renorm=False)
+
+
+@pytest.mark.parametrize("T", [1, 2, 31, 33])
+def test_ragged_token_counts(T):
+    w = W("ragged", T=T, d=256, E=16, m=128, k=4, dtype="bf16", bias=False, skip=0.5,
+          skip_of="slots")
+    _check(w, T=T)
+
+
+def test_zero_tokens_is_a_noop():
+    from token_dynamic_expert_b200 import ace
+    w = W("empty", T=4, d=256, E=8, m=128, k=2, dtype="bf16", bias=False, skip=0.5,
+          skip_of="slots")
+    layer = workloads.make_layer(w)
+    amax = np.ones(w.E, dtype=np.float32)
+    from parity_util import gpu_layer
+    g, c = gpu_layer(layer, amax)
+    ws = ace.alloc_workspace(ace.ace_workspace_size(c, 4))
+    u = torch.empty(0, w.d, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(0, w.d, dtype=torch.bfloat16, device="cuda")
+    ace.ace_moe_forward(c, u, 0.1, y, ws)
+    assert ace.ace_read_status(ws) == (ace.ACE_OK, 0)
+
+
+def test_forward_is_deterministic():
+    w = W("det", T=256, d=256, E=16, m=256, k=4, dtype="bf16", bias=False, skip=0.5,
+          skip_of="slots")
+    layer, u, A_gsp, A_rcr, amax, tau, _ = setup_case(w, tables="spread")
+    a = run_gpu(layer, u, amax, tau)
+    b = run_gpu(layer, u, amax, tau)
+    assert np.array_equal(a["y"], b["y"])
+    assert np.array_equal(a["slot_token"], b["slot_token"])
+
+
+def test_forward_on_a_side_stream():
+    w = W("stream", T=100, d=256, E=8, m=128, k=2, dtype="bf16", bias=False, skip=0.3,
+          skip_of="slots")
+    layer, u, A_gsp, A_rcr, amax, tau, _ = setup_case(w)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        gpu = run_gpu(layer, u, amax, tau, stream=s)
+    compare(layer, u, gpu, A_gsp, A_rcr, tau)
+
+
+# ------------------------------------------------------------ full sizes
+def _full(w, n_out=48, seed=0):
+    """Full-size layer drawn on the GPU (the CPU copy feeds the oracle); RCR
+    table from the oracle, a spread GSP table; every token's routing and
+    mask compared, outputs on a sample of tokens."""
+    layer = workloads.make_layer(w, seed=seed, device="cuda")
+    u = workloads.make_tokens(w, device="cuda")
+    layer_cpu = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in layer.items()}
+    u_cpu = u.cpu()
+    r = oracle.rcr(layer_cpu["gamma"], layer_cpu["wr"], layer_cpu["wg"], layer_cpu["wu"],
+                   layer_cpu["wd"])
+    A_rcr = r["A"].astype(np.float32)
+    e = np.arange(w.E)
+    A_gsp = (0.5 + (e * 7 % 11) / 10.0).astype(np.float32)
+    ref = oracle.moe_forward(layer_cpu, u_cpu, 0.0, A_gsp, A_rcr, outputs=False)
+    n = oracle.n_skip_for(w.T, w.k, w.skip, of=w.skip_of)
+    tau = midpoint_tau(ref["c"], n)
+    gpu = run_gpu(layer_cpu, u_cpu, np.maximum(A_gsp, A_rcr), tau)
+    rng = np.random.default_rng(0)
+    toks = np.sort(rng.choice(w.T, size=n_out, replace=False))
+    res = compare(layer_cpu, u_cpu, gpu, A_gsp, A_rcr, tau, out_tokens=toks)
+    return res, gpu, n
+
+
+def test_full_prefill_1024():
+    res, gpu, n = _full(workloads.WORKLOADS["prefill_1024"])
+    assert res["mask_mismatch"] == 0
+    assert abs(int((gpu["keep"] == 0).sum()) - n) <= res["band"] + res["ties"] * 8
+
+
+def test_full_prefill_8192_e256_skewed():
+    res, gpu, n = _full(workloads.WORKLOADS["prefill_8192_e256"], n_out=32)
+    counts = np.diff(gpu["expert_offsets"])
+    assert counts.max() > 256  # skewed: some experts need several slot tiles

@@ -1,0 +1,273 @@
+// ace_api.cu -- the C ABI of libace (declared in include/ace.h): argument
+// validation, the workspace layout, and the launch sequence of the forward.
+#include <string.h>
+
+#include "ace_common.cuh"
+#include "ace_internal.h"
+
+namespace ace {
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+static size_t esize(ace_dtype dt) { return dt == ACE_BF16 ? 2 : 4; }
+
+FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms) {
+  FwdLayout o;
+  memset(&o, 0, sizeof(o));
+  const size_t T = (size_t)(max_tokens > 0 ? max_tokens : 1), k = (size_t)L.k, E = (size_t)L.E;
+  const size_t d = (size_t)L.d, m = (size_t)L.m, es = esize(L.dtype);
+  const size_t nchunk = (T + kChunk - 1) / kChunk, cap = T * k;
+  // largest split-K x tokens product over the token counts this workspace serves
+  size_t part = 0;
+  for (int gx = 1; gx <= cdiv((int)T, kRouterBT); ++gx) {
+    const int t = gx == cdiv((int)T, kRouterBT) ? (int)T : gx * kRouterBT;
+    const size_t p = (size_t)router_splitk(t, L.d, L.E, num_sms) * (size_t)t * E;
+    if (p > part) part = p;
+  }
+  o.max_tokens = (int)T;
+  o.part_floats = (int)part;
+  o.max_tiles = (int)E + cdiv((int)cap, kTileN);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  o.status = take(256);
+  o.part = take(part * 4);
+  o.inv_rms = take(T * 4);
+  o.x = take(T * d * es);
+  o.idx = take(cap * 4);
+  o.gate = take(cap * 4);
+  o.score = take(cap * 4);
+  o.keep = take(cap);
+  o.bitmap = take(nchunk * E * 4);
+  o.hist = take(nchunk * E * 4);
+  o.base = take(nchunk * E * 4);
+  o.counts = take(E * 4);
+  o.offsets = take((E + 1) * 4);
+  o.n_kept = take(4);
+  o.tiles = take((size_t)o.max_tiles * 16);
+  o.n_tiles = take(4);
+  o.slot_token = take(cap * 4);
+  o.slot_rank = take(cap * 4);
+  o.slot_gate = take(cap * 4);
+  o.slot_of = take(cap * 4);
+  o.xp = take(cap * d * es);
+  o.h = take(cap * m * es);
+  o.yslot = take(cap * d * 4);
+  o.total = off;
+  return o;
+}
+
+}  // namespace ace
+
+using namespace ace;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+ace_status check_layer(const ace_layer* L, bool need_experts) {
+  if (!L) return ACE_ERR_INVALID_ARG;
+  if (L->d <= 0 || L->E <= 0 || L->m <= 0 || L->k <= 0) return ACE_ERR_INVALID_ARG;
+  if (L->k > L->E || L->k > kMaxK) return ACE_ERR_INVALID_ARG;
+  if (L->dtype != ACE_BF16 && L->dtype != ACE_F32) return ACE_ERR_INVALID_ARG;
+  if (!L->gamma || !L->w_router) return ACE_ERR_INVALID_ARG;
+  if (L->E > kMaxE) return ACE_ERR_UNSUPPORTED;
+  if (L->d % 64 != 0 || L->m % 64 != 0) return ACE_ERR_UNSUPPORTED;
+  if (need_experts) {
+    if (!L->w_gate || !L->w_up || !L->w_down) return ACE_ERR_INVALID_ARG;
+    if (!aligned(L->w_gate, 16) || !aligned(L->w_up, 16) || !aligned(L->w_down, 16))
+      return ACE_ERR_INVALID_ARG;
+    if (L->dtype == ACE_BF16 && (L->d % 128 != 0 || L->m % 128 != 0)) return ACE_ERR_UNSUPPORTED;
+  }
+  if (!aligned(L->w_router, 16)) return ACE_ERR_INVALID_ARG;
+  return ACE_OK;
+}
+
+#define ACE_CK(call)                          \
+  do {                                        \
+    if ((call) != cudaSuccess) return ACE_ERR_CUDA; \
+  } while (0)
+
+template <typename P>
+P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// The routing half shared by the forward and the score query.
+ace_status run_routing(const ace_layer& L, const void* u, int T, const ace_fwd_opts& o,
+                       const FwdLayout& ly, void* ws, int num_sms, float* logits_dbg,
+                       cudaStream_t s) {
+  const int splitk = router_splitk(T, L.d, L.E, num_sms);
+  ACE_CK(launch_rmsnorm(L.dtype, u, T, L.d, L.gamma, o.eps_rms, at<float>(ws, ly.inv_rms),
+                        at<void>(ws, ly.x), s));
+  ACE_CK(launch_router_logits(L.dtype, u, at<float>(ws, ly.inv_rms), L.gamma, L.w_router, T, L.d,
+                              L.E, splitk, at<float>(ws, ly.part), s));
+  ACE_CK(launch_topk_mask(at<float>(ws, ly.part), splitk, T, L.E, L.k, L.router_bias, L.amax,
+                          o.tau, o.renorm_topk, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
+                          at<float>(ws, ly.score), at<uint8_t>(ws, ly.keep),
+                          at<uint32_t>(ws, ly.bitmap), at<int32_t>(ws, ly.hist), logits_dbg,
+                          at<uint32_t>(ws, ly.status), s));
+  return ACE_OK;
+}
+
+ace_status check_common(const ace_layer* layer, const void* u, int T, const ace_fwd_opts* opts,
+                        void* ws, bool need_experts) {
+  ace_status st = check_layer(layer, need_experts);
+  if (st != ACE_OK) return st;
+  if (!opts || T < 0) return ACE_ERR_INVALID_ARG;
+  if (opts->fusion != ACE_FUSE_MAX) return ACE_ERR_UNSUPPORTED;
+  if (T > 0 && (!u || !aligned(u, 16))) return ACE_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256)) return ACE_ERR_WORKSPACE;
+  return ACE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ace_workspace_size(const ace_layer* layer, int max_tokens) {
+  if (check_layer(layer, false) != ACE_OK || max_tokens < 0) return 0;
+  return fwd_layout(*layer, max_tokens, device_sm_count()).total;
+}
+
+ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T, const ace_fwd_opts* opts,
+                           void* y, void* ws, size_t ws_bytes, ace_debug_out* dbg,
+                           void* stream) {
+  ace_status st = check_common(layer, u, T, opts, ws, true);
+  if (st != ACE_OK) return st;
+  if (T > 0 && (!y || !aligned(y, 16))) return ACE_ERR_INVALID_ARG;
+  const ace_layer& L = *layer;
+  const size_t es = esize(L.dtype);
+  if (T > 0) {  // u and y may not overlap
+    const uint8_t *ub = (const uint8_t*)u, *yb = (const uint8_t*)y;
+    const size_t bytes = (size_t)T * L.d * es;
+    if (ub < yb + bytes && yb < ub + bytes) return ACE_ERR_INVALID_ARG;
+  }
+  const int num_sms = device_sm_count();
+  const FwdLayout ly = fwd_layout(L, T, num_sms);
+  if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ACE_CK(cudaMemsetAsync(at<void>(ws, ly.status), 0, 4, s));
+  if (T == 0) return ACE_OK;
+
+  st = run_routing(L, u, T, *opts, ly, ws, num_sms, dbg ? dbg->logits : nullptr, s);
+  if (st != ACE_OK) return st;
+  const int nchunk = cdiv(T, kChunk);
+  ACE_CK(launch_scan(at<int32_t>(ws, ly.hist), nchunk, L.E, kTileN, ly.max_tiles,
+                     at<int32_t>(ws, ly.base), at<int32_t>(ws, ly.counts),
+                     at<int32_t>(ws, ly.offsets), at<int32_t>(ws, ly.n_kept),
+                     at<int4>(ws, ly.tiles), at<int32_t>(ws, ly.n_tiles), s));
+  ACE_CK(launch_scatter(L.dtype, T, L.k, L.E, L.d, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
+                        at<uint8_t>(ws, ly.keep), at<uint32_t>(ws, ly.bitmap),
+                        at<int32_t>(ws, ly.base), at<void>(ws, ly.x),
+                        at<int32_t>(ws, ly.slot_token), at<int32_t>(ws, ly.slot_rank),
+                        at<float>(ws, ly.slot_gate), at<int32_t>(ws, ly.slot_of),
+                        at<void>(ws, ly.xp), at<uint32_t>(ws, ly.status), s));
+  cudaEvent_t ev_b = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_begin) : nullptr;
+  cudaEvent_t ev_m = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_mid) : nullptr;
+  cudaEvent_t ev_e = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_end) : nullptr;
+  if (ev_b) ACE_CK(cudaEventRecord(ev_b, s));
+  if (L.dtype == ACE_BF16) {
+    if (launch_experts_sm100(L, T * L.k, at<void>(ws, ly.xp), at<void>(ws, ly.h),
+                             at<float>(ws, ly.yslot), at<int4>(ws, ly.tiles),
+                             at<int32_t>(ws, ly.n_tiles), ly.max_tiles,
+                             at<float>(ws, ly.slot_gate), at<uint32_t>(ws, ly.status), num_sms,
+                             s, ev_m) != cudaSuccess)
+      return ACE_ERR_CUDA;
+  } else {
+    ACE_CK(launch_experts_simt(L, at<void>(ws, ly.xp), at<void>(ws, ly.h), at<float>(ws, ly.yslot),
+                               at<int4>(ws, ly.tiles), at<int32_t>(ws, ly.n_tiles), ly.max_tiles,
+                               at<float>(ws, ly.slot_gate), s));
+    if (ev_m) ACE_CK(cudaEventRecord(ev_m, s));
+  }
+  if (ev_e) ACE_CK(cudaEventRecord(ev_e, s));
+  ACE_CK(launch_combine(L.dtype, T, L.k, L.d, at<int32_t>(ws, ly.slot_of), at<float>(ws, ly.yslot),
+                        y, s));
+  if (dbg) {
+    const size_t tk = (size_t)T * L.k;
+    auto cp = [&](void* dst, size_t off, size_t bytes) -> bool {
+      return !dst || cudaMemcpyAsync(dst, at<void>(ws, off), bytes, cudaMemcpyDeviceToDevice, s) ==
+                         cudaSuccess;
+    };
+    if (!cp(dbg->topk_idx, ly.idx, tk * 4) || !cp(dbg->gate, ly.gate, tk * 4) ||
+        !cp(dbg->score, ly.score, tk * 4) || !cp(dbg->keep, ly.keep, tk) ||
+        !cp(dbg->expert_offsets, ly.offsets, ((size_t)L.E + 1) * 4) ||
+        !cp(dbg->slot_token, ly.slot_token, tk * 4) || !cp(dbg->slot_rank, ly.slot_rank, tk * 4) ||
+        !cp(dbg->n_kept, ly.n_kept, 4))
+      return ACE_ERR_CUDA;
+  }
+  return ACE_OK;
+}
+
+ace_status ace_moe_scores(const ace_layer* layer, const void* u, int T, const ace_fwd_opts* opts,
+                          float* score, int32_t* topk_idx, void* ws, size_t ws_bytes,
+                          void* stream) {
+  ace_status st = check_common(layer, u, T, opts, ws, false);
+  if (st != ACE_OK) return st;
+  if (T > 0 && !score) return ACE_ERR_INVALID_ARG;
+  const ace_layer& L = *layer;
+  const int num_sms = device_sm_count();
+  const FwdLayout ly = fwd_layout(L, T, num_sms);
+  if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ACE_CK(cudaMemsetAsync(at<void>(ws, ly.status), 0, 4, s));
+  if (T == 0) return ACE_OK;
+  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, s);
+  if (st != ACE_OK) return st;
+  const size_t tk = (size_t)T * L.k;
+  ACE_CK(cudaMemcpyAsync(score, at<void>(ws, ly.score), tk * 4, cudaMemcpyDeviceToDevice, s));
+  if (topk_idx)
+    ACE_CK(cudaMemcpyAsync(topk_idx, at<void>(ws, ly.idx), tk * 4, cudaMemcpyDeviceToDevice, s));
+  return ACE_OK;
+}
+
+ace_status ace_read_status(void* ws, size_t ws_bytes, uint32_t* flags, void* stream) {
+  if (!ws || ws_bytes < 4) return ACE_ERR_WORKSPACE;
+  uint32_t v = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return ACE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ACE_ERR_CUDA;
+  if (flags) *flags = v;
+  if (v & ACE_FLAG_TIMEOUT) return ACE_ERR_TIMEOUT;
+  if (v & (ACE_FLAG_BAD_INDEX | ACE_FLAG_OVERFLOW)) return ACE_ERR_DEVICE_FAULT;
+  return ACE_OK;
+}
+
+const char* ace_status_str(ace_status s) {
+  switch (s) {
+    case ACE_OK: return "ACE_OK";
+    case ACE_ERR_INVALID_ARG: return "ACE_ERR_INVALID_ARG";
+    case ACE_ERR_WORKSPACE: return "ACE_ERR_WORKSPACE";
+    case ACE_ERR_CUDA: return "ACE_ERR_CUDA";
+    case ACE_ERR_UNSUPPORTED: return "ACE_ERR_UNSUPPORTED";
+    case ACE_ERR_DEVICE_FAULT: return "ACE_ERR_DEVICE_FAULT";
+    case ACE_ERR_TIMEOUT: return "ACE_ERR_TIMEOUT";
+  }
+  return "ACE_UNKNOWN_STATUS";
+}
+
+const char* ace_version(void) { return "0.1.0"; }
+
+size_t ace_tables_workspace_size(const ace_layer* layer) {
+  (void)layer;
+  return 0;
+}
+
+ace_status ace_build_tables(const ace_layer* layers, int n_layers, const ace_table_opts* opts,
+                            float* a_gsp, float* a_rcr, float* amax, float* sigma, void* ws,
+                            size_t ws_bytes, void* stream) {
+  (void)layers; (void)n_layers; (void)opts; (void)a_gsp; (void)a_rcr; (void)amax; (void)sigma;
+  (void)ws; (void)ws_bytes; (void)stream;
+  return ACE_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

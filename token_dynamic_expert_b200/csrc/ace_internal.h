@@ -1,0 +1,70 @@
+// ace_internal.h -- host-side declarations shared by the libace translation
+// units: the forward workspace layout and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ace.h"
+
+namespace ace {
+
+constexpr int kChunk = 32;        // tokens per compaction chunk (one bit each)
+constexpr int kMaxE = 512;        // experts per layer the routing kernel holds
+constexpr int kMaxK = 16;         // top-k limit
+constexpr int kTileN = 256;       // kept slots per expert tile (GEMM N limit)
+constexpr int kRouterBT = 64;     // router GEMM tile: tokens
+constexpr int kRouterBE = 64;     // router GEMM tile: experts
+constexpr int kRouterBK = 32;     // router GEMM K step
+constexpr int kMaxSplitK = 16;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// Split of the router GEMM's K dimension for T tokens: enough CTAs to cover
+// the GPU twice, each split a multiple of the K step.
+int router_splitk(int T, int d, int E, int num_sms);
+
+// Byte offsets of the forward's scratch arrays inside the caller's
+// workspace.  Everything is sized for max_tokens and no skipping.
+struct FwdLayout {
+  size_t status, part, inv_rms, x, idx, gate, score, keep, bitmap, hist, base, counts,
+      offsets, n_kept, tiles, n_tiles, slot_token, slot_rank, slot_gate, slot_of, xp, h,
+      yslot, total;
+  int max_tokens, part_floats, max_tiles;
+};
+FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms);
+
+int device_sm_count();
+
+// ---------------------------------------------------------------- launchers
+cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
+                           float eps, float* inv_rms, void* x, cudaStream_t s);
+cudaError_t launch_router_logits(ace_dtype dt, const void* u, const float* inv_rms,
+                                 const float* gamma, const void* wr, int T, int d, int E,
+                                 int splitk, float* part, cudaStream_t s);
+cudaError_t launch_topk_mask(const float* part, int splitk, int T, int E, int k,
+                             const float* bias, const float* amax, float tau, int renorm,
+                             int32_t* idx, float* gate, float* score, uint8_t* keep,
+                             uint32_t* bitmap, int32_t* hist, float* logits_out,
+                             uint32_t* status, cudaStream_t s);
+cudaError_t launch_scan(const int32_t* hist, int nchunk, int E, int tile_n, int max_tiles,
+                        int32_t* base, int32_t* counts, int32_t* offsets, int32_t* n_kept,
+                        int4* tiles, int32_t* n_tiles, cudaStream_t s);
+cudaError_t launch_scatter(ace_dtype dt, int T, int k, int E, int d, const int32_t* idx,
+                           const float* gate, const uint8_t* keep, const uint32_t* bitmap,
+                           const int32_t* base, const void* x, int32_t* slot_token,
+                           int32_t* slot_rank, float* slot_gate, int32_t* slot_of, void* xp,
+                           uint32_t* status, cudaStream_t s);
+cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* xp, void* h,
+                                 float* yslot, const int4* tiles, const int32_t* n_tiles,
+                                 int max_tiles, const float* slot_gate, uint32_t* status,
+                                 int num_sms, cudaStream_t s, cudaEvent_t ev_mid);
+cudaError_t launch_experts_simt(const ace_layer& L, const void* xp, void* h, float* yslot,
+                                const int4* tiles, const int32_t* n_tiles, int max_tiles,
+                                const float* slot_gate, cudaStream_t s);
+cudaError_t launch_combine(ace_dtype dt, int T, int k, int d, const int32_t* slot_of,
+                           const float* yslot, void* y, cudaStream_t s);
+
+}  // namespace ace

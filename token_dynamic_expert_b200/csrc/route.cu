@@ -1,0 +1,253 @@
+// route.cu -- the online routing half of the ACE MoE forward.
+//
+//   k_rmsnorm        x_t = RMSNorm(u_t) * gamma, the expert input, and 1/rms_t
+//                    ([ACE] "Theoretical Foundation": x = xbar Gamma_l)
+//   k_router_logits  l_{t,e} = x_t . w_e, fp32 CUDA-core GEMM over a K split
+//   k_topk_mask      per token: top-k by logit, gates, ACE scores
+//                    c = g * max(A^GSP, A^RCR), skip mask with the top-1 slot
+//                    always kept ([ACE] "3. Conservative Fusion"; [NEWS]:
+//                    table lookups, the gate and scalar operations), plus the
+//                    per-chunk expert bitmaps the compaction consumes.
+//
+// The router logits use the unrounded fp32 x (u * (1/rms) * gamma); the
+// experts consume x rounded to the storage type.
+#include <float.h>
+#include <math.h>
+
+#include "ace_common.cuh"
+#include "ace_internal.h"
+
+namespace ace {
+
+// ------------------------------------------------------------------ RMSNorm
+template <typename T>
+__global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn, int d,
+                                                 const float* __restrict__ gamma, float eps,
+                                                 float* __restrict__ inv_rms, T* __restrict__ x) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= Tn) return;
+  const T* ur = u + (size_t)t * d;
+  float ss = 0.f;
+  for (int i = lane; i < d; i += 32) {
+    const float v = to_f(ur[i]);
+    ss = fmaf(v, v, ss);
+  }
+  ss = warp_sum(ss);
+  const float r = 1.0f / sqrtf(ss / (float)d + eps);
+  if (lane == 0) inv_rms[t] = r;
+  T* xr = x + (size_t)t * d;
+  for (int i = lane; i < d; i += 32) xr[i] = from_f<T>(to_f(ur[i]) * r * gamma[i]);
+}
+
+cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
+                           float eps, float* inv_rms, void* x, cudaStream_t s) {
+  dim3 grid(cdiv(T, 8));
+  if (dt == ACE_BF16)
+    k_rmsnorm<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)u, T, d, gamma, eps,
+                                                  inv_rms, (__nv_bfloat16*)x);
+  else
+    k_rmsnorm<float><<<grid, 256, 0, s>>>((const float*)u, T, d, gamma, eps, inv_rms, (float*)x);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ router logits
+// part[split][t][e] = sum over k in split's range of xhat[t][k] * w[e][k],
+// xhat = u * inv_rms * gamma.  64 x 64 output tile, 4 x 4 per thread.
+template <typename T>
+__global__ void __launch_bounds__(256) k_router_logits(const T* __restrict__ u,
+                                                       const float* __restrict__ inv_rms,
+                                                       const float* __restrict__ gamma,
+                                                       const T* __restrict__ wr, int Tn, int d,
+                                                       int E, int kper, float* __restrict__ part) {
+  __shared__ float As[kRouterBK][kRouterBT + 4];
+  __shared__ float Bs[kRouterBK][kRouterBE + 4];
+  const int t0 = blockIdx.x * kRouterBT, e0 = blockIdx.y * kRouterBE, split = blockIdx.z;
+  const int kbeg = split * kper, kend = kbeg + kper;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int lr = tid >> 2, lk = (tid & 3) * 8;
+  const bool arow = (t0 + lr) < Tn, brow = (e0 + lr) < E;
+  const float rr = arow ? inv_rms[t0 + lr] : 0.f;
+  const T* ua = u + (size_t)(arow ? t0 + lr : 0) * d;
+  const T* wb = wr + (size_t)(brow ? e0 + lr : 0) * d;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  for (int k0 = kbeg; k0 < kend; k0 += kRouterBK) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int kk = k0 + lk + j;
+      As[lk + j][lr] = arow ? to_f(ua[kk]) * rr * gamma[kk] : 0.f;
+      Bs[lk + j][lr] = brow ? to_f(wb[kk]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kRouterBK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* out = part + (size_t)split * Tn * E;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= Tn) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < E) out[(size_t)t * E + e] = acc[i][j];
+    }
+  }
+}
+
+int router_splitk(int T, int d, int E, int num_sms) {
+  const int tiles = cdiv(T, kRouterBT) * cdiv(E, kRouterBE);
+  int s = cdiv(2 * num_sms, tiles);
+  if (s > kMaxSplitK) s = kMaxSplitK;
+  if (s < 1) s = 1;
+  while (s > 1 && (d % (s * kRouterBK)) != 0) --s;
+  return s;
+}
+
+cudaError_t launch_router_logits(ace_dtype dt, const void* u, const float* inv_rms,
+                                 const float* gamma, const void* wr, int T, int d, int E,
+                                 int splitk, float* part, cudaStream_t s) {
+  dim3 grid(cdiv(T, kRouterBT), cdiv(E, kRouterBE), splitk);
+  const int kper = d / splitk;
+  if (dt == ACE_BF16)
+    k_router_logits<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)u, inv_rms, gamma,
+                                                        (const __nv_bfloat16*)wr, T, d, E, kper,
+                                                        part);
+  else
+    k_router_logits<float><<<grid, 256, 0, s>>>((const float*)u, inv_rms, gamma,
+                                                (const float*)wr, T, d, E, kper, part);
+  return cudaGetLastError();
+}
+
+// -------------------------------------------------------- top-k and the mask
+// One CTA per chunk of 32 tokens, one warp per token (8 warps, 4 tokens
+// each).  Lane l holds the logits of experts l, l+32, ...  Selection order is
+// (logit descending, expert index ascending); slot 0 is the top-1 expert.
+template <int V>
+__global__ void __launch_bounds__(256) k_topk_mask(
+    const float* __restrict__ part, int splitk, int Tn, int E, int k,
+    const float* __restrict__ bias, const float* __restrict__ amax, float tau, int renorm,
+    int32_t* __restrict__ idx, float* __restrict__ gate, float* __restrict__ score,
+    uint8_t* __restrict__ keep, uint32_t* __restrict__ bitmap, int32_t* __restrict__ hist,
+    float* __restrict__ logits_out, uint32_t* status) {
+  __shared__ uint32_t bm[kMaxE];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) bm[e] = 0u;
+  __syncthreads();
+  const int c = blockIdx.x;
+  for (int r = 0; r < kChunk / 8; ++r) {
+    const int tl = warp + 8 * r;
+    const int t = c * kChunk + tl;
+    if (t >= Tn) continue;
+    float v[V];
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+      const int e = lane + 32 * q;
+      if (e < E) {
+        float sum = 0.f;
+        for (int sp = 0; sp < splitk; ++sp) sum += part[((size_t)sp * Tn + t) * E + e];
+        if (bias) sum += bias[e];
+        if (logits_out) logits_out[(size_t)t * E + e] = sum;
+        v[q] = sum;
+      } else {
+        v[q] = -INFINITY;
+      }
+    }
+    uint32_t taken = 0u;
+    int my_e = 0;
+    float my_v = -INFINITY;
+    for (int i = 0; i < k; ++i) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int q = 0; q < V; ++q) {
+        const int e = lane + 32 * q;
+        if (!((taken >> q) & 1u) && e < E && (v[q] > bv || (v[q] == bv && e < be))) {
+          bv = v[q];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      if (be < 0 || be >= E) {  // non-finite logits: flag and fall back to expert 0
+        raise_flag(status, ACE_FLAG_BAD_INDEX);
+        be = 0;
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      if (lane == i) {
+        my_e = be;
+        my_v = bv;
+      }
+    }
+    const float v0 = __shfl_sync(0xffffffffu, my_v, 0);  // the top-1 logit is the maximum
+    const float ex = (lane < k) ? expf(my_v - v0) : 0.f;
+    float denom;
+    if (renorm) {
+      denom = warp_sum(ex);
+    } else {
+      float z = 0.f;
+#pragma unroll
+      for (int q = 0; q < V; ++q) z += (lane + 32 * q < E) ? expf(v[q] - v0) : 0.f;
+      denom = warp_sum(z);
+    }
+    if (lane < k) {
+      const float g = ex / denom;
+      const float sc = g * (amax ? amax[my_e] : 1.0f);
+      const bool kept = (lane == 0) || !(sc < tau);
+      const size_t o = (size_t)t * k + lane;
+      idx[o] = my_e;
+      gate[o] = g;
+      score[o] = sc;
+      keep[o] = kept ? 1 : 0;
+      if (kept) atomicOr(&bm[my_e], 1u << tl);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    bitmap[(size_t)c * E + e] = bm[e];
+    hist[(size_t)c * E + e] = __popc(bm[e]);
+  }
+}
+
+cudaError_t launch_topk_mask(const float* part, int splitk, int T, int E, int k,
+                             const float* bias, const float* amax, float tau, int renorm,
+                             int32_t* idx, float* gate, float* score, uint8_t* keep,
+                             uint32_t* bitmap, int32_t* hist, float* logits_out,
+                             uint32_t* status, cudaStream_t s) {
+  dim3 grid(cdiv(T, kChunk));
+#define ACE_TOPK(V)                                                                          \
+  k_topk_mask<V><<<grid, 256, 0, s>>>(part, splitk, T, E, k, bias, amax, tau, renorm, idx,    \
+                                      gate, score, keep, bitmap, hist, logits_out, status)
+  if (E <= 32) ACE_TOPK(1);
+  else if (E <= 64) ACE_TOPK(2);
+  else if (E <= 128) ACE_TOPK(4);
+  else if (E <= 256) ACE_TOPK(8);
+  else ACE_TOPK(16);
+#undef ACE_TOPK
+  return cudaGetLastError();
+}
+
+}  // namespace ace
