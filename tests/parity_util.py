@@ -136,7 +136,7 @@ def compare(layer_cpu, u_cpu, gpu, A_gsp32, A_rcr32, tau32, renorm=True, out_tok
     return res
 
 
-def setup_case(w, seed=0, token_seed=1000, T=None, tables="oracle", rate=None):
+def setup_case(w, seed=0, token_seed=1000, T=None, tables="oracle", rate=None, renorm=True):
     """Layer, tokens, fp32 tables and the midpoint threshold for a workload."""
     layer = workloads.make_layer(w, seed=seed)
     u = workloads.make_tokens(w, T=T, token_seed=token_seed)
@@ -149,7 +149,7 @@ def setup_case(w, seed=0, token_seed=1000, T=None, tables="oracle", rate=None):
     amax = np.maximum(A_gsp, A_rcr)
     rate = w.skip if rate is None else rate
     T_ = u.shape[0]
-    ref = oracle.moe_forward(layer, u, 0.0, A_gsp, A_rcr, outputs=False)
+    ref = oracle.moe_forward(layer, u, 0.0, A_gsp, A_rcr, renorm=renorm, outputs=False)
     n = oracle.n_skip_for(T_, w.k, rate, of=w.skip_of)
     tau = midpoint_tau(ref["c"], n)
     return layer, u, A_gsp, A_rcr, amax, tau, n

@@ -25,10 +25,12 @@ def _lib():
 
 def _check(w, tables="oracle", rate=None, T=None, renorm=True, seed=0, y_tol=2e-2,
            out_tokens=None):
-    layer, u, A_gsp, A_rcr, amax, tau, n = setup_case(w, seed=seed, T=T, tables=tables, rate=rate)
+    layer, u, A_gsp, A_rcr, amax, tau, n = setup_case(w, seed=seed, T=T, tables=tables, rate=rate,
+                                                      renorm=renorm)
     gpu = run_gpu(layer, u, amax, tau, renorm=renorm)
     res = compare(layer, u, gpu, A_gsp, A_rcr, tau, renorm=renorm, y_tol=y_tol,
                   out_tokens=out_tokens)
+    print(w.name, res)
     skipped = int((gpu["keep"] == 0).sum())
     if res["band"] == 0 and res["ties"] == 0 and np.isfinite(tau) and tau > 0:
         assert skipped == n  # the threshold realises exactly the requested count
@@ -172,6 +174,7 @@ def _full(w, n_out=48, seed=0):
     rng = np.random.default_rng(0)
     toks = np.sort(rng.choice(w.T, size=n_out, replace=False))
     res = compare(layer_cpu, u_cpu, gpu, A_gsp, A_rcr, tau, out_tokens=toks)
+    print(w.name, res)
     return res, gpu, n
 
 
