@@ -34,7 +34,8 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (prefill, decode) at skip rate; % of tensor/HBM roofline"
-KERNELS_PER_FORWARD = 8  # rmsnorm, router GEMM, top-k/mask, scan, scatter, gate/up, down, combine
+# rmsnorm, router GEMM, top-k/mask, scan, scatter, gather, gate/up, down, combine
+KERNELS_PER_FORWARD = 9
 
 
 # ----------------------------------------------------------------- helpers
@@ -51,60 +52,60 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """SM clock and clock-event (throttle) reasons, polled through NVML every
+    ~2 ms on a background thread while the timed region runs."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap"}
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.stop = threading.Event()
+        self.max_mhz = None
+        self.ok = False
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+            self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
-        except (OSError, ValueError):
-            self.proc = None
+        except Exception:  # NVML unavailable: report unsampled
+            self.ok = False
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self.nv
+        while not self.stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self.stop.set()
+        if self.ok:
+            self.t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        reasons = set()
+        for _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": "nvml"}
 
 
 def dist_setup(n):
@@ -202,39 +203,60 @@ def run_ours(args, w, rate, ws_n, rank, local):
     dev = torch.device("cuda", local)
     st = setup_prefill(w, rate, dev)
     ss = slot_stats(st, w)
-    stream = torch.cuda.current_stream()
+    stream = torch.cuda.Stream(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    dbgs = [ace.timing_debug(e[1], e[2], e[3]) for e in evs]
 
-    def step(i=None):
-        if i is None:
-            ace.ace_moe_forward(st["L"], st["u"], st["tau"], st["y"], st["ws"], stream=stream)
-        else:
-            e = evs[i]
-            e[0].record(stream)
-            ace.ace_moe_forward(st["L"], st["u"], st["tau"], st["y"], st["ws"], dbg=dbgs[i],
-                                stream=stream)
-            e[4].record(stream)
+    def fwd(dbg=None):
+        ace.ace_moe_forward(st["L"], st["u"], st["tau"], st["y"], st["ws"], dbg=dbg,
+                            stream=stream)
 
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        step()
-    code, flags = ace.ace_read_status(st["ws"])
-    if code != ace.ACE_OK:
-        raise RuntimeError("device status %s flags %#x" % (ace.ace_status_str(code), flags))
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            fwd()
+        code, flags = ace.ace_read_status(st["ws"], stream=stream)
+        if code != ace.ACE_OK:
+            raise RuntimeError("device status %s flags %#x" % (ace.ace_status_str(code), flags))
+        # the whole forward captured once and replayed: one graph launch per step
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            fwd()
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            graph.replay()
+    stream.synchronize()
+
+    # timed: K steps, each bracketed by events on the launching stream
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
     barrier(ws_n)
-    with ClockSampler(local) as clk:
+    with ClockSampler(local) as clk, torch.cuda.stream(stream):
         for i in range(args.steps):
             flush.fill_(1)
-            step(i)
-        barrier(ws_n)
-    t_steps = [e[0].elapsed_time(e[4]) for e in evs]
-    t_gu = [e[1].elapsed_time(e[2]) for e in evs]
-    t_dn = [e[2].elapsed_time(e[3]) for e in evs]
+            evs[i][0].record(stream)
+            graph.replay()
+            evs[i][1].record(stream)
+        stream.synchronize()
+    barrier(ws_n)
+    t_steps = [a.elapsed_time(b) for a, b in evs]
     total_ms = max_over_ranks(sum(t_steps), ws_n)
     ms_step = total_ms / args.steps
     value = ws_n * args.steps * w.T / (total_ms / 1e3)
+    code, flags = ace.ace_read_status(st["ws"], stream=stream)
+    if code != ace.ACE_OK:
+        raise RuntimeError("device status %s flags %#x" % (ace.ace_status_str(code), flags))
+
+    # per-kernel times of the expert GEMMs, recorded by the library on its stream
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    dbgs = [ace.timing_debug(*e) for e in kev]
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.fill_(1)
+            fwd(dbgs[i])
+        stream.synchronize()
+    t_gu = [e[0].elapsed_time(e[1]) for e in kev]
+    t_dn = [e[1].elapsed_time(e[2]) for e in kev]
 
     # roofline of the dominant kernel (gate/up GEMM + SiLU) and of the down GEMM
     pk = peaks()
@@ -249,28 +271,32 @@ def run_ours(args, w, rate, ws_n, rank, local):
     layer_bytes = touched * 3 * d * m * 2 + w.T * d * 2 * 2 + w.E * d * 2
     roof_ms = max(flops / (pk["bf16_tflops"] * 1e12), layer_bytes / (pk["hbm_gbs"] * 1e9)) * 1e3
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers (no graph)
     u_host = st["u"].cpu().pin_memory()
     y_host = torch.empty_like(u_host).pin_memory()
     u_dev, y_dev = st["u"], st["y"]
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
-    for _ in range(2):
-        u_dev.copy_(u_host, non_blocking=True)
-        step()
-        y_host.copy_(y_dev, non_blocking=True)
-    barrier(ws_n)
-    for i in range(args.steps):
-        flush.fill_(1)
-        e2e_ev[i][0].record(stream)
-        u_dev.copy_(u_host, non_blocking=True)
-        ace.ace_moe_forward(st["L"], u_dev, st["tau"], y_dev, st["ws"], stream=stream)
-        y_host.copy_(y_dev, non_blocking=True)
-        e2e_ev[i][1].record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            u_dev.copy_(u_host, non_blocking=True)
+            fwd()
+            y_host.copy_(y_dev, non_blocking=True)
+        stream.synchronize()
+        barrier(ws_n)
+        for i in range(args.steps):
+            flush.fill_(1)
+            e2e_ev[i][0].record(stream)
+            u_dev.copy_(u_host, non_blocking=True)
+            fwd()
+            y_host.copy_(y_dev, non_blocking=True)
+            e2e_ev[i][1].record(stream)
+        stream.synchronize()
     barrier(ws_n)
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), ws_n)
     e2e_value = ws_n * args.steps * w.T / (e2e_ms / 1e3)
     nbytes = w.T * w.d * u_host.element_size()
+    del graph
 
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
@@ -283,6 +309,7 @@ def run_ours(args, w, rate, ws_n, rank, local):
                    "realised_skip": ss["skipped"] / (w.T * w.k), "kept_slots": S,
                    "touched_experts": touched, "tables": st["tables"],
                    "parallelism": "replicas" if ws_n > 1 else "single",
+                   "launch": "forward captured in one CUDA graph, replayed per step",
                    "l2": "flushed before each timed step (256 MiB write), flush untimed"},
         "roofline": {"bound": "hbm", "achieved": gu_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": gu_gbs / pk["hbm_gbs"], "traffic": None,
@@ -297,7 +324,7 @@ def run_ours(args, w, rate, ws_n, rank, local):
                       "flops": flops, "bytes": layer_bytes}},
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
-                "d2h_bytes_per_step": nbytes},
+                "d2h_bytes_per_step": nbytes, "launch": "plain API calls, no graph"},
         "gpu_launches": KERNELS_PER_FORWARD * args.steps,
     }
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
@@ -307,9 +334,16 @@ def run_ours(args, w, rate, ws_n, rank, local):
 
 # ---------------------------------------------------------- CPU baselines
 def _oracle_inputs(st):
-    layer = {k: (v.detach().cpu() if torch.is_tensor(v) else v) for k, v in st["layer"].items()}
+    """Host copies in the oracle's input types (converted once, untimed)."""
+    def conv(v):
+        if not torch.is_tensor(v):
+            return v
+        v = v.detach().cpu()
+        return np.ascontiguousarray(v.float().numpy())
+    layer = {k: conv(v) for k, v in st["layer"].items()}
     amax = st["amax"].cpu().numpy().astype(np.float32)
-    return layer, st["u"].cpu(), amax
+    u = np.ascontiguousarray(st["u"].detach().cpu().float().numpy().astype(np.float64))
+    return layer, u, amax
 
 
 def cpu_baseline(w, st, rate, target_s=12.0):
@@ -370,8 +404,8 @@ def run_reference(args, w, rate):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="prefill_1024",
                     choices=["prefill_1024", "prefill_8192_e256", "sweep_4096"])
     ap.add_argument("--rate", type=float, default=None, help="override the skip rate")

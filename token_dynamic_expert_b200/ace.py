@@ -197,7 +197,10 @@ class DebugOut:
 
 
 def event_handle(ev):
-    """The cudaEvent_t behind a torch.cuda.Event, as a void* for the C ABI."""
+    """The cudaEvent_t behind a torch.cuda.Event, as a void* for the C ABI
+    (torch creates the CUDA event at its first record, so record it once)."""
+    if not ev.cuda_event:
+        ev.record()
     return ctypes.c_void_p(ev.cuda_event)
 
 

@@ -172,6 +172,8 @@ ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T, const a
                         at<int32_t>(ws, ly.slot_token), at<int32_t>(ws, ly.slot_rank),
                         at<float>(ws, ly.slot_gate), at<int32_t>(ws, ly.slot_of),
                         at<void>(ws, ly.xp), at<uint32_t>(ws, ly.status), s));
+  ACE_CK(launch_gather(L.dtype, T * L.k, L.d, at<int32_t>(ws, ly.n_kept),
+                       at<int32_t>(ws, ly.slot_token), at<void>(ws, ly.x), at<void>(ws, ly.xp), s));
   cudaEvent_t ev_b = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_begin) : nullptr;
   cudaEvent_t ev_m = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_mid) : nullptr;
   cudaEvent_t ev_e = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_end) : nullptr;
@@ -258,16 +260,29 @@ const char* ace_status_str(ace_status s) {
 const char* ace_version(void) { return "0.1.0"; }
 
 size_t ace_tables_workspace_size(const ace_layer* layer) {
-  (void)layer;
-  return 0;
+  if (check_layer(layer, true) != ACE_OK) return 0;
+  return tables_workspace_size(*layer);
 }
 
 ace_status ace_build_tables(const ace_layer* layers, int n_layers, const ace_table_opts* opts,
                             float* a_gsp, float* a_rcr, float* amax, float* sigma, void* ws,
                             size_t ws_bytes, void* stream) {
-  (void)layers; (void)n_layers; (void)opts; (void)a_gsp; (void)a_rcr; (void)amax; (void)sigma;
-  (void)ws; (void)ws_bytes; (void)stream;
-  return ACE_ERR_UNSUPPORTED;
+  if (!layers || n_layers <= 0 || !opts) return ACE_ERR_INVALID_ARG;
+  if (!a_gsp || !a_rcr || !amax) return ACE_ERR_INVALID_ARG;
+  if (opts->gsp_norm != ACE_GSP_FRO && opts->gsp_norm != ACE_GSP_SPECTRAL)
+    return ACE_ERR_INVALID_ARG;
+  if (opts->power_iters < 0 || !(opts->eps >= 0.f)) return ACE_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    const ace_status st = check_layer(&layers[l], true);
+    if (st != ACE_OK) return st;
+    const ace_layer& a = layers[0];
+    const ace_layer& b = layers[l];
+    if (a.d != b.d || a.E != b.E || a.m != b.m || a.dtype != b.dtype) return ACE_ERR_INVALID_ARG;
+  }
+  if (layers[0].m > 4096) return ACE_ERR_UNSUPPORTED;
+  if (!ws || !aligned(ws, 256)) return ACE_ERR_WORKSPACE;
+  return build_tables_impl(layers, n_layers, *opts, a_gsp, a_rcr, amax, sigma, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

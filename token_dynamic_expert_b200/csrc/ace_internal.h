@@ -57,6 +57,8 @@ cudaError_t launch_scatter(ace_dtype dt, int T, int k, int E, int d, const int32
                            const int32_t* base, const void* x, int32_t* slot_token,
                            int32_t* slot_rank, float* slot_gate, int32_t* slot_of, void* xp,
                            uint32_t* status, cudaStream_t s);
+cudaError_t launch_gather(ace_dtype dt, int cap, int d, const int32_t* n_kept,
+                          const int32_t* slot_token, const void* x, void* xp, cudaStream_t s);
 cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* xp, void* h,
                                  float* yslot, const int4* tiles, const int32_t* n_tiles,
                                  int max_tiles, const float* slot_gate, uint32_t* status,
@@ -64,6 +66,10 @@ cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* 
 cudaError_t launch_experts_simt(const ace_layer& L, const void* xp, void* h, float* yslot,
                                 const int4* tiles, const int32_t* n_tiles, int max_tiles,
                                 const float* slot_gate, cudaStream_t s);
+size_t tables_workspace_size(const ace_layer& L);
+ace_status build_tables_impl(const ace_layer* layers, int n_layers, const ace_table_opts& o,
+                             float* a_gsp, float* a_rcr, float* amax, float* sigma, void* ws,
+                             size_t ws_bytes, cudaStream_t s);
 cudaError_t launch_combine(ace_dtype dt, int T, int k, int d, const int32_t* slot_of,
                            const float* yslot, void* y, cudaStream_t s);
 

@@ -9,7 +9,8 @@
 //              (expert, first slot, rows <= kTileN) in expert order.
 //   k_scatter  one CTA per chunk: position of slot (t, i) of expert e =
 //              base[c][e] + popcount(bitmap[c][e] below t); writes the slot
-//              tables and copies x_t into row `pos` of the gathered matrix.
+//              tables.
+//   k_gather   copies x_t into row `pos` of the gathered matrix Xp.
 // No result depends on the order atomics resolve in.
 #include "ace_common.cuh"
 #include "ace_internal.h"
@@ -112,12 +113,7 @@ __global__ void __launch_bounds__(256) k_scatter(
     const int32_t* __restrict__ base, const T* __restrict__ x, int32_t* __restrict__ slot_token,
     int32_t* __restrict__ slot_rank, float* __restrict__ slot_gate,
     int32_t* __restrict__ slot_of, T* __restrict__ xp, int cap, uint32_t* status) {
-  __shared__ int s_pos[kChunk * kMaxK];
-  __shared__ int s_tok[kChunk * kMaxK];
-  __shared__ int s_n;
   const int c = blockIdx.x;
-  if (threadIdx.x == 0) s_n = 0;
-  __syncthreads();
   for (int s = threadIdx.x; s < kChunk * k; s += blockDim.x) {
     const int tl = s / k, i = s - tl * k;
     const int t = c * kChunk + tl;
@@ -138,23 +134,26 @@ __global__ void __launch_bounds__(256) k_scatter(
           slot_token[pos] = t;
           slot_rank[pos] = i;
           slot_gate[pos] = gate[o];
-          const int j = atomicAdd(&s_n, 1);
-          s_pos[j] = pos;
-          s_tok[j] = t;
         }
       }
     }
     slot_of[o] = pos;
   }
-  __syncthreads();
-  const int n = s_n;
-  const int vpr = d * (int)sizeof(T) / 16;  // 16-byte vectors per row
-  for (int q = threadIdx.x; q < n * vpr; q += blockDim.x) {
-    const int j = q / vpr, v = q - j * vpr;
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)s_tok[j] * d);
-    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)s_pos[j] * d);
-    dst[v] = src[v];
-  }
+}
+
+// Xp[pos] = x[slot_token[pos]] for pos < n_kept: 4 rows per CTA, 16-byte
+// vectors.  Launched over the worst-case slot count; CTAs past n_kept exit.
+template <typename T>
+__global__ void __launch_bounds__(256) k_gather(int d, const int32_t* __restrict__ n_kept,
+                                                const int32_t* __restrict__ slot_token,
+                                                const T* __restrict__ x, T* __restrict__ xp) {
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 6);
+  if (row >= *n_kept) return;
+  const int t = slot_token[row];
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+  uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)row * d);
+  const int vpr = d * (int)sizeof(T) / 16;
+  for (int v = threadIdx.x & 63; v < vpr; v += 64) dst[v] = src[v];
 }
 
 cudaError_t launch_scatter(ace_dtype dt, int T, int k, int E, int d, const int32_t* idx,
@@ -172,6 +171,17 @@ cudaError_t launch_scatter(ace_dtype dt, int T, int k, int E, int d, const int32
     k_scatter<float><<<grid, 256, 0, s>>>(T, k, E, d, idx, gate, keep, bitmap, base,
                                           (const float*)x, slot_token, slot_rank, slot_gate,
                                           slot_of, (float*)xp, cap, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(ace_dtype dt, int cap, int d, const int32_t* n_kept,
+                          const int32_t* slot_token, const void* x, void* xp, cudaStream_t s) {
+  dim3 grid(cdiv(cap, 4));
+  if (dt == ACE_BF16)
+    k_gather<__nv_bfloat16><<<grid, 256, 0, s>>>(d, n_kept, slot_token, (const __nv_bfloat16*)x,
+                                                 (__nv_bfloat16*)xp);
+  else
+    k_gather<float><<<grid, 256, 0, s>>>(d, n_kept, slot_token, (const float*)x, (float*)xp);
   return cudaGetLastError();
 }
 

@@ -6,28 +6,36 @@
 //   MODE 0:  H = SiLU(Xp W^gate_e) (.) (Xp W^up_e)      -> bf16 [S][m]
 //   MODE 1:  Yslot = g * (H W^down_e)                   -> fp32 [S][d]
 //
-// Operand roles are swapped ("swap-AB"): the weight rows sit on the MMA's M
-// side (128 rows per tile, the tensor-core M) and the expert's kept slots on
-// N (16..256, rounded up to a multiple of 16), because an expert typically
-// receives tens of slots while its weight matrix has hundreds of rows.  The
-// accumulator lives in tensor memory: TMEM lane = weight row, column = slot.
+// Operand roles are swapped ("swap-AB"): weight rows sit on the MMA's M side
+// (128, the tensor-core M) and the expert's kept slots on N (16..256, rounded
+// up to a multiple of 16), because an expert receives tens of slots while its
+// weight matrices have hundreds of rows.  The accumulator lives in tensor
+// memory: TMEM lane = weight row, column = slot.
 //
-// One persistent CTA per SM, 6 warps:
-//   warp 0      TMA producer: weight tile(s) 128 x 64 and the slot tile
-//               (32-row boxes, only as many as the tile's slots need) per
-//               stage, 128-byte swizzle, mbarrier transaction counts.
+// MODE 0 stacks 64 rows of W^gate and the same 64 rows of W^up into one
+// 128-row A tile, so a work item covers 64 intermediate columns: lanes 0-63
+// accumulate the gate pre-activations, lanes 64-127 the up projections.  The
+// epilogue pairs them through a small shared-memory exchange.  Work items are
+// (tile, 64-column block) in MODE 0 and (tile, 128-row block of W^down) in
+// MODE 1, dealt round-robin to one persistent CTA per SM; the small items
+// keep the last wave short.
+//
+// Warp roles (6 warps):
+//   warp 0      TMA producer: weight rows (128 x 64 bf16 per stage) and the
+//               tile's slot rows (32-row boxes, only as many as it needs),
+//               128-byte swizzle, mbarrier transaction counts.
 //   warp 1      TMEM allocator and MMA issuer (one thread): 4 MMAs of K=16
-//               per 64-wide stage; tcgen05.commit frees the stage and, after
-//               the last stage of a work item, signals the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld of 16 columns at a time, SiLU(.)*up or
-//               gate scaling, stores to global memory.
-// Work items are (tile, 128-row block of the weight) pairs, dealt round-robin.
-// MODE 0 keeps two accumulators (gate, up) of up to 256 columns each; MODE 1
-// double-buffers one accumulator so the epilogue overlaps the next item.
-// Every mbarrier wait is bounded in time; a wait that runs out raises
-// ACE_FLAG_TIMEOUT, the CTA drains what it issued and exits.
+//               per stage; tcgen05.commit frees the stage and, after the last
+//               stage of an item, hands the accumulator to the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld 16 columns at a time, SiLU(.)*up or
+//               gate scaling, global stores.
+// Two TMEM accumulators of 256 columns alternate between items, so the
+// epilogue of one item overlaps the main loop of the next.  The stage count
+// adapts to the largest slot tile of the launch (more stages when tiles are
+// small, to keep more weight bytes in flight).  Every mbarrier wait is bounded
+// in time; a wait that runs out raises ACE_FLAG_TIMEOUT, the CTA drains what
+// it issued and exits.
 #include <math.h>
-#include <stdio.h>
 
 #include "ace_common.cuh"
 #include "ace_internal.h"
@@ -35,34 +43,17 @@
 namespace ace {
 namespace {
 
-constexpr int kBM = 128;                   // weight rows per work item (UMMA M)
-constexpr int kBK = 64;                    // K per stage: one 128-B swizzle row of bf16
-constexpr int kBoxN = 32;                  // slot rows per B TMA box
-constexpr int kAStage = kBM * kBK * 2;     // 16 KB
-constexpr int kBStage = kTileN * kBK * 2;  // 32 KB
-constexpr int kBoxBytes = kBoxN * kBK * 2; // 4 KB
+constexpr int kBM = 128;                    // MMA M (weight rows per A tile)
+constexpr int kBK = 64;                     // K per stage: one 128-B swizzle row of bf16
+constexpr int kBoxN = 32;                   // slot rows per B TMA box
+constexpr int kAStage = kBM * kBK * 2;      // 16 KB
+constexpr int kBoxBytes = kBoxN * kBK * 2;  // 4 KB
+constexpr int kMaxStages = 8;
+constexpr int kStageBudget = 200 * 1024;
+constexpr int kXchgBytes = 2 * 2 * 64 * 8 * 4;  // 2 buffers x (gate, up) x 64 rows x 8 floats
 constexpr int kThreads = 192;
-
-template <int MODE>
-struct Cfg;
-template <>
-struct Cfg<0> {
-  static constexpr int NA = 2;      // A operands per stage (gate, up)
-  static constexpr int NS = 3;      // pipeline stages
-  static constexpr int NACC = 1;    // accumulator buffers
-};
-template <>
-struct Cfg<1> {
-  static constexpr int NA = 1;
-  static constexpr int NS = 4;
-  static constexpr int NACC = 2;
-};
-constexpr uint32_t kTmemCols = 512;
-
-template <int MODE>
-constexpr int smem_bytes() {
-  return 1024 /*alignment slack*/ + Cfg<MODE>::NS * (Cfg<MODE>::NA * kAStage + kBStage) + 256;
-}
+constexpr uint32_t kTmemCols = 512;         // two accumulators of 256 columns
+constexpr int kSmemBytes = 1024 + kStageBudget + kXchgBytes + 512;
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_ns();
@@ -73,28 +64,30 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
 
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
 
+__device__ __forceinline__ void epilogue_bar() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     k_experts(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
               const __grid_constant__ CUtensorMap tmB, const int4* __restrict__ tiles,
               const int32_t* __restrict__ n_tiles_ptr, int max_tiles, int rows_per_expert,
-              int K, int mtiles, void* __restrict__ out, int out_ld,
+              int K, int items_per_tile, void* __restrict__ out, int out_ld,
               const float* __restrict__ slot_gate, uint32_t* status) {
-  using C = Cfg<MODE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sA0 = smem;
-  uint8_t* sA1 = smem + C::NS * kAStage;  // MODE 0 only
-  uint8_t* sB = smem + C::NS * C::NA * kAStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + C::NS * kBStage);
+  float* xchg = reinterpret_cast<float*>(smem + kStageBudget);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStageBudget + kXchgBytes);
   uint64_t* full = bars;
-  uint64_t* empty = bars + C::NS;
-  uint64_t* tfull = bars + 2 * C::NS;
+  uint64_t* empty = bars + kMaxStages;
+  uint64_t* tfull = bars + 2 * kMaxStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* s_maxn = reinterpret_cast<int*>(tmem_holder + 2);
 
   const int warp = (int)warp_id(), lane = (int)lane_id();
   int n_tiles = *n_tiles_ptr;
@@ -102,12 +95,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) raise_flag(status, ACE_FLAG_BAD_INDEX);
     n_tiles = n_tiles < 0 ? 0 : max_tiles;
   }
-  const int total = n_tiles * mtiles;
+  const int total = n_tiles * items_per_tile;
   if ((int)blockIdx.x >= total) return;  // uniform across the CTA: no work, no TMEM
   const int ksteps = K / kBK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NS; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -117,6 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
+    *s_maxn = 1;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -131,6 +125,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // largest slot tile of the launch -> stage size and count
+  {
+    int mx = 1;
+    for (int i = threadIdx.x; i < n_tiles; i += blockDim.x) mx = max(mx, tiles[i].z);
+    atomicMax(s_maxn, mx);
+  }
+  __syncthreads();
+  const int maxbox = (min(*s_maxn, kTileN) + kBoxN - 1) / kBoxN;
+  const int stage_bytes = kAStage + maxbox * kBoxBytes;
+  int NS = kStageBudget / stage_bytes;
+  NS = NS > kMaxStages ? kMaxStages : NS;
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
@@ -141,30 +146,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
       for (int w = blockIdx.x; w < total && !*abort_flag; w += gridDim.x) {
-        const int ti = w / mtiles, mt = w - ti * mtiles;
+        const int ti = w / items_per_tile, it = w - ti * items_per_tile;
         const int4 tl = tiles[ti];
         const int nbox = (tl.z + kBoxN - 1) / kBoxN;
-        const uint32_t bytes = C::NA * kAStage + nbox * kBoxBytes;
-        const int arow = tl.x * rows_per_expert + mt * kBM;
+        const uint32_t bytes = kAStage + nbox * kBoxBytes;
         for (int kb = 0; kb < ksteps; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, status, abort_flag)) break;
+          uint8_t* sa = smem + stage * stage_bytes;
+          uint8_t* sb = sa + kAStage;
           mbar_expect_tx(&full[stage], bytes);
-          tma_load_2d(sA0 + stage * kAStage, &tmA0, kb * kBK, arow, &full[stage], pol_w);
-          if (MODE == 0)
-            tma_load_2d(sA1 + stage * kAStage, &tmA1, kb * kBK, arow, &full[stage], pol_w);
+          if (MODE == 0) {  // 64 gate rows over 64 up rows of the same columns
+            const int r = tl.x * rows_per_expert + it * 64;
+            tma_load_2d(sa, &tmA0, kb * kBK, r, &full[stage], pol_w);
+            tma_load_2d(sa + kAStage / 2, &tmA1, kb * kBK, r, &full[stage], pol_w);
+          } else {
+            tma_load_2d(sa, &tmA0, kb * kBK, tl.x * rows_per_expert + it * kBM, &full[stage],
+                        pol_w);
+          }
           for (int b = 0; b < nbox; ++b)
-            tma_load_2d(sB + stage * kBStage + b * kBoxBytes, &tmB, kb * kBK, tl.y + b * kBoxN,
-                        &full[stage], pol_x);
+            tma_load_2d(sb + b * kBoxBytes, &tmB, kb * kBK, tl.y + b * kBoxN, &full[stage], pol_x);
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == C::NS) {
+          if (++stage == NS) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
       if (*abort_flag) {  // let every copy this thread started land before exiting
-        for (int s = 0; s < C::NS; ++s)
+        for (int s = 0; s < NS; ++s)
           if ((issued >> s) & 1u) mbar_wait_drain(&full[s], (issued_par >> s) & 1u);
       }
     }
@@ -175,42 +185,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-        const int4 tl = tiles[w / mtiles];
+        const int4 tl = tiles[w / items_per_tile];
         const int npad = (tl.z + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(kBM, npad);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, status, abort_flag)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem + (MODE == 1 ? (uint32_t)acc * 256u : 0u);
+        const uint32_t d0 = tmem + (uint32_t)acc * 256u;
         for (int kb = 0; kb < ksteps; ++kb) {
           if (!mbar_wait(&full[stage], phase, status, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA0 + stage * kAStage);
-          const uint32_t a1 = smem_u32(sA1 + stage * kAStage);
-          const uint32_t b = smem_u32(sB + stage * kBStage);
+          const uint32_t a0 = smem_u32(smem + stage * stage_bytes);
+          const uint32_t b0 = a0 + kAStage;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint32_t accum = (kb | kk) != 0;
-            const uint64_t db = sw128_kmajor_desc(b + kk * 32);
-            mma_bf16(d0, sw128_kmajor_desc(a0 + kk * 32), db, idesc, accum);
-            if (MODE == 0) mma_bf16(tmem + 256u, sw128_kmajor_desc(a1 + kk * 32), db, idesc, accum);
-          }
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_bf16(d0, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc,
+                     (kb | kk) != 0);
           mma_commit(&empty[stage]);
-          if (++stage == C::NS) {
+          if (++stage == NS) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
         mma_commit(&tfull[acc]);
-        if (C::NACC == 2) {
-          acc ^= 1;
-          if (acc == 0) acc_phase ^= 1u;
-        } else {
-          acc_phase ^= 1u;
-        }
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
       }
       // wait for every MMA this thread issued before TMEM is released
       mma_commit(drain);
@@ -219,48 +221,64 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may read
-    const int row = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
+    int xb = 0;  // exchange buffer parity (MODE 0)
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
-      const int ti = w / mtiles, mt = w - ti * mtiles;
+      const int ti = w / items_per_tile, it = w - ti * items_per_tile;
       const int4 tl = tiles[ti];
       const int row0 = tl.y, n = tl.z;
       if (!mbar_wait(&tfull[acc], acc_phase, status, abort_flag)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (MODE == 1 ? (uint32_t)acc * 256u : 0u);
-      const int col = mt * kBM + row;
-      for (int c0 = 0; c0 < n; c0 += 16) {
-        float g[16];
-        tmem_ld16(tbase + (uint32_t)c0, g);
-        if (MODE == 0) {
-          float u[16];
-          tmem_ld16(tbase + 256u + (uint32_t)c0, u);
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * 256u;
+      if (MODE == 0) {
+        const bool is_gate = q < 2;
+        const int r = (q & 1) * 32 + lane;  // intermediate row within the 64-block
+        const int col = it * 64 + r;
+        __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(out);
+        for (int c0 = 0; c0 < n; c0 += 16) {
+          float v[16];
+          tmem_ld16(tbase + (uint32_t)c0, v);
           tmem_ld_wait();
-          __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(out);
+          float* xg = xchg + xb * 1024;  // gate values of columns 8..15
+          float* xu = xg + 512;          // up values of columns 0..7
+          float4* mine = reinterpret_cast<float4*>((is_gate ? xg : xu) + r * 8);
+          const int off = is_gate ? 8 : 0;
+          mine[0] = make_float4(v[off + 0], v[off + 1], v[off + 2], v[off + 3]);
+          mine[1] = make_float4(v[off + 4], v[off + 5], v[off + 6], v[off + 7]);
+          epilogue_bar();
+          const float4* other = reinterpret_cast<const float4*>((is_gate ? xu : xg) + r * 8);
+          const float4 o0 = other[0], o1 = other[1];
+          const float ov[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+          const int base = is_gate ? c0 : c0 + 8;
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            if (c0 + c < n)
-              H[(size_t)(row0 + c0 + c) * out_ld + col] = __float2bfloat16_rn(silu(g[c]) * u[c]);
-        } else {
+          for (int c = 0; c < 8; ++c) {
+            const float g = is_gate ? v[c] : ov[c];
+            const float u = is_gate ? ov[c] : v[8 + c];
+            if (base + c < n)
+              H[(size_t)(row0 + base + c) * out_ld + col] = __float2bfloat16_rn(silu(g) * u);
+          }
+          xb ^= 1;
+        }
+      } else {
+        const int col = it * kBM + q * 32 + lane;
+        float* Y = reinterpret_cast<float*>(out);
+        for (int c0 = 0; c0 < n; c0 += 16) {
+          float v[16];
+          tmem_ld16(tbase + (uint32_t)c0, v);
           tmem_ld_wait();
-          float* Y = reinterpret_cast<float*>(out);
 #pragma unroll
           for (int c = 0; c < 16; ++c)
             if (c0 + c < n) {
               const int slot = row0 + c0 + c;
-              Y[(size_t)slot * out_ld + col] = slot_gate[slot] * g[c];
+              Y[(size_t)slot * out_ld + col] = slot_gate[slot] * v[c];
             }
         }
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
-      if (C::NACC == 2) {
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-      } else {
-        acc_phase ^= 1u;
-      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
     }
   }
   __syncthreads();
@@ -305,11 +323,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 template <int MODE>
 cudaError_t set_smem_attr() {
-  static int done = -1;  // per process; the attribute is per function and device-agnostic here
-  if (done == 1) return cudaSuccess;
+  static bool done = false;
+  if (done) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(k_experts<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       smem_bytes<MODE>());
-  if (e == cudaSuccess) done = 1;
+                                       kSmemBytes);
+  if (e == cudaSuccess) done = true;
   return e;
 }
 
@@ -321,7 +339,7 @@ cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* 
                                  int num_sms, cudaStream_t s, cudaEvent_t ev_mid) {
   CUtensorMap mg, mu, mx, md, mh;
   const uint64_t E = (uint64_t)L.E, d = (uint64_t)L.d, m = (uint64_t)L.m;
-  if (!make_map(&mg, L.w_gate, E * m, d, kBM) || !make_map(&mu, L.w_up, E * m, d, kBM) ||
+  if (!make_map(&mg, L.w_gate, E * m, d, 64) || !make_map(&mu, L.w_up, E * m, d, 64) ||
       !make_map(&mx, xp, (uint64_t)cap_slots, d, kBoxN) ||
       !make_map(&md, L.w_down, E * d, m, kBM) || !make_map(&mh, h, (uint64_t)cap_slots, m, kBoxN))
     return cudaErrorInvalidValue;
@@ -329,14 +347,12 @@ cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* 
   if ((e = set_smem_attr<0>()) != cudaSuccess) return e;
   if ((e = set_smem_attr<1>()) != cudaSuccess) return e;
   const int grid = num_sms;
-  k_experts<0><<<grid, kThreads, smem_bytes<0>(), s>>>(mg, mu, mx, tiles, n_tiles, max_tiles,
-                                                      L.m, L.d, L.m / kBM, h, L.m, slot_gate,
-                                                      status);
+  k_experts<0><<<grid, kThreads, kSmemBytes, s>>>(mg, mu, mx, tiles, n_tiles, max_tiles, L.m, L.d,
+                                                 L.m / 64, h, L.m, slot_gate, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
-  k_experts<1><<<grid, kThreads, smem_bytes<1>(), s>>>(md, md, mh, tiles, n_tiles, max_tiles,
-                                                      L.d, L.m, L.d / kBM, yslot, L.d, slot_gate,
-                                                      status);
+  k_experts<1><<<grid, kThreads, kSmemBytes, s>>>(md, md, mh, tiles, n_tiles, max_tiles, L.d, L.m,
+                                                 L.d / kBM, yslot, L.d, slot_gate, status);
   return cudaGetLastError();
 }
 

@@ -20,24 +20,40 @@
 namespace ace {
 
 // ------------------------------------------------------------------ RMSNorm
+// One warp per token, 16-byte loads and stores (d is a multiple of 64).
 template <typename T>
 __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn, int d,
                                                  const float* __restrict__ gamma, float eps,
                                                  float* __restrict__ inv_rms, T* __restrict__ x) {
+  constexpr int V = 16 / sizeof(T);
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= Tn) return;
-  const T* ur = u + (size_t)t * d;
+  const uint4* ur = reinterpret_cast<const uint4*>(u + (size_t)t * d);
+  const int nv = d / V;
   float ss = 0.f;
-  for (int i = lane; i < d; i += 32) {
-    const float v = to_f(ur[i]);
-    ss = fmaf(v, v, ss);
+  for (int v = lane; v < nv; v += 32) {
+    const uint4 q = ur[v];
+    const T* e = reinterpret_cast<const T*>(&q);
+#pragma unroll
+    for (int c = 0; c < V; ++c) {
+      const float f = to_f(e[c]);
+      ss = fmaf(f, f, ss);
+    }
   }
   ss = warp_sum(ss);
   const float r = 1.0f / sqrtf(ss / (float)d + eps);
   if (lane == 0) inv_rms[t] = r;
-  T* xr = x + (size_t)t * d;
-  for (int i = lane; i < d; i += 32) xr[i] = from_f<T>(to_f(ur[i]) * r * gamma[i]);
+  uint4* xr = reinterpret_cast<uint4*>(x + (size_t)t * d);
+  for (int v = lane; v < nv; v += 32) {
+    const uint4 q = ur[v];
+    const T* e = reinterpret_cast<const T*>(&q);
+    uint4 o;
+    T* oe = reinterpret_cast<T*>(&o);
+#pragma unroll
+    for (int c = 0; c < V; ++c) oe[c] = from_f<T>(to_f(e[c]) * r * gamma[v * V + c]);
+    xr[v] = o;
+  }
 }
 
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
@@ -136,11 +152,11 @@ cudaError_t launch_router_logits(ace_dtype dt, const void* u, const float* inv_r
 }
 
 // -------------------------------------------------------- top-k and the mask
-// One CTA per chunk of 32 tokens, one warp per token (8 warps, 4 tokens
-// each).  Lane l holds the logits of experts l, l+32, ...  Selection order is
-// (logit descending, expert index ascending); slot 0 is the top-1 expert.
+// One CTA per chunk of 32 tokens, one warp per token.  Lane l holds the
+// logits of experts l, l+32, ...  Selection order is (logit descending,
+// expert index ascending); slot 0 is the top-1 expert.
 template <int V>
-__global__ void __launch_bounds__(256) k_topk_mask(
+__global__ void __launch_bounds__(1024) k_topk_mask(
     const float* __restrict__ part, int splitk, int Tn, int E, int k,
     const float* __restrict__ bias, const float* __restrict__ amax, float tau, int renorm,
     int32_t* __restrict__ idx, float* __restrict__ gate, float* __restrict__ score,
@@ -151,10 +167,9 @@ __global__ void __launch_bounds__(256) k_topk_mask(
   for (int e = threadIdx.x; e < E; e += blockDim.x) bm[e] = 0u;
   __syncthreads();
   const int c = blockIdx.x;
-  for (int r = 0; r < kChunk / 8; ++r) {
-    const int tl = warp + 8 * r;
-    const int t = c * kChunk + tl;
-    if (t >= Tn) continue;
+  const int tl = warp;
+  const int t = c * kChunk + tl;
+  if (t < Tn) {
     float v[V];
 #pragma unroll
     for (int q = 0; q < V; ++q) {
@@ -239,7 +254,7 @@ cudaError_t launch_topk_mask(const float* part, int splitk, int T, int E, int k,
                              uint32_t* status, cudaStream_t s) {
   dim3 grid(cdiv(T, kChunk));
 #define ACE_TOPK(V)                                                                          \
-  k_topk_mask<V><<<grid, 256, 0, s>>>(part, splitk, T, E, k, bias, amax, tau, renorm, idx,    \
+  k_topk_mask<V><<<grid, kChunk * 32, 0, s>>>(part, splitk, T, E, k, bias, amax, tau, renorm, idx,    \
                                       gate, score, keep, bitmap, hist, logits_out, status)
   if (E <= 32) ACE_TOPK(1);
   else if (E <= 64) ACE_TOPK(2);
