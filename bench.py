@@ -332,6 +332,163 @@ def run_ours(args, w, rate, ws_n, rank, local):
     return out
 
 
+# ------------------------------------------------------------ decode workload
+def setup_decode(w, device, n_layers=None):
+    """48 independently seeded layers (their weights exceed L2 many times
+    over), tables for all of them from one ace_build_tables call (timed), a
+    threshold per layer from a 4096-token synthetic pool (quantile mapping),
+    and the decode tokens of every layer."""
+    from token_dynamic_expert_b200 import ace
+    nl = w.layers if n_layers is None else n_layers
+    layers = [workloads.make_layer(w, seed=1000 + l, device=device) for l in range(nl)]
+    structs = [ace.make_layer(L["gamma"], L["wr"], L["wg"], L["wu"], L["wd"], w.k,
+                              router_bias=L["bias"]) for L in layers]
+    a_gsp = torch.empty(nl, w.E, dtype=torch.float32, device=device)
+    a_rcr = torch.empty_like(a_gsp)
+    amax = torch.empty_like(a_gsp)
+    sigma = torch.empty(nl, w.E, 3, dtype=torch.float32, device=device)
+    tws = ace.alloc_workspace(ace.ace_tables_workspace_size(structs[0]), device)
+    ace.ace_build_tables(structs[:1], a_gsp[:1], a_rcr[:1], amax[:1], tws, sigma=sigma[:1])
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    ace.ace_build_tables(structs, a_gsp, a_rcr, amax, tws, sigma=sigma)
+    t1.record()
+    torch.cuda.synchronize()
+    tables_ms = t0.elapsed_time(t1)
+    code, flags = ace.ace_read_status(tws)
+    if code != ace.ACE_OK:
+        raise RuntimeError("table build status %s" % ace.ace_status_str(code))
+    del tws
+    full = [ace.make_layer(L["gamma"], L["wr"], L["wg"], L["wu"], L["wd"], w.k, amax=amax[l],
+                           router_bias=L["bias"]) for l, L in enumerate(layers)]
+    pool = max(w.pool, 1)
+    pws = ace.alloc_workspace(ace.ace_workspace_size(full[0], pool), device)
+    score = torch.empty(pool, w.k, dtype=torch.float32, device=device)
+    n_skip = int(np.floor(w.skip * pool * w.k + 0.5))
+    taus = []
+    for l in range(nl):
+        up = workloads.make_tokens(w, T=pool, token_seed=2000 + l, device=device)
+        ace.ace_moe_scores(full[l], up, score, pws)
+        t = tau_quantile_host(score.cpu().numpy(), n_skip)
+        taus.append(float(np.float32(t)))
+    del pws
+    us = [workloads.make_tokens(w, T=w.T, token_seed=5000 + l, device=device) for l in range(nl)]
+    ys = [torch.empty_like(x) for x in us]
+    ws = ace.alloc_workspace(ace.ace_workspace_size(full[0], max(w.T, 1)), device)
+    return dict(layers=layers, L=full, taus=taus, u=us, y=ys, ws=ws, amax=amax,
+                tables_ms=tables_ms, n_layers=nl)
+
+
+def run_decode(args, w, ws_n, rank, local):
+    from token_dynamic_expert_b200 import ace
+    dev = torch.device("cuda", local)
+    st = setup_decode(w, dev, n_layers=args.layers)
+    nl = st["n_layers"]
+    stream = torch.cuda.Stream(dev)
+    # kept slots and distinct experts per layer (one untimed pass)
+    touched, kept, skipped = [], [], 0
+    for l in range(nl):
+        dbg = ace.DebugOut(w.T, w.k, w.E, dev)
+        ace.ace_moe_forward(st["L"][l], st["u"][l], st["taus"][l], st["y"][l], st["ws"], dbg=dbg.c)
+        off = dbg.expert_offsets.cpu().numpy()
+        touched.append(int((np.diff(off) > 0).sum()))
+        kept.append(int(dbg.n_kept.item()))
+        skipped += int((dbg.keep == 0).sum().item())
+    code, flags = ace.ace_read_status(st["ws"])
+    if code != ace.ACE_OK:
+        raise RuntimeError("device status %s flags %#x" % (ace.ace_status_str(code), flags))
+
+    def step():
+        for l in range(nl):
+            ace.ace_moe_forward(st["L"][l], st["u"][l], st["taus"][l], st["y"][l], st["ws"],
+                                stream=stream)
+
+    # plain launches: the cooperative decode kernel replays slowly from a
+    # CUDA graph at 8 tokens (observed on B200), and at these kernel lengths
+    # launch overhead is hidden by the queue anyway
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(ws_n)
+    with ClockSampler(local) as clk, torch.cuda.stream(stream):
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        stream.synchronize()
+    barrier(ws_n)
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), ws_n)
+    ms_step = total_ms / args.steps
+    value = ws_n * args.steps * nl * w.T / (total_ms / 1e3)
+    # the decode kernel alone, per layer, events recorded by the library
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nl)]
+    with torch.cuda.stream(stream):
+        for l in range(nl):
+            ace.ace_moe_forward(st["L"][l], st["u"][l], st["taus"][l], st["y"][l], st["ws"],
+                                dbg=ace.timing_debug(*kev[l]), stream=stream)
+        stream.synchronize()
+    k_ms = sum(e[0].elapsed_time(e[2]) for e in kev)
+    pk = peaks()
+    ebytes = 3 * w.d * w.m * 2
+    surv = sum(touched) * ebytes
+    router = nl * w.E * w.d * 2
+    kernel_gbs = (surv + router) / (k_ms / 1e3) / 1e9
+    step_gbs = (surv + router) / (ms_step / 1e3) / 1e9
+    # e2e: host tokens in, host outputs back, every layer, plain API calls
+    u_host = [x.cpu().pin_memory() for x in st["u"]]
+    y_host = [torch.empty_like(x).pin_memory() for x in u_host]
+    e2e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            e2e[i][0].record(stream)
+            for l in range(nl):
+                st["u"][l].copy_(u_host[l], non_blocking=True)
+                ace.ace_moe_forward(st["L"][l], st["u"][l], st["taus"][l], st["y"][l], st["ws"],
+                                    stream=stream)
+                y_host[l].copy_(st["y"][l], non_blocking=True)
+            e2e[i][1].record(stream)
+        stream.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e), ws_n)
+    nbytes = nl * w.T * w.d * 2
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s (per MoE layer, mean of %d layers)" % nl,
+        "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) weights, N(0,1) tokens)",
+        "config": {"workload": w.name, "tokens_per_step": w.T, "layers": nl, "hidden": w.d,
+                   "experts": w.E, "expert_ffn": w.m, "top_k": w.k, "skip_rate": w.skip,
+                   "tau": "per layer, quantile of a %d-token pool" % w.pool,
+                   "realised_skip": skipped / (nl * w.T * w.k),
+                   "mean_kept_slots": float(np.mean(kept)),
+                   "mean_surviving_experts": float(np.mean(touched)),
+                   "us_per_layer": ms_step * 1e3 / nl,
+                   "parallelism": "replicas" if ws_n > 1 else "single",
+                   "launch": "%d layer forwards per step, plain launches" % nl,
+                   "l2": "weights of %d layers (%.1f GB) exceed L2; no flush" % (
+                       nl, nl * 3 * w.E * w.d * w.m * 2 / 1e9)},
+        "roofline": {"bound": "hbm", "achieved": kernel_gbs, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": kernel_gbs / pk["hbm_gbs"], "traffic": None,
+                     "kernel": "k_decode (surviving experts' weights + router)",
+                     "algorithmic_bytes": (surv + router) / nl, "kernel_ms": k_ms / nl,
+                     "peak_source": pk["source"]},
+        "kernels": {"step": {"achieved_gbs": step_gbs, "frac": step_gbs / pk["hbm_gbs"]},
+                    "tables": {"layers": nl, "experts": w.E, "ms": st["tables_ms"],
+                               "ms_per_layer": st["tables_ms"] / nl,
+                               "includes": "GSP Grams, power iteration (sigma, 200 steps), RCR"}},
+        "clocks": clk.summary(),
+        "e2e": {"value": ws_n * args.steps * nl * w.T / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+                "launch": "plain API calls, no graph"},
+        "gpu_launches": nl * args.steps,
+    }
+
+
 # ---------------------------------------------------------- CPU baselines
 def _oracle_inputs(st):
     """Host copies in the oracle's input types (converted once, untimed)."""
@@ -413,10 +570,13 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="prefill_1024",
-                    choices=["prefill_1024", "prefill_8192_e256", "sweep_4096"])
+                    choices=["prefill_1024", "prefill_8192_e256", "sweep_4096", "decode_bs1",
+                             "decode_bs8"])
     ap.add_argument("--rate", type=float, default=None, help="override the skip rate")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="decode: number of layers (default: the workload's 48)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     w = workloads.WORKLOADS[args.workload]
@@ -431,6 +591,14 @@ def main():
 
     from token_dynamic_expert_b200 import build as _b  # noqa: F401  (the .so ships prebuilt)
     ws_n, rank, local = dist_setup(args.gpus)
+    if args.workload.startswith("decode"):
+        out = run_decode(args, w, ws_n, rank, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        if ws_n > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     rates = [w.skip if args.rate is None else args.rate]
     if args.workload == "sweep_4096" and args.rate is None:
         rates = list(workloads.SWEEP_RATES)

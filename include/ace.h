@@ -124,6 +124,12 @@ typedef struct {
   void* ev_experts_begin;
   void* ev_experts_mid;
   void* ev_experts_end;
+  /* Optional trace (device, uint64 [grid][8]): the decode kernel (T <= 8)
+   * writes the %globaltimer value (ns) of each CTA at its phase boundaries:
+   * start, x ready, after the first grid barrier, after the slot list,
+   * after gate/up, after the second barrier, end, and (entry 7) after the
+   * first token's sum of squares.  NULL = off. */
+  unsigned long long* trace;
 } ace_debug_out;
 
 /* Table-build options ([ACE] "Methodology 1-2"). */
@@ -216,6 +222,11 @@ ACE_API ace_status ace_read_status(void* ws, size_t ws_bytes, uint32_t* flags,
 
 /* Human-readable name of a status code (static storage). */
 ACE_API const char* ace_status_str(ace_status s);
+
+/* Name and description of the CUDA runtime error behind the most recent
+ * ACE_ERR_CUDA returned on the calling thread ("no error" if none), static
+ * storage. */
+ACE_API const char* ace_last_cuda_error(void);
 
 /* Library version, "major.minor.patch" (static storage). */
 ACE_API const char* ace_version(void);

@@ -188,3 +188,64 @@ def test_full_prefill_8192_e256_skewed():
     res, gpu, n = _full(workloads.WORKLOADS["prefill_8192_e256"], n_out=32)
     counts = np.diff(gpu["expert_offsets"])
     assert counts.max() > 256  # skewed: some experts need several slot tiles
+
+
+# ------------------------------------------------------------------ decode
+@pytest.mark.parametrize("T", [1, 3, 8])
+def test_full_shape_decode(T):
+    """T <= 8 runs the cooperative decode kernel: Qwen3-30B-A3B layer shape,
+    every token's routing, mask, slot order and output compared."""
+    w = workloads.WORKLOADS["decode_bs8"].with_(T=T)
+    layer = workloads.make_layer(w, seed=11, device="cuda")
+    layer_cpu = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in layer.items()}
+    u_cpu = workloads.make_tokens(w, T=T, token_seed=77)
+    r = oracle.rcr(layer_cpu["gamma"], layer_cpu["wr"], layer_cpu["wg"], layer_cpu["wu"],
+                   layer_cpu["wd"])
+    A_rcr = r["A"].astype(np.float32)
+    e = np.arange(w.E)
+    A_gsp = (0.5 + (e * 7 % 11) / 10.0).astype(np.float32)
+    ref = oracle.moe_forward(layer_cpu, u_cpu, 0.0, A_gsp, A_rcr, outputs=False)
+    n = oracle.n_skip_for(T, w.k, 0.6)
+    tau = midpoint_tau(ref["c"], n)
+    gpu = run_gpu(layer_cpu, u_cpu, np.maximum(A_gsp, A_rcr), tau)
+    res = compare(layer_cpu, u_cpu, gpu, A_gsp, A_rcr, tau)
+    print("decode", T, res)
+    assert res["compared_tokens"] == T
+
+
+@pytest.mark.parametrize("tau", [-1.0, float("inf")])
+def test_decode_skip_extremes(tau):
+    w = W("dec_ext", T=8, d=256, E=32, m=128, k=8, dtype="bf16", bias=True, skip=0.5,
+          skip_of="slots")
+    layer, u, A_gsp, A_rcr, amax, _, _ = setup_case(w, tables="spread")
+    gpu = run_gpu(layer, u, amax, tau)
+    res = compare(layer, u, gpu, A_gsp, A_rcr, tau)
+    if tau < 0:
+        assert (gpu["keep"] == 1).all()
+    else:
+        assert (gpu["keep"][:, 1:] == 0).all() and (gpu["keep"][:, 0] == 1).all()
+    assert res["compared_tokens"] == 8
+
+
+def test_decode_in_a_cuda_graph():
+    """The forward (decode kernel included) captures into a CUDA graph and
+    replays to the same result."""
+    from token_dynamic_expert_b200 import ace
+    w = W("dec_graph", T=4, d=256, E=16, m=128, k=4, dtype="bf16", bias=False, skip=0.5,
+          skip_of="slots")
+    layer, u, A_gsp, A_rcr, amax, tau, _ = setup_case(w)
+    from parity_util import gpu_layer
+    g, c = gpu_layer(layer, amax)
+    ud = u.cuda()
+    y1 = torch.empty_like(ud)
+    y2 = torch.empty_like(ud)
+    ws = ace.alloc_workspace(ace.ace_workspace_size(c, w.T))
+    ace.ace_moe_forward(c, ud, tau, y1, ws)
+    s = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        ace.ace_moe_forward(c, ud, tau, y2, ws, stream=s)
+    y2.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)

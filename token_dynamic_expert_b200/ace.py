@@ -44,7 +44,7 @@ class ace_debug_out(ctypes.Structure):
     _fields_ = [("topk_idx", _vp), ("gate", _vp), ("score", _vp), ("keep", _vp),
                 ("expert_offsets", _vp), ("slot_token", _vp), ("slot_rank", _vp),
                 ("n_kept", _vp), ("logits", _vp), ("ev_experts_begin", _vp),
-                ("ev_experts_mid", _vp), ("ev_experts_end", _vp)]
+                ("ev_experts_mid", _vp), ("ev_experts_end", _vp), ("trace", _vp)]
 
 
 class ace_table_opts(ctypes.Structure):
@@ -71,12 +71,16 @@ _lib.ace_read_status.restype = ctypes.c_int
 _lib.ace_status_str.argtypes = [ctypes.c_int]
 _lib.ace_status_str.restype = ctypes.c_char_p
 _lib.ace_version.restype = ctypes.c_char_p
+_lib.ace_last_cuda_error.restype = ctypes.c_char_p
 
 
 class AceError(RuntimeError):
     def __init__(self, code, where):
         self.code = code
-        super().__init__("%s: %s" % (where, ace_status_str(code)))
+        msg = "%s: %s" % (where, ace_status_str(code))
+        if code == ACE_ERR_CUDA:
+            msg += " (%s)" % _lib.ace_last_cuda_error().decode()
+        super().__init__(msg)
 
 
 def _check(code, where):
@@ -193,7 +197,7 @@ class DebugOut:
         self.n_kept = torch.empty(1, **i32)
         self.logits = torch.empty(T, E, **f32)
         self.c = ace_debug_out(**{f: _ptr(getattr(self, f)) for f, _ in ace_debug_out._fields_
-                                  if not f.startswith("ev_")})
+                                  if not f.startswith("ev_") and f != "trace"})
 
 
 def event_handle(ev):

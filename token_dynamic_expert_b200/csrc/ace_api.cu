@@ -92,9 +92,17 @@ ace_status check_layer(const ace_layer* L, bool need_experts) {
   return ACE_OK;
 }
 
-#define ACE_CK(call)                          \
-  do {                                        \
-    if ((call) != cudaSuccess) return ACE_ERR_CUDA; \
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+ace_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = e;
+  return ACE_ERR_CUDA;
+}
+
+#define ACE_CK(call)                                \
+  do {                                              \
+    const cudaError_t ace_e_ = (call);              \
+    if (ace_e_ != cudaSuccess) return cuda_fail(ace_e_); \
   } while (0)
 
 template <typename P>
@@ -130,6 +138,47 @@ ace_status check_common(const ace_layer* layer, const void* u, int T, const ace_
   return ACE_OK;
 }
 
+// The prefill launch sequence: routing, compaction, gather, expert GEMMs,
+// combine.
+ace_status run_prefill(const ace_layer& L, const void* u, int T, const ace_fwd_opts& o, void* y,
+                       const FwdLayout& ly, void* ws, int num_sms, ace_debug_out* dbg,
+                       cudaEvent_t ev_b, cudaEvent_t ev_m, cudaEvent_t ev_e, cudaStream_t s) {
+  ace_status st = run_routing(L, u, T, o, ly, ws, num_sms, dbg ? dbg->logits : nullptr, s);
+  if (st != ACE_OK) return st;
+  const int nchunk = cdiv(T, kChunk);
+  ACE_CK(launch_scan(at<int32_t>(ws, ly.hist), nchunk, L.E, kTileN, ly.max_tiles,
+                     at<int32_t>(ws, ly.base), at<int32_t>(ws, ly.counts),
+                     at<int32_t>(ws, ly.offsets), at<int32_t>(ws, ly.n_kept),
+                     at<int4>(ws, ly.tiles), at<int32_t>(ws, ly.n_tiles), s));
+  ACE_CK(launch_scatter(L.dtype, T, L.k, L.E, L.d, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
+                        at<uint8_t>(ws, ly.keep), at<uint32_t>(ws, ly.bitmap),
+                        at<int32_t>(ws, ly.base), at<void>(ws, ly.x),
+                        at<int32_t>(ws, ly.slot_token), at<int32_t>(ws, ly.slot_rank),
+                        at<float>(ws, ly.slot_gate), at<int32_t>(ws, ly.slot_of),
+                        at<void>(ws, ly.xp), at<uint32_t>(ws, ly.status), s));
+  ACE_CK(launch_gather(L.dtype, T * L.k, L.d, at<int32_t>(ws, ly.n_kept),
+                       at<int32_t>(ws, ly.slot_token), at<void>(ws, ly.x), at<void>(ws, ly.xp), s));
+  if (ev_b) ACE_CK(cudaEventRecord(ev_b, s));
+  if (L.dtype == ACE_BF16) {
+    if (launch_experts_sm100(L, T * L.k, at<void>(ws, ly.xp), at<void>(ws, ly.h),
+                             at<float>(ws, ly.yslot), at<int4>(ws, ly.tiles),
+                             at<int32_t>(ws, ly.n_tiles), ly.max_tiles,
+                             at<float>(ws, ly.slot_gate), at<uint32_t>(ws, ly.status), num_sms,
+                             s, ev_m) != cudaSuccess)
+      return cuda_fail(cudaGetLastError());
+  } else {
+    ACE_CK(launch_experts_simt(L, at<void>(ws, ly.xp), at<void>(ws, ly.h), at<float>(ws, ly.yslot),
+                               at<int4>(ws, ly.tiles), at<int32_t>(ws, ly.n_tiles), ly.max_tiles,
+                               at<float>(ws, ly.slot_gate), s));
+    if (ev_m) ACE_CK(cudaEventRecord(ev_m, s));
+  }
+  if (ev_e) ACE_CK(cudaEventRecord(ev_e, s));
+  ACE_CK(launch_combine(L.dtype, T, L.k, L.d, at<int32_t>(ws, ly.slot_of), at<float>(ws, ly.yslot),
+                        y, s));
+  return ACE_OK;
+}
+
+
 }  // namespace
 
 extern "C" {
@@ -156,44 +205,30 @@ ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T, const a
   const FwdLayout ly = fwd_layout(L, T, num_sms);
   if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ACE_CK(cudaMemsetAsync(at<void>(ws, ly.status), 0, 4, s));
+  // status word (offset 0) and the decode kernel's grid-barrier words
+  ACE_CK(cudaMemsetAsync(at<void>(ws, ly.status), 0, 256, s));
   if (T == 0) return ACE_OK;
-
-  st = run_routing(L, u, T, *opts, ly, ws, num_sms, dbg ? dbg->logits : nullptr, s);
-  if (st != ACE_OK) return st;
-  const int nchunk = cdiv(T, kChunk);
-  ACE_CK(launch_scan(at<int32_t>(ws, ly.hist), nchunk, L.E, kTileN, ly.max_tiles,
-                     at<int32_t>(ws, ly.base), at<int32_t>(ws, ly.counts),
-                     at<int32_t>(ws, ly.offsets), at<int32_t>(ws, ly.n_kept),
-                     at<int4>(ws, ly.tiles), at<int32_t>(ws, ly.n_tiles), s));
-  ACE_CK(launch_scatter(L.dtype, T, L.k, L.E, L.d, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
-                        at<uint8_t>(ws, ly.keep), at<uint32_t>(ws, ly.bitmap),
-                        at<int32_t>(ws, ly.base), at<void>(ws, ly.x),
-                        at<int32_t>(ws, ly.slot_token), at<int32_t>(ws, ly.slot_rank),
-                        at<float>(ws, ly.slot_gate), at<int32_t>(ws, ly.slot_of),
-                        at<void>(ws, ly.xp), at<uint32_t>(ws, ly.status), s));
-  ACE_CK(launch_gather(L.dtype, T * L.k, L.d, at<int32_t>(ws, ly.n_kept),
-                       at<int32_t>(ws, ly.slot_token), at<void>(ws, ly.x), at<void>(ws, ly.xp), s));
   cudaEvent_t ev_b = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_begin) : nullptr;
   cudaEvent_t ev_m = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_mid) : nullptr;
   cudaEvent_t ev_e = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_end) : nullptr;
-  if (ev_b) ACE_CK(cudaEventRecord(ev_b, s));
-  if (L.dtype == ACE_BF16) {
-    if (launch_experts_sm100(L, T * L.k, at<void>(ws, ly.xp), at<void>(ws, ly.h),
-                             at<float>(ws, ly.yslot), at<int4>(ws, ly.tiles),
-                             at<int32_t>(ws, ly.n_tiles), ly.max_tiles,
-                             at<float>(ws, ly.slot_gate), at<uint32_t>(ws, ly.status), num_sms,
-                             s, ev_m) != cudaSuccess)
-      return ACE_ERR_CUDA;
-  } else {
-    ACE_CK(launch_experts_simt(L, at<void>(ws, ly.xp), at<void>(ws, ly.h), at<float>(ws, ly.yslot),
-                               at<int4>(ws, ly.tiles), at<int32_t>(ws, ly.n_tiles), ly.max_tiles,
-                               at<float>(ws, ly.slot_gate), s));
+
+  const bool decode = L.dtype == ACE_BF16 && T <= kDecodeMaxT && decode_fits(T, L.d, L.m, L.k, L.E, num_sms);
+  if (decode) {
+    // decode: one cooperative kernel streams the surviving experts' weights
+    if (ev_b) ACE_CK(cudaEventRecord(ev_b, s));
     if (ev_m) ACE_CK(cudaEventRecord(ev_m, s));
+    ACE_CK(launch_decode(L, u, T, opts->tau, opts->renorm_topk, opts->eps_rms, y,
+                         at<float>(ws, ly.part), at<void>(ws, ly.h), at<int32_t>(ws, ly.idx),
+                         at<float>(ws, ly.gate), at<float>(ws, ly.score), at<uint8_t>(ws, ly.keep),
+                         at<int32_t>(ws, ly.offsets), at<int32_t>(ws, ly.slot_token),
+                         at<int32_t>(ws, ly.slot_rank), at<int32_t>(ws, ly.slot_of),
+                         at<int32_t>(ws, ly.n_kept), at<uint32_t>(ws, ly.status) + 16,
+                         at<uint32_t>(ws, ly.status), dbg ? dbg->trace : nullptr, num_sms, s));
+    if (ev_e) ACE_CK(cudaEventRecord(ev_e, s));
+  } else {
+    st = run_prefill(L, u, T, *opts, y, ly, ws, num_sms, dbg, ev_b, ev_m, ev_e, s);
+    if (st != ACE_OK) return st;
   }
-  if (ev_e) ACE_CK(cudaEventRecord(ev_e, s));
-  ACE_CK(launch_combine(L.dtype, T, L.k, L.d, at<int32_t>(ws, ly.slot_of), at<float>(ws, ly.yslot),
-                        y, s));
   if (dbg) {
     const size_t tk = (size_t)T * L.k;
     auto cp = [&](void* dst, size_t off, size_t bytes) -> bool {
@@ -205,6 +240,9 @@ ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T, const a
         !cp(dbg->expert_offsets, ly.offsets, ((size_t)L.E + 1) * 4) ||
         !cp(dbg->slot_token, ly.slot_token, tk * 4) || !cp(dbg->slot_rank, ly.slot_rank, tk * 4) ||
         !cp(dbg->n_kept, ly.n_kept, 4))
+      return ACE_ERR_CUDA;
+    if (dbg->logits && decode &&
+        !cp(dbg->logits, ly.part, (size_t)T * L.E * 4))
       return ACE_ERR_CUDA;
   }
   return ACE_OK;
@@ -258,6 +296,8 @@ const char* ace_status_str(ace_status s) {
 }
 
 const char* ace_version(void) { return "0.1.0"; }
+
+const char* ace_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 size_t ace_tables_workspace_size(const ace_layer* layer) {
   if (check_layer(layer, true) != ACE_OK) return 0;

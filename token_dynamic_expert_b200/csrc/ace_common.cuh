@@ -209,6 +209,55 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- top-k
+// order-preserving map of a float to an unsigned key (larger float, larger key)
+__device__ __forceinline__ uint32_t fkey(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Warp-wide top-k of the logits held as v[q] = logit of expert lane + 32 q:
+// k rounds of (largest key by redux.max, then the smallest expert index among
+// the lanes holding it by redux.min).  Lane i < k receives rank i.
+template <int NV>
+__device__ __forceinline__ void topk_select(const float (&v)[NV], int nq, int E, int k, int lane,
+                                            int& sel_e, float& sel_v, uint32_t* status) {
+  uint32_t taken = 0u;
+  for (int i = 0; i < k; ++i) {
+    uint32_t bk = 0u;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int q = 0; q < NV; ++q) {
+      if (q >= nq) break;
+      const int e = lane + 32 * q;
+      if (e < E && !((taken >> q) & 1u)) {
+        const uint32_t kk = fkey(v[q]);
+        if (kk > bk || be == 0x7fffffff) {  // lower index wins ties: q ascends
+          bk = kk;
+          be = e;
+        }
+      }
+    }
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+    const int we = (int)__reduce_min_sync(0xffffffffu, (bk == mk) ? (uint32_t)be : 0x7fffffffu);
+    int e_sel = we;
+    if (e_sel < 0 || e_sel >= E) {
+      raise_flag(status, ACE_FLAG_BAD_INDEX);
+      e_sel = 0;
+    }
+    if ((e_sel & 31) == lane) taken |= 1u << (e_sel >> 5);
+    if (lane == i) sel_e = e_sel;
+  }
+  // the selected logits: lane i < k fetches v of expert sel_e from its owner lane
+  float mine = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < NV; ++q) {
+    const float x = __shfl_sync(0xffffffffu, v[q], sel_e & 31);
+    if ((sel_e >> 5) == q) mine = x;
+  }
+  sel_v = mine;
+}
+
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 

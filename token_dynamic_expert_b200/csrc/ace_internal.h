@@ -18,6 +18,7 @@ constexpr int kRouterBT = 64;     // router GEMM tile: tokens
 constexpr int kRouterBE = 64;     // router GEMM tile: experts
 constexpr int kRouterBK = 32;     // router GEMM K step
 constexpr int kMaxSplitK = 16;
+constexpr int kDecodeMaxT = 8;    // token counts served by the decode kernel
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -66,6 +67,14 @@ cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* 
 cudaError_t launch_experts_simt(const ace_layer& L, const void* xp, void* h, float* yslot,
                                 const int4* tiles, const int32_t* n_tiles, int max_tiles,
                                 const float* slot_gate, cudaStream_t s);
+size_t decode_smem_bytes(int T, int d, int m, int k, int E, int num_sms);
+bool decode_fits(int T, int d, int m, int k, int E, int num_sms);
+cudaError_t launch_decode(const ace_layer& L, const void* u, int T, float tau, int renorm,
+                          float eps_rms, void* y, float* logits, void* h, int32_t* idx,
+                          float* gate, float* score, uint8_t* keep, int32_t* offsets,
+                          int32_t* slot_token, int32_t* slot_rank, int32_t* slot_of,
+                          int32_t* n_kept, uint32_t* bar, uint32_t* status,
+                          unsigned long long* trace, int num_sms, cudaStream_t s);
 size_t tables_workspace_size(const ace_layer& L);
 ace_status build_tables_impl(const ace_layer* layers, int n_layers, const ace_table_opts& o,
                              float* a_gsp, float* a_rcr, float* amax, float* sigma, void* ws,

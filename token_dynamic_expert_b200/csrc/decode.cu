@@ -1,0 +1,691 @@
+// decode.cu -- the ACE MoE layer forward for a handful of tokens (T <= 8).
+//
+// At decode sizes the layer is bound by reading the weights of the experts
+// that survive skipping ([ExFold] abstract: decode is limited by the memory
+// traffic of the activated experts), so one persistent cooperative kernel
+// streams exactly those bytes once, spread over every SM:
+//   phase A  x = RMSNorm(u) * gamma into shared memory (the warp of token t
+//            normalises its row), router logits, one warp per expert spread
+//            over the CTAs (its weight row fetched before x is ready)
+//   -- grid barrier --
+//   phase B  every CTA, redundantly: top-k, gates, ACE scores and the skip
+//            mask ([ACE] "3. Conservative Fusion", top-1 always kept), the
+//            kept slots sorted by (expert, token), the distinct experts
+//   phase C  gate/up ([ACE] eq. f): the CTA's contiguous share of the
+//            surviving (expert, row) pairs streams through a shared-memory
+//            ring by TMA bulk copies issued from a producer warp; 16 warps
+//            form h = SiLU(x W^gate) (.) x W^up for the expert's kept tokens;
+//            meanwhile the W^down rows the CTA will need go to L2
+//   -- grid barrier --
+//   phase D  down + combine: the CTA's output rows of every surviving
+//            expert's W^down stream through the ring; warp w owns output row
+//            w and sums g * (h W^down) over the token's kept slots, experts
+//            in ascending order
+// The grid barrier is a generation counter in the workspace with a bounded
+// spin; the launch is cooperative so every CTA is resident.  Every mbarrier
+// wait is bounded as well.  Numerics follow the prefill path: fp32 router on
+// the unrounded x, experts on bf16(x), h rounded to bf16, fp32 sums.
+#include <math.h>
+
+#include "ace_common.cuh"
+#include "ace_internal.h"
+
+// How the W^down rows of phase D reach L2 ahead of use: 0 none, 1 plain
+// prefetches from the producer warp's idle lanes, 2 bulk prefetches queued
+// after the phase-C copies.
+#ifndef ACE_DECODE_PREFETCH
+#define ACE_DECODE_PREFETCH 1
+#endif
+
+namespace ace {
+namespace {
+
+constexpr int kCompWarps = 16;                      // compute warps
+constexpr int kDecThreads = (kCompWarps + 1) * 32;  // + one producer warp
+constexpr int kRing = 6;                            // most stages of the copy ring
+constexpr int kStageBytes = 32 * 1024;              // bytes per stage
+constexpr int kSmemBudget = 226 * 1024;             // dynamic + static shared memory
+constexpr int kMaxStageRows = 4;                    // (gate, up) row pairs per phase-C stage
+constexpr int kMaxSlots = kDecodeMaxT * kMaxK;
+// phase-C dot table: [row of the CTA's share][kept token of the row's
+// expert][gate, up], in dynamic shared memory after bf16(x)
+
+struct DecodeArgs {
+  const float* gamma;
+  const __nv_bfloat16* wr;
+  const float* bias;
+  const __nv_bfloat16* wg;
+  const __nv_bfloat16* wu;
+  const __nv_bfloat16* wd;
+  const float* amax;
+  const __nv_bfloat16* u;
+  __nv_bfloat16* y;
+  int T, d, E, m, k;
+  float tau, eps_rms;
+  int renorm;
+  float* logits;          // [T][E]
+  __nv_bfloat16* h;       // [T*k][m]
+  int32_t* idx;           // [T][k]
+  float* gate;            // [T][k]
+  float* score;           // [T][k]
+  uint8_t* keep;          // [T][k]
+  int32_t* offsets;       // [E+1]
+  int32_t* slot_token;    // [T*k]
+  int32_t* slot_rank;     // [T*k]
+  int32_t* slot_of;       // [T][k]
+  int32_t* n_kept;        // [1]
+  uint32_t* bar_count;
+  uint32_t* status;
+  unsigned long long* trace;  // optional [grid][8] phase stamps
+  int nring;                  // stages of the copy ring for this call
+  int region;                 // byte offset of the region after the ring
+  size_t dyn_bytes;           // dynamic shared memory of the launch
+};
+
+struct DecShared {
+  uint64_t full_c[kRing], empty_c[kRing], full_d[kRing], empty_d[kRing];
+  int n_slots;                 // kept slots
+  int n_uexp;                  // distinct experts among them
+  int slot_e[kMaxSlots];
+  int slot_t[kMaxSlots];
+  int slot_r[kMaxSlots];
+  float slot_g[kMaxSlots];
+  int uexp[kMaxSlots];         // distinct experts, ascending
+  int ufirst[kMaxSlots + 1];   // first slot of each distinct expert
+  int t_idx[kMaxSlots];        // per (token, rank): expert, gate, score, keep, slot
+  float t_gate[kMaxSlots];
+  float t_score[kMaxSlots];
+  int t_keep[kMaxSlots];
+  int t_pos[kMaxSlots];
+  float acc_d[kCompWarps][kDecodeMaxT];  // phase-D per-warp token sums
+  int abort;
+};
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// global -> shared bulk copy completing `bytes` of transaction on `bar`
+// (addresses 16-byte aligned, size a multiple of 16)
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void stamp(const DecodeArgs& a, int i) {
+  if (a.trace && threadIdx.x == 0) a.trace[blockIdx.x * 8 + i] = global_ns();
+}
+
+// Grid-wide barrier number `n` (1, 2, ...) over co-resident CTAs: a
+// monotonic arrival counter (zeroed before the launch); the barrier opens when
+// it reaches n * gridDim.x.  False when the bounded wait ran out
+// (ACE_FLAG_TIMEOUT raised) or an earlier wait failed.
+__device__ bool grid_barrier(const DecodeArgs& a, DecShared& sh, uint32_t n) {
+  __syncthreads();
+  if (threadIdx.x == 0 && !sh.abort) {
+    const uint32_t target = n * gridDim.x;
+    uint32_t seen;
+    asm volatile("atom.add.release.gpu.global.u32 %0, [%1], 1;" : "=r"(seen) : "l"(a.bar_count) : "memory");
+    if (seen + 1 < target) {
+      const uint64_t t0 = global_ns();
+      while (ld_acquire(a.bar_count) < target) {
+        if (global_ns() - t0 > kWaitLimitNs) {
+          raise_flag(a.status, ACE_FLAG_TIMEOUT);
+          sh.abort = 1;
+          break;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  return !sh.abort;
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const DecodeArgs& a,
+                                         DecShared& sh) {
+  return mbar_wait(bar, parity, a.status, &sh.abort);
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& q, float (&f)[8]) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 v = __bfloat1622float2(p[i]);
+    f[2 * i] = v.x;
+    f[2 * i + 1] = v.y;
+  }
+}
+
+__device__ __forceinline__ void lds8(const float* p, float (&f)[8]) {
+  const float4 a0 = reinterpret_cast<const float4*>(p)[0];
+  const float4 a1 = reinterpret_cast<const float4*>(p)[1];
+  f[0] = a0.x; f[1] = a0.y; f[2] = a0.z; f[3] = a0.w;
+  f[4] = a1.x; f[5] = a1.y; f[6] = a1.z; f[7] = a1.w;
+}
+
+__device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
+
+
+
+// NT = the call's token count.
+template <int NT>
+__global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* dsm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ DecShared sh;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = a.d, E = a.E, m = a.m, k = a.k;
+  const int G = gridDim.x;
+  const bool producer = warp == kCompWarps;
+  const int nring = a.nring;
+  uint8_t* ring = dsm;
+  float* xf = reinterpret_cast<float*>(dsm);  // phase A only, inside the ring
+  __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(dsm + a.region);  // bf16(x)
+  float* part = reinterpret_cast<float*>(dsm + a.region + (size_t)NT * a.d * 2);
+  if (threadIdx.x == 0) {
+    sh.abort = 0;
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&sh.full_c[i], 1);
+      mbar_init(&sh.empty_c[i], kCompWarps / 2);
+      mbar_init(&sh.full_d[i], 1);
+      mbar_init(&sh.empty_d[i], kCompWarps);
+    }
+    fence_barrier_init();
+  }
+  stamp(a, 0);
+
+  // ---------------------------------------------------------- phase A
+  const int n_router_warps = (E + G - 1) / G;
+  const int rwarp = kCompWarps - 1 - warp;  // router warps count down from the last
+  const int my_e = (int)blockIdx.x + G * rwarp;
+  const bool router = warp < kCompWarps && rwarp < n_router_warps && my_e < E;
+  constexpr int kRV = 8;  // 16-byte chunks per lane of a router row (d <= 2048)
+  uint4 wrq[kRV];
+  if (router) {
+    const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + (size_t)my_e * d);
+#pragma unroll
+    for (int i = 0; i < kRV; ++i) {
+      const int v = lane + 32 * i;
+      wrq[i] = v < d / 8 ? __ldg(wrow + v) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  if (warp < NT) {  // token warps: one pass, the row stays in registers
+    const int t = warp;
+    const uint4* ur = reinterpret_cast<const uint4*>(a.u + (size_t)t * d);
+    const float4* gp = reinterpret_cast<const float4*>(a.gamma);
+    constexpr int kUV = 8;  // d <= 2048
+    uint4 uq[kUV];
+#pragma unroll
+    for (int i = 0; i < kUV; ++i) {
+      const int v = lane + 32 * i;
+      uq[i] = v < d / 8 ? ur[v] : make_uint4(0, 0, 0, 0);
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < kUV; ++i) {
+      float f[8];
+      bf16x8_to_f32(uq[i], f);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) ss = fmaf(f[c], f[c], ss);
+    }
+    ss = warp_sum(ss);
+    stamp(a, 7);
+    const float r = 1.0f / sqrtf(ss / (float)d + a.eps_rms);
+#pragma unroll
+    for (int i = 0; i < kUV; ++i) {
+      const int v = lane + 32 * i;
+      if (v >= d / 8) continue;
+      float f[8];
+      bf16x8_to_f32(uq[i], f);
+      const float4 g0 = __ldg(gp + 2 * v), g1 = __ldg(gp + 2 * v + 1);
+      const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      float xv[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) xv[c] = f[c] * r * gg[c];
+      float4* xo = reinterpret_cast<float4*>(xf + t * d + v * 8);
+      xo[0] = make_float4(xv[0], xv[1], xv[2], xv[3]);
+      xo[1] = make_float4(xv[4], xv[5], xv[6], xv[7]);
+      uint4 bq;
+      __nv_bfloat16* bp = reinterpret_cast<__nv_bfloat16*>(&bq);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) bp[c] = __float2bfloat16_rn(xv[c]);
+      reinterpret_cast<uint4*>(xb + (size_t)t * d)[v] = bq;
+    }
+  }
+  __syncthreads();
+  stamp(a, 1);
+  if (router) {
+    float acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+#pragma unroll
+    for (int i = 0; i < kRV; ++i) {
+      const int v = lane + 32 * i;
+      if (v >= d / 8) continue;
+      float w[8];
+      bf16x8_to_f32(wrq[i], w);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        float xv[8];
+        lds8(xf + t * d + v * 8, xv);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[t] = fmaf(xv[c], w[c], acc[t]);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const float s = warp_sum(acc[t]);
+      if (lane == 0) a.logits[(size_t)t * E + my_e] = s + (a.bias ? a.bias[my_e] : 0.f);
+    }
+  }
+  if (!grid_barrier(a, sh, 1)) return;
+  stamp(a, 2);
+
+  // ---------------------------------------------------------- phase B
+  const int nq = (E + 31) / 32;
+  if (warp < NT) {
+    const int t = warp;
+    float v[kMaxE / 32];
+#pragma unroll
+    for (int q = 0; q < kMaxE / 32; ++q) {
+      const int e = lane + 32 * q;
+      v[q] = (q < nq && e < E) ? a.logits[(size_t)t * E + e] : -INFINITY;
+    }
+    int sel_e = 0;
+    float sel_v = -INFINITY;
+    topk_select(v, nq, E, k, lane, sel_e, sel_v, a.status);
+    const float v0 = __shfl_sync(0xffffffffu, sel_v, 0);
+    const float ex = lane < k ? expf(sel_v - v0) : 0.f;
+    float denom;
+    if (a.renorm) {
+      denom = warp_sum(ex);
+    } else {
+      float z = 0.f;
+#pragma unroll
+      for (int q = 0; q < kMaxE / 32; ++q)
+        if (q < nq) z += (lane + 32 * q < E) ? expf(v[q] - v0) : 0.f;
+      denom = warp_sum(z);
+    }
+    if (lane < k) {
+      const float g = ex / denom;
+      const float sc = g * (a.amax ? a.amax[sel_e] : 1.0f);
+      sh.t_idx[t * k + lane] = sel_e;
+      sh.t_gate[t * k + lane] = g;
+      sh.t_score[t * k + lane] = sc;
+      sh.t_keep[t * k + lane] = (lane == 0) || !(sc < a.tau);
+    }
+  }
+  __syncthreads();
+  // slot position = number of kept slots with a smaller (expert, token) key
+  const int TK = NT * k;
+  if ((int)threadIdx.x < TK) {
+    const int s = threadIdx.x;
+    int pos = -1;
+    if (sh.t_keep[s]) {
+      const int key = sh.t_idx[s] * kDecodeMaxT + s / k;
+      pos = 0;
+      for (int o = 0; o < TK; ++o)
+        pos += (sh.t_keep[o] && sh.t_idx[o] * kDecodeMaxT + o / k < key) ? 1 : 0;
+      sh.slot_e[pos] = sh.t_idx[s];
+      sh.slot_t[pos] = s / k;
+      sh.slot_r[pos] = s % k;
+      sh.slot_g[pos] = sh.t_gate[s];
+    }
+    sh.t_pos[s] = pos;
+  }
+  __syncthreads();
+  if (warp == 0) {  // slot count and distinct experts by ballots (TK <= 128)
+    int S = 0;
+    for (int b = 0; b < TK; b += 32)
+      S += __popc(__ballot_sync(0xffffffffu, b + lane < TK && sh.t_keep[b + lane]));
+    int nu = 0;
+    for (int b = 0; b < S; b += 32) {
+      const int s = b + lane;
+      const bool first = s < S && (s == 0 || sh.slot_e[s] != sh.slot_e[s - 1]);
+      const uint32_t mk = __ballot_sync(0xffffffffu, first);
+      if (first) {
+        const int at = nu + __popc(mk & ((1u << lane) - 1u));
+        sh.uexp[at] = sh.slot_e[s];
+        sh.ufirst[at] = s;
+      }
+      nu += __popc(mk);
+    }
+    if (lane == 0) {
+      sh.n_slots = S;
+      sh.n_uexp = nu;
+      sh.ufirst[nu] = S;
+    }
+  }
+  __syncthreads();
+  stamp(a, 3);
+  const int S = sh.n_slots, U = sh.n_uexp;
+
+  // ---------------------------------------------------------- phase C
+  const int rows_per_cta = (d + G - 1) / G;  // phase-D output rows per CTA (<= 16)
+  const int i0 = min(d, (int)blockIdx.x * rows_per_cta), i1 = min(d, i0 + rows_per_cta);
+  const int P = U * m;  // surviving (expert, row) pairs
+  const int p0 = (int)(((long long)P * blockIdx.x) / G);
+  const int p1 = (int)(((long long)P * (blockIdx.x + 1)) / G);
+  const int SR = max(1, min(kMaxStageRows, kStageBytes / (4 * d)));  // row pairs per stage
+  const int nstage_c = (p1 - p0 + SR - 1) / SR;
+  if (producer) {
+    if (lane > 0) {
+#if ACE_DECODE_PREFETCH == 1
+      // lanes 1..31: the phase-D rows of every surviving expert into L2, by
+      // plain prefetches (bulk prefetches would queue ahead of the ring's
+      // copies in the CTA's copy engine)
+      const int lines = (i1 - i0) * m * 2 / 128;
+      for (int q = lane - 1; q < U * lines; q += 31) {
+        const int ui = q / lines, ln = q - ui * lines;
+        const char* p =
+            reinterpret_cast<const char*>(a.wd + ((size_t)sh.uexp[ui] * d + i0) * m) + ln * 128;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+      }
+#endif
+    } else {
+      for (int st = 0; st < nstage_c; ++st) {
+        const int slot = st % nring;
+        if (!wait_bar(&sh.empty_c[slot], ((st / nring) & 1) ^ 1u, a, sh)) break;
+        const int pa = p0 + st * SR, pb = min(p1, pa + SR);
+        mbar_expect_tx(&sh.full_c[slot], (uint32_t)((pb - pa) * d * 4));
+        uint8_t* sg = ring + slot * kStageBytes;
+        uint8_t* su = sg + kStageBytes / 2;
+        for (int p = pa; p < pb;) {  // runs of consecutive rows of one expert
+          const int ui = p / m, j = p - ui * m;
+          const int run = min(pb - p, m - j);
+          const size_t off = ((size_t)sh.uexp[ui] * m + j) * d;
+          bulk_g2s(sg + (size_t)(p - pa) * d * 2, a.wg + off, (uint32_t)(run * d * 2),
+                   &sh.full_c[slot]);
+          bulk_g2s(su + (size_t)(p - pa) * d * 2, a.wu + off, (uint32_t)(run * d * 2),
+                   &sh.full_c[slot]);
+          p += run;
+        }
+      }
+#if ACE_DECODE_PREFETCH == 2
+      if (i0 < i1)  // the phase-D rows, after every ring copy of this CTA
+        for (int ui = 0; ui < U; ++ui) {
+          const char* p = reinterpret_cast<const char*>(a.wd + ((size_t)sh.uexp[ui] * d + i0) * m);
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p),
+                       "r"((uint32_t)((i1 - i0) * m * 2))
+                       : "memory");
+        }
+#endif
+    }
+  } else {
+    // two groups of 8 warps take alternate stages; in a group, warp
+    // 2r + mat reduces row r of the stage against W^gate (mat 0) or W^up
+    // (mat 1) for every kept token of the row's expert.  The dots go to the
+    // CTA's table; each warp releases the stage on its own.
+    const int grp = warp >> 3, wi = warp & 7;
+    const int rpos = wi >> 1, mat = wi & 1;
+    const int nv = d / 8;
+    for (int st = grp; st < nstage_c; st += 2) {
+      const int slot = st % nring;
+      if (!wait_bar(&sh.full_c[slot], (st / nring) & 1, a, sh)) break;
+      const int pa = p0 + st * SR, nr = min(p1, pa + SR) - pa;
+      if (rpos < nr) {
+        const int p = pa + rpos;
+        const int ui = p / m;
+        const int s0 = sh.ufirst[ui], s1 = sh.ufirst[ui + 1];
+        const uint4* wrow = reinterpret_cast<const uint4*>(
+            ring + slot * kStageBytes + mat * (kStageBytes / 2) + (size_t)rpos * d * 2);
+        float* trow = part + (size_t)(p - p0) * NT * 2;
+        for (int sg = s0; sg < s1; sg += 4) {  // the expert's kept tokens, 4 at a time
+          const int nt = min(4, s1 - sg);
+          const uint4* xt[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            xt[q] = reinterpret_cast<const uint4*>(xb + (size_t)sh.slot_t[sg + min(q, nt - 1)] * d);
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          for (int c = lane; c < nv; c += 32) {
+            float w8[8];
+            bf16x8_to_f32(wrow[c], w8);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (q >= nt) break;
+              float xv[8];
+              bf16x8_to_f32(xt[q][c], xv);
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) acc[q] = fmaf(w8[cc], xv[cc], acc[q]);
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (q >= nt) break;
+            const float r = warp_sum(acc[q]);
+            if (lane == 0) trow[(sg - s0 + q) * 2 + mat] = r;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.empty_c[slot]);
+    }
+  }
+  __syncthreads();  // every (row, kept token) gate and up dot is in the table
+  for (int q = threadIdx.x; q < (p1 - p0) * NT; q += blockDim.x) {
+    const int r = q / NT, x = q - r * NT;
+    const int p = p0 + r;
+    const int ui = p / m, j = p - ui * m;
+    const int s0 = sh.ufirst[ui], s1 = sh.ufirst[ui + 1];
+    if (s0 + x < s1) {
+      const float gs = part[(size_t)q * 2], us = part[(size_t)q * 2 + 1];
+      a.h[(size_t)(s0 + x) * m + j] = __float2bfloat16_rn(silu(gs) * us);
+    }
+  }
+  stamp(a, 4);
+  if (!grid_barrier(a, sh, 2)) return;
+  stamp(a, 5);
+
+  // ---------------------------------------------------------- phase D
+  // shared memory: h of the kept slots, then a ring of stages that each hold
+  // the CTA's output rows of one surviving expert's W^down
+  const int nrows = i1 - i0;  // <= kCompWarps: output row i0 + w belongs to warp w
+  const uint32_t dbytes = (uint32_t)(nrows * m * 2);
+  const size_t hbytes = ((size_t)S * m * 2 + 1023) & ~(size_t)1023;
+  const uint32_t dstage = (dbytes + 1023u) & ~1023u;
+  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(dsm);
+  uint8_t* ring_d = dsm + hbytes;
+  const int nring_d =
+      dstage ? (int)min((size_t)kRing, (a.dyn_bytes - 1024 - hbytes) / dstage) : 1;
+  for (int q = threadIdx.x; q < S * m / 8; q += blockDim.x)
+    reinterpret_cast<uint4*>(hs)[q] = reinterpret_cast<const uint4*>(a.h)[q];
+  __syncthreads();
+  if (nrows > 0) {
+    if (producer) {
+      if (lane == 0)
+        for (int ui = 0; ui < U; ++ui) {
+          const int slot = ui % nring_d;
+          if (!wait_bar(&sh.empty_d[slot], ((ui / nring_d) & 1) ^ 1u, a, sh)) break;
+          mbar_expect_tx(&sh.full_d[slot], dbytes);
+          bulk_g2s(ring_d + (size_t)slot * dstage, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m,
+                   dbytes, &sh.full_d[slot]);
+        }
+    } else {
+      if (lane < NT) sh.acc_d[warp][lane] = 0.f;
+      __syncwarp();
+      for (int ui = 0; ui < U; ++ui) {
+        const int slot = ui % nring_d;
+        if (!wait_bar(&sh.full_d[slot], (ui / nring_d) & 1, a, sh)) break;
+        if (warp < nrows) {
+          const int s0 = sh.ufirst[ui], s1 = sh.ufirst[ui + 1];
+          const uint4* wrow =
+              reinterpret_cast<const uint4*>(ring_d + (size_t)slot * dstage + (size_t)warp * m * 2);
+          for (int sg = s0; sg < s1; sg += 4) {  // the expert's kept tokens, 4 at a time
+            const int nt = min(4, s1 - sg);
+            float dot[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int c = lane; c < m / 8; c += 32) {
+              float w8[8];
+              bf16x8_to_f32(wrow[c], w8);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                if (q >= nt) break;
+                float hv[8];
+                bf16x8_to_f32(reinterpret_cast<const uint4*>(hs + (size_t)(sg + q) * m)[c], hv);
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) dot[q] = fmaf(w8[cc], hv[cc], dot[q]);
+              }
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (q >= nt) break;
+              const float r = warp_sum(dot[q]);
+              if (lane == 0) {
+                const int t = sh.slot_t[sg + q];
+                sh.acc_d[warp][t] = fmaf(sh.slot_g[sg + q], r, sh.acc_d[warp][t]);
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty_d[slot]);
+      }
+      __syncwarp();
+      if (warp < nrows && lane < NT)
+        a.y[(size_t)lane * d + i0 + warp] = __float2bfloat16_rn(sh.acc_d[warp][lane]);
+    }
+  }
+  stamp(a, 6);
+
+  // debug / compaction outputs (CTA 0, off the critical path)
+  if (blockIdx.x == 0) {
+    if ((int)threadIdx.x < TK) {
+      const int s = threadIdx.x;
+      a.idx[s] = sh.t_idx[s];
+      a.gate[s] = sh.t_gate[s];
+      a.score[s] = sh.t_score[s];
+      a.keep[s] = (uint8_t)sh.t_keep[s];
+      a.slot_of[s] = sh.t_pos[s];
+    }
+    if ((int)threadIdx.x < S) {
+      a.slot_token[threadIdx.x] = sh.slot_t[threadIdx.x];
+      a.slot_rank[threadIdx.x] = sh.slot_r[threadIdx.x];
+    }
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+      int c = 0;  // first slot of expert >= e
+      for (int s = 0; s < S; ++s) c += sh.slot_e[s] < e;
+      a.offsets[e] = c;
+    }
+    if (threadIdx.x == 0) *a.n_kept = S;
+  }
+}
+
+template <int NT>
+cudaError_t launch_nt(cudaLaunchConfig_t& cfg, const DecodeArgs& a, size_t smem) {
+  static size_t attr_bytes = 0;  // largest dynamic shared memory enabled so far
+  if (smem > attr_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(k_decode<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_bytes = smem;
+  }
+  return cudaLaunchKernelEx(&cfg, k_decode<NT>, a);
+}
+
+}  // namespace
+
+// Dynamic shared memory: [ring of nring 32 KB stages | bf16(x) [T][d] |
+// phase-C dot table (rows of the CTA's share x T x 2 floats)].  The unrounded
+// fp32 x of phase A lives inside the ring.
+static size_t region_bytes(int T, int d, int m, int k, int E, int num_sms) {
+  const int umax = E < T * k ? E : T * k;
+  const size_t rows = ((size_t)umax * m + num_sms - 1) / num_sms + 1;
+  return (size_t)T * d * 2 + rows * T * 2 * 4;
+}
+
+static int ring_stages(int T, int d, int m, int k, int E, int num_sms) {
+  const size_t avail = (size_t)kSmemBudget - sizeof(DecShared) - 1024 -
+                       region_bytes(T, d, m, k, E, num_sms);
+  int n = (int)(avail / kStageBytes);
+  return n > kRing ? kRing : n;
+}
+
+size_t decode_smem_bytes(int T, int d, int m, int k, int E, int num_sms) {
+  return 1024 + (size_t)ring_stages(T, d, m, k, E, num_sms) * kStageBytes +
+         region_bytes(T, d, m, k, E, num_sms);
+}
+
+bool decode_fits(int T, int d, int m, int k, int E, int num_sms) {
+  if (T < 1 || T > kDecodeMaxT || d > 2048 || d % 32 != 0 || m % 8 != 0) return false;
+  const int n = ring_stages(T, d, m, k, E, num_sms);
+  if (n < 3) return false;
+  if ((size_t)T * d * 4 > (size_t)n * kStageBytes) return false;  // the unrounded x
+  const int rows = (d + num_sms - 1) / num_sms;                    // phase-D rows per CTA
+  if (rows > kCompWarps) return false;
+  // phase D: h of every kept slot plus at least two stages of W^down rows
+  const size_t hbytes = ((size_t)T * k * m * 2 + 1023) & ~(size_t)1023;
+  const size_t dstage = ((size_t)rows * m * 2 + 1023) & ~(size_t)1023;
+  return decode_smem_bytes(T, d, m, k, E, num_sms) >= 1024 + hbytes + 2 * dstage;
+}
+
+cudaError_t launch_decode(const ace_layer& L, const void* u, int T, float tau, int renorm,
+                          float eps_rms, void* y, float* logits, void* h, int32_t* idx,
+                          float* gate, float* score, uint8_t* keep, int32_t* offsets,
+                          int32_t* slot_token, int32_t* slot_rank, int32_t* slot_of,
+                          int32_t* n_kept, uint32_t* bar, uint32_t* status,
+                          unsigned long long* trace, int num_sms, cudaStream_t s) {
+  DecodeArgs a;
+  a.gamma = L.gamma;
+  a.wr = (const __nv_bfloat16*)L.w_router;
+  a.bias = L.router_bias;
+  a.wg = (const __nv_bfloat16*)L.w_gate;
+  a.wu = (const __nv_bfloat16*)L.w_up;
+  a.wd = (const __nv_bfloat16*)L.w_down;
+  a.amax = L.amax;
+  a.u = (const __nv_bfloat16*)u;
+  a.y = (__nv_bfloat16*)y;
+  a.T = T;
+  a.d = L.d;
+  a.E = L.E;
+  a.m = L.m;
+  a.k = L.k;
+  a.tau = tau;
+  a.eps_rms = eps_rms;
+  a.renorm = renorm;
+  a.logits = logits;
+  a.h = (__nv_bfloat16*)h;
+  a.idx = idx;
+  a.gate = gate;
+  a.score = score;
+  a.keep = keep;
+  a.offsets = offsets;
+  a.slot_token = slot_token;
+  a.slot_rank = slot_rank;
+  a.slot_of = slot_of;
+  a.n_kept = n_kept;
+  a.bar_count = bar;
+  a.status = status;
+  a.trace = trace;
+  a.nring = ring_stages(T, L.d, L.m, L.k, L.E, num_sms);
+  a.region = a.nring * kStageBytes;
+  const size_t smem = decode_smem_bytes(T, L.d, L.m, L.k, L.E, num_sms);
+  a.dyn_bytes = smem;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeCooperative;
+  attrs[0].val.cooperative = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  switch (T) {
+    case 1: return launch_nt<1>(cfg, a, smem);
+    case 2: return launch_nt<2>(cfg, a, smem);
+    case 3: return launch_nt<3>(cfg, a, smem);
+    case 4: return launch_nt<4>(cfg, a, smem);
+    case 5: return launch_nt<5>(cfg, a, smem);
+    case 6: return launch_nt<6>(cfg, a, smem);
+    case 7: return launch_nt<7>(cfg, a, smem);
+    case 8: return launch_nt<8>(cfg, a, smem);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ace

@@ -170,53 +170,32 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
   const int tl = warp;
   const int t = c * kChunk + tl;
   if (t < Tn) {
+    // split-K partial sums, all of a split's loads in flight together
     float v[V];
+#pragma unroll
+    for (int q = 0; q < V; ++q) v[q] = 0.f;
+#pragma unroll 4
+    for (int sp = 0; sp < splitk; ++sp) {
+      const float* pr = part + ((size_t)sp * Tn + t) * E;
+#pragma unroll
+      for (int q = 0; q < V; ++q) {
+        const int e = lane + 32 * q;
+        if (e < E) v[q] += pr[e];
+      }
+    }
 #pragma unroll
     for (int q = 0; q < V; ++q) {
       const int e = lane + 32 * q;
       if (e < E) {
-        float sum = 0.f;
-        for (int sp = 0; sp < splitk; ++sp) sum += part[((size_t)sp * Tn + t) * E + e];
-        if (bias) sum += bias[e];
-        if (logits_out) logits_out[(size_t)t * E + e] = sum;
-        v[q] = sum;
+        if (bias) v[q] += bias[e];
+        if (logits_out) logits_out[(size_t)t * E + e] = v[q];
       } else {
         v[q] = -INFINITY;
       }
     }
-    uint32_t taken = 0u;
     int my_e = 0;
     float my_v = -INFINITY;
-    for (int i = 0; i < k; ++i) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int q = 0; q < V; ++q) {
-        const int e = lane + 32 * q;
-        if (!((taken >> q) & 1u) && e < E && (v[q] > bv || (v[q] == bv && e < be))) {
-          bv = v[q];
-          be = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if (be < 0 || be >= E) {  // non-finite logits: flag and fall back to expert 0
-        raise_flag(status, ACE_FLAG_BAD_INDEX);
-        be = 0;
-      }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      if (lane == i) {
-        my_e = be;
-        my_v = bv;
-      }
-    }
+    topk_select(v, V, E, k, lane, my_e, my_v, status);
     const float v0 = __shfl_sync(0xffffffffu, my_v, 0);  // the top-1 logit is the maximum
     const float ex = (lane < k) ? expf(my_v - v0) : 0.f;
     float denom;

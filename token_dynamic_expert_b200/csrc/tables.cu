@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(1024) k_gram_stats(const float* __restrict__ G
 // (sqrt of the dominant eigenvalue, by v <- P v/||P v||, then sqrt(v^T P v));
 // q = 3, 4 -> sigma of the products Gamma W_g W^down, Gamma W_u W^down
 // (v <- G (D v)/||.||, then sqrt(||G D v||)).  sig[(e0+b)*5 + q].
-__global__ void __launch_bounds__(1024) k_power(const float* __restrict__ Gg,
+__global__ void __launch_bounds__(512) k_power(const float* __restrict__ Gg,
                                                 const float* __restrict__ Gu,
                                                 const float* __restrict__ Dm, int m, int e0,
                                                 int iters, float* __restrict__ sig) {
@@ -299,13 +299,37 @@ __global__ void __launch_bounds__(1024) k_power(const float* __restrict__ Gg,
   const float v0 = 1.0f / sqrtf((float)m);
   for (int j = threadIdx.x; j < m; j += blockDim.x) v[j] = v0;
   __syncthreads();
+  // y = P x: a warp takes two rows at a time and issues all of its 16-byte
+  // loads of both rows before the arithmetic (m is a multiple of 128)
   auto matvec = [&](const float* P, const float* x, float* y) {
-    for (int r = warp; r < m; r += nw) {
-      const float* row = P + (size_t)r * m;
-      float s = 0.f;
-      for (int c = lane; c < m; c += 32) s = fmaf(row[c], x[c], s);
-      s = warp_sum(s);
-      if (lane == 0) y[r] = s;
+    const int m4 = m / 4;
+    for (int r = 2 * warp; r < m; r += 2 * nw) {
+      const float4* r0 = reinterpret_cast<const float4*>(P + (size_t)r * m);
+      const float4* r1 = reinterpret_cast<const float4*>(P + (size_t)(r + 1) * m);
+      float s0 = 0.f, s1 = 0.f;
+      for (int base = 0; base < m4; base += 32 * 8) {
+        float4 a0[8], a1[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c = base + lane + 32 * i;
+          a0[i] = c < m4 ? __ldg(r0 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+          a1[i] = c < m4 ? __ldg(r1 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c = base + lane + 32 * i;
+          if (c >= m4) continue;
+          const float4 xv = reinterpret_cast<const float4*>(x)[c];
+          s0 = fmaf(a0[i].x, xv.x, fmaf(a0[i].y, xv.y, fmaf(a0[i].z, xv.z, fmaf(a0[i].w, xv.w, s0))));
+          s1 = fmaf(a1[i].x, xv.x, fmaf(a1[i].y, xv.y, fmaf(a1[i].z, xv.z, fmaf(a1[i].w, xv.w, s1))));
+        }
+      }
+      s0 = warp_sum(s0);
+      s1 = warp_sum(s1);
+      if (lane == 0) {
+        y[r] = s0;
+        y[r + 1] = s1;
+      }
     }
     __syncthreads();
   };
@@ -545,7 +569,7 @@ struct TabLayout {
 TabLayout tab_layout(const ace_layer& L) {
   TabLayout t{};
   const size_t d = L.d, m = L.m, E = L.E;
-  t.eb = (int)(E < 32 ? E : 32);
+  t.eb = (int)(E < 64 ? E : 64);
   const size_t eb = (size_t)t.eb;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -643,7 +667,7 @@ ace_status build_tables_impl(const ace_layer* layers, int n_layers, const ace_ta
       }
       k_gram_stats<<<nb, 1024, 0, s>>>(Gg, Gu, Dm, m, e0, stats);
       if (nq > 0)
-        k_power<<<dim3(nb, nq), 1024, 2 * m * sizeof(float), s>>>(Gg, Gu, Dm, m, e0,
+        k_power<<<dim3(nb, nq), 512, 2 * m * sizeof(float), s>>>(Gg, Gu, Dm, m, e0,
                                                                  o.power_iters, sig);
       if (cudaGetLastError() != cudaSuccess) return ACE_ERR_CUDA;
     }
