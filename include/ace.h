@@ -183,6 +183,38 @@ ACE_API ace_status ace_moe_scores(const ace_layer* layer, const void* u, int T,
                           void* stream);
 
 /* ------------------------------------------------------------------------
+ * ace_moe_decode_noalloc -- the decode forward (1 <= T <= 8 tokens, bf16
+ *   layers) for callers that cannot allocate device memory.  The paper has
+ *   no counterpart: this is a deployment variant of ace_moe_forward.
+ *   Some callers cannot call cudaMalloc: plugins inside a host framework
+ *   that owns every device allocation and gives them no allocator, or
+ *   serving loops that must not allocate once running (an allocation can
+ *   synchronise the device).  This entry point takes the inputs and outputs
+ *   from the caller (layer weights and amax table, u [T][d], y [T][d],
+ *   device pointers as for ace_moe_forward) and uses, instead of a
+ *   workspace, a scratch array of 512 KiB compiled into the library
+ *   (static device memory, present on every GPU that loads the library
+ *   until the process exits).  It allocates nothing and calls no allocating
+ *   library routine.
+ *   - The first call on a device, with that device current, looks up the
+ *     array's device address once; make that first call before any stream
+ *     capture.
+ *   - Every call shares the one array and leaves its last contents there;
+ *     each call zeroes what must start at zero.  Calls whose GPU work
+ *     overlaps (on different streams or host threads) race on the array:
+ *     serialise them.
+ *   - Shapes whose scratch exceeds the array (router logits T x E fp32,
+ *     gated intermediates T x k x m bf16, slot tables), non-bf16 layers and
+ *     shapes the decode kernel does not serve return ACE_ERR_UNSUPPORTED
+ *     before anything is launched; bad pointers return ACE_ERR_INVALID_ARG.
+ *   - Device-detected flags stay in the array (there is no workspace to
+ *     read them from); the kernel's waits are bounded as elsewhere.
+ *   Results equal ace_moe_forward's for the same inputs.
+ * ---------------------------------------------------------------------- */
+ACE_API ace_status ace_moe_decode_noalloc(const ace_layer* layer, const void* u, int T,
+                                          const ace_fwd_opts* opts, void* y, void* stream);
+
+/* ------------------------------------------------------------------------
  * ace_tables_workspace_size
  *   Bytes of workspace ace_build_tables needs for layers shaped like
  *   `layer` (d, E, m, dtype).

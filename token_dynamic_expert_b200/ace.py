@@ -61,6 +61,9 @@ _lib.ace_moe_forward.restype = ctypes.c_int
 _lib.ace_moe_scores.argtypes = [_P(ace_layer), _vp, ctypes.c_int, _P(ace_fwd_opts), _vp, _vp, _vp,
                                 ctypes.c_size_t, _vp]
 _lib.ace_moe_scores.restype = ctypes.c_int
+_lib.ace_moe_decode_noalloc.argtypes = [_P(ace_layer), _vp, ctypes.c_int, _P(ace_fwd_opts), _vp,
+                                        _vp]
+_lib.ace_moe_decode_noalloc.restype = ctypes.c_int
 _lib.ace_tables_workspace_size.argtypes = [_P(ace_layer)]
 _lib.ace_tables_workspace_size.restype = ctypes.c_size_t
 _lib.ace_build_tables.argtypes = [_P(ace_layer), ctypes.c_int, _P(ace_table_opts), _vp, _vp, _vp,
@@ -157,6 +160,17 @@ def ace_moe_scores(layer, u, score, ws, topk_idx=None, renorm=True, eps_rms=1e-6
                                _ptr(score), _ptr(topk_idx), _ptr(ws), ws.numel(), _stream(stream))
     _check(code, "ace_moe_scores")
     return score
+
+
+def ace_moe_decode_noalloc(layer, u, tau, y, renorm=True, eps_rms=1e-6, stream=None):
+    """Decode forward (1-8 tokens) with the library's fixed scratch array
+    instead of a caller workspace; see include/ace.h."""
+    opts = ace_fwd_opts(tau=float(tau), renorm_topk=int(bool(renorm)), fusion=ACE_FUSE_MAX,
+                        eps_rms=float(eps_rms))
+    code = _lib.ace_moe_decode_noalloc(ctypes.byref(layer), _ptr(u), int(u.shape[0]),
+                                       ctypes.byref(opts), _ptr(y), _stream(stream))
+    _check(code, "ace_moe_decode_noalloc")
+    return y
 
 
 def ace_tables_workspace_size(layer):
