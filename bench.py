@@ -141,12 +141,21 @@ def dist_setup(n):
 
 
 def max_over_ranks(x, ws):
+    """Largest value over the ranks (the slowest replica's time)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(ws, steps, units_per_step, rank_total_ms):
+    """Whole-job throughput of N replicas: every rank's units over the
+    slowest rank's timed region."""
+    slowest = max_over_ranks(rank_total_ms, ws)
+    return ws * steps * units_per_step / (slowest / 1e3), slowest
 
 
 def barrier(ws):
@@ -256,9 +265,8 @@ def run_ours(args, w, rate, ws_n, rank, local):
         stream.synchronize()
     barrier(ws_n)
     t_steps = [a.elapsed_time(b) for a, b in evs]
-    total_ms = max_over_ranks(sum(t_steps), ws_n)
+    value, total_ms = replica_throughput(ws_n, args.steps, w.T, sum(t_steps))
     ms_step = total_ms / args.steps
-    value = ws_n * args.steps * w.T / (total_ms / 1e3)
     code, flags = ace.ace_read_status(st["ws"], stream=stream)
     if code != ace.ACE_OK:
         raise RuntimeError("device status %s flags %#x" % (ace.ace_status_str(code), flags))
@@ -439,9 +447,9 @@ def run_decode(args, w, ws_n, rank, local):
             evs[i][1].record(stream)
         stream.synchronize()
     barrier(ws_n)
-    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), ws_n)
+    value, total_ms = replica_throughput(ws_n, args.steps, nl * w.T,
+                                         sum(a.elapsed_time(b) for a, b in evs))
     ms_step = total_ms / args.steps
-    value = ws_n * args.steps * nl * w.T / (total_ms / 1e3)
     # the decode kernel alone, per layer, events recorded by the library
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nl)]
     with torch.cuda.stream(stream):
