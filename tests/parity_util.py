@@ -112,7 +112,8 @@ def compare(layer_cpu, u_cpu, gpu, A_gsp32, A_rcr32, tau32, renorm=True, out_tok
     exact_tokens = ok & ~(mism.any(axis=1))
     # compaction: identical when every token agrees
     res = dict(ties=len(ties), band=n_band, mask_mismatch=int(mism.sum()),
-               n_kept=int(gpu["n_kept"][0]), S_ref=ref["S"])
+               n_kept=int(gpu["n_kept"][0]), S_ref=ref["S"], logit_err=float(lerr),
+               logit_scale=float(scale))
     if exact_tokens.all():
         S = ref["S"]
         assert int(gpu["n_kept"][0]) == S

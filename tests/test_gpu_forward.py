@@ -178,16 +178,25 @@ def _full(w, n_out=48, seed=0):
     return res, gpu, n
 
 
+# The tensor-core router sums exact bf16 x bf16 products of a three-term split
+# of the fp32 input in 64-wide chunks, adding chunk sums in fp32: its logits
+# must be at least as close to the fp64 definition as an fp32 dot product
+# (about 1.5e-6 of the largest logit on these shapes).
+ROUTER_TC_REL = 5e-7
+
+
 def test_full_prefill_1024():
     res, gpu, n = _full(workloads.WORKLOADS["prefill_1024"])
     assert res["mask_mismatch"] == 0
     assert abs(int((gpu["keep"] == 0).sum()) - n) <= res["band"] + res["ties"] * 8
+    assert res["logit_err"] <= ROUTER_TC_REL * res["logit_scale"], res
 
 
 def test_full_prefill_8192_e256_skewed():
     res, gpu, n = _full(workloads.WORKLOADS["prefill_8192_e256"], n_out=32)
     counts = np.diff(gpu["expert_offsets"])
     assert counts.max() > 256  # skewed: some experts need several slot tiles
+    assert res["logit_err"] <= ROUTER_TC_REL * res["logit_scale"], res
 
 
 # ------------------------------------------------------------------ decode

@@ -17,6 +17,11 @@ int device_sm_count() {
 
 static size_t esize(ace_dtype dt) { return dt == ACE_BF16 ? 2 : 4; }
 
+int router_splits_for(const ace_layer& L, int T, int num_sms) {
+  return L.dtype == ACE_BF16 ? router_tc_splits(T, L.d, L.E, num_sms)
+                             : router_splitk(T, L.d, L.E, num_sms);
+}
+
 FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms) {
   FwdLayout o;
   memset(&o, 0, sizeof(o));
@@ -24,10 +29,12 @@ FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms) {
   const size_t d = (size_t)L.d, m = (size_t)L.m, es = esize(L.dtype);
   const size_t nchunk = (T + kChunk - 1) / kChunk, cap = T * k;
   // largest split-K x tokens product over the token counts this workspace serves
+  // (the split count only changes at multiples of the router's token tile)
   size_t part = 0;
-  for (int gx = 1; gx <= cdiv((int)T, kRouterBT); ++gx) {
-    const int t = gx == cdiv((int)T, kRouterBT) ? (int)T : gx * kRouterBT;
-    const size_t p = (size_t)router_splitk(t, L.d, L.E, num_sms) * (size_t)t * E;
+  const int rbt = L.dtype == ACE_BF16 ? 128 : kRouterBT;
+  for (int gx = 1; gx <= cdiv((int)T, rbt); ++gx) {
+    const int t = gx == cdiv((int)T, rbt) ? (int)T : gx * rbt;
+    const size_t p = (size_t)router_splits_for(L, t, num_sms) * (size_t)t * E;
     if (p > part) part = p;
   }
   o.max_tokens = (int)T;
@@ -43,6 +50,7 @@ FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms) {
   o.part = take(part * 4);
   o.inv_rms = take(T * 4);
   o.x = take(T * d * es);
+  o.xs3 = take(L.dtype == ACE_BF16 ? T * 3 * d * 2 : 0);
   o.idx = take(cap * 4);
   o.gate = take(cap * 4);
   o.score = take(cap * 4);
@@ -114,11 +122,16 @@ P* at(void* ws, size_t off) {
 ace_status run_routing(const ace_layer& L, const void* u, int T, const ace_fwd_opts& o,
                        const FwdLayout& ly, void* ws, int num_sms, float* logits_dbg,
                        cudaStream_t s) {
-  const int splitk = router_splitk(T, L.d, L.E, num_sms);
+  const int splitk = router_splits_for(L, T, num_sms);
+  const bool tc = L.dtype == ACE_BF16;
   ACE_CK(launch_rmsnorm(L.dtype, u, T, L.d, L.gamma, o.eps_rms, at<float>(ws, ly.inv_rms),
-                        at<void>(ws, ly.x), s));
-  ACE_CK(launch_router_logits(L.dtype, u, at<float>(ws, ly.inv_rms), L.gamma, L.w_router, T, L.d,
-                              L.E, splitk, at<float>(ws, ly.part), s));
+                        at<void>(ws, ly.x), tc ? at<void>(ws, ly.xs3) : nullptr, s));
+  if (tc)
+    ACE_CK(launch_router_tc(at<void>(ws, ly.xs3), L.w_router, T, L.d, L.E, splitk,
+                            at<float>(ws, ly.part), at<uint32_t>(ws, ly.status), num_sms, s));
+  else
+    ACE_CK(launch_router_logits(L.dtype, u, at<float>(ws, ly.inv_rms), L.gamma, L.w_router, T,
+                                L.d, L.E, splitk, at<float>(ws, ly.part), s));
   ACE_CK(launch_topk_mask(at<float>(ws, ly.part), splitk, T, L.E, L.k, L.router_bias, L.amax,
                           o.tau, o.renorm_topk, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
                           at<float>(ws, ly.score), at<uint8_t>(ws, ly.keep),

@@ -26,11 +26,14 @@ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 // Split of the router GEMM's K dimension for T tokens: enough CTAs to cover
 // the GPU twice, each split a multiple of the K step.
 int router_splitk(int T, int d, int E, int num_sms);
+// The K split the forward uses for this layer's router (CUDA-core router for
+// fp32 layers, tensor-core router for bf16 layers).
+int router_splits_for(const ace_layer& L, int T, int num_sms);
 
 // Byte offsets of the forward's scratch arrays inside the caller's
 // workspace.  Everything is sized for max_tokens and no skipping.
 struct FwdLayout {
-  size_t status, part, inv_rms, x, idx, gate, score, keep, bitmap, hist, base, counts,
+  size_t status, part, inv_rms, x, xs3, idx, gate, score, keep, bitmap, hist, base, counts,
       offsets, n_kept, tiles, n_tiles, slot_token, slot_rank, slot_gate, slot_of, xp, h,
       yslot, total;
   int max_tokens, part_floats, max_tiles;
@@ -41,7 +44,12 @@ int device_sm_count();
 
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
-                           float eps, float* inv_rms, void* x, cudaStream_t s);
+                           float eps, float* inv_rms, void* x, void* xs3, cudaStream_t s);
+// Tensor-core router (bf16 layers): part[split][t][e] from the three-term
+// bf16 split xs3 [T][3d] of the fp32 router input and w_router [E][d].
+int router_tc_splits(int T, int d, int E, int num_sms);
+cudaError_t launch_router_tc(const void* xs3, const void* wr, int T, int d, int E, int splits,
+                             float* part, uint32_t* status, int num_sms, cudaStream_t s);
 cudaError_t launch_router_logits(ace_dtype dt, const void* u, const float* inv_rms,
                                  const float* gamma, const void* wr, int T, int d, int E,
                                  int splitk, float* part, cudaStream_t s);

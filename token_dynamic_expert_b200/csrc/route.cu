@@ -3,6 +3,8 @@
 //   k_rmsnorm        x_t = RMSNorm(u_t) * gamma, the expert input, and 1/rms_t
 //                    ([ACE] "Theoretical Foundation": x = xbar Gamma_l)
 //   k_router_logits  l_{t,e} = x_t . w_e, fp32 CUDA-core GEMM over a K split
+//                    (fp32 layers; bf16 layers use the tensor-core router in
+//                    router_sm100.cu)
 //   k_topk_mask      per token: top-k by logit, gates, ACE scores
 //                    c = g * max(A^GSP, A^RCR), skip mask with the top-1 slot
 //                    always kept ([ACE] "3. Conservative Fusion"; [NEWS]:
@@ -21,10 +23,16 @@ namespace ace {
 
 // ------------------------------------------------------------------ RMSNorm
 // One warp per token, 16-byte loads and stores (d is a multiple of 64).
+// With xs3 given (bf16 layers), also writes the fp32 router input
+// xhat = u * (1/rms) * gamma as three bf16 terms hi + mid + lo, each the
+// rounding of what the previous terms leave, at xs3[t][0 | d | 2d + i]: the
+// operand of the tensor-core router, whose products with bf16 router rows
+// are then exact in fp32.
 template <typename T>
 __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn, int d,
                                                  const float* __restrict__ gamma, float eps,
-                                                 float* __restrict__ inv_rms, T* __restrict__ x) {
+                                                 float* __restrict__ inv_rms, T* __restrict__ x,
+                                                 __nv_bfloat16* __restrict__ xs3) {
   constexpr int V = 16 / sizeof(T);
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -50,20 +58,43 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn
     const T* e = reinterpret_cast<const T*>(&q);
     uint4 o;
     T* oe = reinterpret_cast<T*>(&o);
+    float xf[V];
 #pragma unroll
-    for (int c = 0; c < V; ++c) oe[c] = from_f<T>(to_f(e[c]) * r * gamma[v * V + c]);
+    for (int c = 0; c < V; ++c) {
+      xf[c] = to_f(e[c]) * r * gamma[v * V + c];
+      oe[c] = from_f<T>(xf[c]);
+    }
     xr[v] = o;
+    if (xs3 != nullptr && V == 8) {
+      uint4 oh, om, ol;
+      __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(&oh);
+      __nv_bfloat16* mi = reinterpret_cast<__nv_bfloat16*>(&om);
+      __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(&ol);
+#pragma unroll
+      for (int c = 0; c < V; ++c) {
+        h[c] = __float2bfloat16_rn(xf[c]);
+        const float r1 = xf[c] - __bfloat162float(h[c]);
+        mi[c] = __float2bfloat16_rn(r1);
+        lo[c] = __float2bfloat16_rn(r1 - __bfloat162float(mi[c]));
+      }
+      uint4* xs = reinterpret_cast<uint4*>(xs3 + (size_t)t * 3 * d);
+      xs[v] = oh;
+      xs[nv + v] = om;
+      xs[2 * nv + v] = ol;
+    }
   }
 }
 
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
-                           float eps, float* inv_rms, void* x, cudaStream_t s) {
+                           float eps, float* inv_rms, void* x, void* xs3, cudaStream_t s) {
   dim3 grid(cdiv(T, 8));
   if (dt == ACE_BF16)
     k_rmsnorm<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)u, T, d, gamma, eps,
-                                                  inv_rms, (__nv_bfloat16*)x);
+                                                  inv_rms, (__nv_bfloat16*)x,
+                                                  (__nv_bfloat16*)xs3);
   else
-    k_rmsnorm<float><<<grid, 256, 0, s>>>((const float*)u, T, d, gamma, eps, inv_rms, (float*)x);
+    k_rmsnorm<float><<<grid, 256, 0, s>>>((const float*)u, T, d, gamma, eps, inv_rms, (float*)x,
+                                          nullptr);
   return cudaGetLastError();
 }
 
