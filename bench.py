@@ -51,8 +51,8 @@ def profiled_traffic(workload):
     with open(os.path.join(ROOT, path), "rb") as f:
         cur = hashlib.sha1(f.read()).hexdigest()[:12]
     return nbytes if cur == sha else None
-# rmsnorm, router GEMM, top-k/mask, scan, scatter, gather, gate/up, down, combine
-KERNELS_PER_FORWARD = 9
+# rmsnorm, router GEMM, top-k/mask (+ offset scan), scatter+gather, gate/up, down, combine
+KERNELS_PER_FORWARD = 7
 
 
 # ----------------------------------------------------------------- helpers

@@ -243,6 +243,35 @@ ACE_API ace_status ace_build_tables(const ace_layer* layers, int n_layers,
                             size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * ace_tau_workspace_size -- bytes of workspace ace_tau_quantile needs
+ *   (a constant: the selection state and four 256-bin histograms).
+ * ---------------------------------------------------------------------- */
+ACE_API size_t ace_tau_workspace_size(void);
+
+/* ------------------------------------------------------------------------
+ * ace_tau_quantile -- quantile mapping of a skip budget to the threshold,
+ *   on the device ([ACE] "Efficiency Results", Table 6: the threshold for a
+ *   target skip rate is read off the score distribution of calibration
+ *   tokens).
+ *   score (device) [n_tok][k] fp32: a score pool as ace_moe_scores writes
+ *   it, column 0 the top-1 slot, which is never a candidate.  The
+ *   candidates are the other n_tok * (k - 1) scores; sorted ascending
+ *   c_(1) <= ... <= c_(N), *tau = c_(n_skip + 1), so exactly n_skip slots of
+ *   the pool satisfy c < tau when no scores tie (with ties, fewer).
+ *   n_skip <= 0 gives c_(1) (nothing skipped); n_skip >= N, or N == 0,
+ *   gives +inf (every candidate skipped).  The result is one of the pool's
+ *   values, bit for bit: an exact radix select on the order-preserving
+ *   integer keys of the floats (NaN scores order above +inf).
+ *   tau (device) receives one fp32.  ws (device, 256-byte aligned,
+ *   >= ace_tau_workspace_size() bytes) is scratch; its contents need no
+ *   initialisation.  n_tok >= 0, 1 <= k <= 16; NULL score (n_tok > 0) or
+ *   tau returns ACE_ERR_INVALID_ARG, a short or misaligned ws
+ *   ACE_ERR_WORKSPACE.  Asynchronous on `stream`; allocates nothing.
+ * ---------------------------------------------------------------------- */
+ACE_API ace_status ace_tau_quantile(const float* score, int n_tok, int k, int64_t n_skip,
+                                    float* tau, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * ace_read_status -- synchronise `stream` and return the device status
  *   word that the most recent call using `ws` left there (ACE_FLAG_* bits in
  *   *flags; every forward, scores or tables call clears it when it starts).

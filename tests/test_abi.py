@@ -119,3 +119,19 @@ def test_scores_reject_bad_calls(ace):
 
 def test_read_status_rejects_missing_workspace(ace):
     assert ace.lib().ace_read_status(None, 0, None, None) == ace.ACE_ERR_WORKSPACE
+
+
+def test_tau_quantile_rejects_bad_calls(ace):
+    f = ace.lib().ace_tau_quantile
+    n = ace.ace_tau_workspace_size()
+    assert n >= 256 + 4 * 256 * 4
+    ws, tau, sc = 0x100000, 0x200000, 0x300000  # never dereferenced: rejected first
+    assert f(sc, 4, 0, 1, tau, ws, n, None) == ace.ACE_ERR_INVALID_ARG        # k < 1
+    assert f(sc, 4, 17, 1, tau, ws, n, None) == ace.ACE_ERR_INVALID_ARG       # k > 16
+    assert f(sc, -1, 8, 1, tau, ws, n, None) == ace.ACE_ERR_INVALID_ARG       # n_tok < 0
+    assert f(None, 4, 8, 1, tau, ws, n, None) == ace.ACE_ERR_INVALID_ARG      # no scores
+    assert f(sc, 4, 8, 1, None, ws, n, None) == ace.ACE_ERR_INVALID_ARG       # no output
+    assert f(sc, 4, 8, 1, tau + 2, ws, n, None) == ace.ACE_ERR_INVALID_ARG    # misaligned
+    assert f(sc, 4, 8, 1, tau, ws, n - 1, None) == ace.ACE_ERR_WORKSPACE      # short
+    assert f(sc, 4, 8, 1, tau, ws + 16, n, None) == ace.ACE_ERR_WORKSPACE     # misaligned
+    assert f(sc, 4, 8, 1, tau, None, n, None) == ace.ACE_ERR_WORKSPACE

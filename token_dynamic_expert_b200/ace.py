@@ -69,6 +69,11 @@ _lib.ace_tables_workspace_size.restype = ctypes.c_size_t
 _lib.ace_build_tables.argtypes = [_P(ace_layer), ctypes.c_int, _P(ace_table_opts), _vp, _vp, _vp,
                                   _vp, _vp, ctypes.c_size_t, _vp]
 _lib.ace_build_tables.restype = ctypes.c_int
+_lib.ace_tau_workspace_size.argtypes = []
+_lib.ace_tau_workspace_size.restype = ctypes.c_size_t
+_lib.ace_tau_quantile.argtypes = [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp,
+                                  ctypes.c_size_t, _vp]
+_lib.ace_tau_quantile.restype = ctypes.c_int
 _lib.ace_read_status.argtypes = [_vp, ctypes.c_size_t, _P(ctypes.c_uint32), _vp]
 _lib.ace_read_status.restype = ctypes.c_int
 _lib.ace_status_str.argtypes = [ctypes.c_int]
@@ -185,6 +190,20 @@ def ace_build_tables(layers, a_gsp, a_rcr, amax, ws, sigma=None, gsp_norm=ACE_GS
     code = _lib.ace_build_tables(arr, len(layers), ctypes.byref(opts), _ptr(a_gsp), _ptr(a_rcr),
                                  _ptr(amax), _ptr(sigma), _ptr(ws), ws.numel(), _stream(stream))
     _check(code, "ace_build_tables")
+
+
+def ace_tau_workspace_size():
+    return int(_lib.ace_tau_workspace_size())
+
+
+def ace_tau_quantile(score, n_skip, tau, ws, stream=None):
+    """tau[0] = the (n_skip + 1)-th smallest non-top-1 score of the pool
+    score [n_tok][k] (device fp32); see include/ace.h."""
+    n_tok, k = score.shape
+    code = _lib.ace_tau_quantile(_ptr(score), int(n_tok), int(k), int(n_skip), _ptr(tau),
+                                 _ptr(ws), ws.numel(), _stream(stream))
+    _check(code, "ace_tau_quantile")
+    return tau
 
 
 def ace_read_status(ws, stream=None):

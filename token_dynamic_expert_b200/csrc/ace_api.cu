@@ -4,6 +4,7 @@
 
 #include "ace_common.cuh"
 #include "ace_internal.h"
+#include "compact.cuh"
 
 namespace ace {
 
@@ -49,7 +50,8 @@ FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms) {
   o.status = take(256);
   o.part = take(part * 4);
   o.inv_rms = take(T * 4);
-  o.x = take(T * d * es);
+  // bf16 layers: bf16(x) is the hi block of the router operand xs3
+  o.x = take(L.dtype == ACE_BF16 ? 0 : T * d * es);
   o.xs3 = take(L.dtype == ACE_BF16 ? T * 3 * d * 2 : 0);
   o.idx = take(cap * 4);
   o.gate = take(cap * 4);
@@ -118,25 +120,40 @@ P* at(void* ws, size_t off) {
   return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
 }
 
-// The routing half shared by the forward and the score query.
+// Word of the status block counting finished routing CTAs (zeroed per call).
+constexpr size_t kDoneCtrWord = 32;
+
+// The routing half shared by the forward and the score query; with_scan adds
+// the compaction's expert-offset scan (run by the routing's last CTA).
 ace_status run_routing(const ace_layer& L, const void* u, int T, const ace_fwd_opts& o,
                        const FwdLayout& ly, void* ws, int num_sms, float* logits_dbg,
-                       cudaStream_t s) {
+                       bool with_scan, cudaStream_t s) {
   const int splitk = router_splits_for(L, T, num_sms);
   const bool tc = L.dtype == ACE_BF16;
   ACE_CK(launch_rmsnorm(L.dtype, u, T, L.d, L.gamma, o.eps_rms, at<float>(ws, ly.inv_rms),
-                        at<void>(ws, ly.x), tc ? at<void>(ws, ly.xs3) : nullptr, s));
+                        tc ? nullptr : at<void>(ws, ly.x), tc ? at<void>(ws, ly.xs3) : nullptr,
+                        s));
   if (tc)
     ACE_CK(launch_router_tc(at<void>(ws, ly.xs3), L.w_router, T, L.d, L.E, splitk,
                             at<float>(ws, ly.part), at<uint32_t>(ws, ly.status), num_sms, s));
   else
     ACE_CK(launch_router_logits(L.dtype, u, at<float>(ws, ly.inv_rms), L.gamma, L.w_router, T,
                                 L.d, L.E, splitk, at<float>(ws, ly.part), s));
+  ScanOut so{};
+  so.base = at<int32_t>(ws, ly.base);
+  so.counts = at<int32_t>(ws, ly.counts);
+  so.offsets = at<int32_t>(ws, ly.offsets);
+  so.n_kept = at<int32_t>(ws, ly.n_kept);
+  so.tiles = at<int4>(ws, ly.tiles);
+  so.n_tiles = at<int32_t>(ws, ly.n_tiles);
+  so.max_tiles = ly.max_tiles;
+  so.tile_n = kTileN;
   ACE_CK(launch_topk_mask(at<float>(ws, ly.part), splitk, T, L.E, L.k, L.router_bias, L.amax,
                           o.tau, o.renorm_topk, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
                           at<float>(ws, ly.score), at<uint8_t>(ws, ly.keep),
                           at<uint32_t>(ws, ly.bitmap), at<int32_t>(ws, ly.hist), logits_dbg,
-                          at<uint32_t>(ws, ly.status), s));
+                          at<uint32_t>(ws, ly.status), at<uint32_t>(ws, ly.status) + kDoneCtrWord,
+                          with_scan ? &so : nullptr, s));
   return ACE_OK;
 }
 
@@ -151,26 +168,22 @@ ace_status check_common(const ace_layer* layer, const void* u, int T, const ace_
   return ACE_OK;
 }
 
-// The prefill launch sequence: routing, compaction, gather, expert GEMMs,
+// The prefill launch sequence: RMSNorm, router, top-k + mask (its last CTA
+// runs the expert-offset scan), slot tables + row gather, expert GEMMs,
 // combine.
 ace_status run_prefill(const ace_layer& L, const void* u, int T, const ace_fwd_opts& o, void* y,
                        const FwdLayout& ly, void* ws, int num_sms, ace_debug_out* dbg,
                        cudaEvent_t ev_b, cudaEvent_t ev_m, cudaEvent_t ev_e, cudaStream_t s) {
-  ace_status st = run_routing(L, u, T, o, ly, ws, num_sms, dbg ? dbg->logits : nullptr, s);
+  ace_status st =
+      run_routing(L, u, T, o, ly, ws, num_sms, dbg ? dbg->logits : nullptr, true, s);
   if (st != ACE_OK) return st;
-  const int nchunk = cdiv(T, kChunk);
-  ACE_CK(launch_scan(at<int32_t>(ws, ly.hist), nchunk, L.E, kTileN, ly.max_tiles,
-                     at<int32_t>(ws, ly.base), at<int32_t>(ws, ly.counts),
-                     at<int32_t>(ws, ly.offsets), at<int32_t>(ws, ly.n_kept),
-                     at<int4>(ws, ly.tiles), at<int32_t>(ws, ly.n_tiles), s));
-  ACE_CK(launch_scatter(L.dtype, T, L.k, L.E, L.d, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
-                        at<uint8_t>(ws, ly.keep), at<uint32_t>(ws, ly.bitmap),
-                        at<int32_t>(ws, ly.base), at<void>(ws, ly.x),
-                        at<int32_t>(ws, ly.slot_token), at<int32_t>(ws, ly.slot_rank),
-                        at<float>(ws, ly.slot_gate), at<int32_t>(ws, ly.slot_of),
-                        at<void>(ws, ly.xp), at<uint32_t>(ws, ly.status), s));
-  ACE_CK(launch_gather(L.dtype, T * L.k, L.d, at<int32_t>(ws, ly.n_kept),
-                       at<int32_t>(ws, ly.slot_token), at<void>(ws, ly.x), at<void>(ws, ly.xp), s));
+  const bool bf = L.dtype == ACE_BF16;
+  ACE_CK(launch_scatter_gather(
+      L.dtype, T, L.k, L.E, L.d, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
+      at<uint8_t>(ws, ly.keep), at<uint32_t>(ws, ly.bitmap), at<int32_t>(ws, ly.base),
+      bf ? at<void>(ws, ly.xs3) : at<void>(ws, ly.x), (size_t)L.d * (bf ? 3 : 1),
+      at<int32_t>(ws, ly.slot_token), at<int32_t>(ws, ly.slot_rank), at<float>(ws, ly.slot_gate),
+      at<int32_t>(ws, ly.slot_of), at<void>(ws, ly.xp), at<uint32_t>(ws, ly.status), s));
   if (ev_b) ACE_CK(cudaEventRecord(ev_b, s));
   if (L.dtype == ACE_BF16) {
     if (launch_experts_sm100(L, T * L.k, at<void>(ws, ly.xp), at<void>(ws, ly.h),
@@ -218,7 +231,8 @@ ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T, const a
   const FwdLayout ly = fwd_layout(L, T, num_sms);
   if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // status word (offset 0) and the decode kernel's grid-barrier words
+  // status word (offset 0), the decode kernel's grid-barrier words (byte 64)
+  // and the routing CTAs' completion count (byte 128)
   ACE_CK(cudaMemsetAsync(at<void>(ws, ly.status), 0, 256, s));
   if (T == 0) return ACE_OK;
   cudaEvent_t ev_b = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_begin) : nullptr;
@@ -272,14 +286,27 @@ ace_status ace_moe_scores(const ace_layer* layer, const void* u, int T, const ac
   const FwdLayout ly = fwd_layout(L, T, num_sms);
   if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ACE_CK(cudaMemsetAsync(at<void>(ws, ly.status), 0, 4, s));
+  ACE_CK(cudaMemsetAsync(at<void>(ws, ly.status), 0, 256, s));
   if (T == 0) return ACE_OK;
-  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, s);
+  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, false, s);
   if (st != ACE_OK) return st;
   const size_t tk = (size_t)T * L.k;
   ACE_CK(cudaMemcpyAsync(score, at<void>(ws, ly.score), tk * 4, cudaMemcpyDeviceToDevice, s));
   if (topk_idx)
     ACE_CK(cudaMemcpyAsync(topk_idx, at<void>(ws, ly.idx), tk * 4, cudaMemcpyDeviceToDevice, s));
+  return ACE_OK;
+}
+
+size_t ace_tau_workspace_size(void) { return tau_workspace_size(); }
+
+ace_status ace_tau_quantile(const float* score, int n_tok, int k, int64_t n_skip, float* tau,
+                            void* ws, size_t ws_bytes, void* stream) {
+  if (n_tok < 0 || k < 1 || k > kMaxK || !tau) return ACE_ERR_INVALID_ARG;
+  if (n_tok > 0 && !score) return ACE_ERR_INVALID_ARG;
+  if (!aligned(tau, 4) || (score && !aligned(score, 4))) return ACE_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < tau_workspace_size()) return ACE_ERR_WORKSPACE;
+  ACE_CK(launch_tau_quantile(score, n_tok, k, (long long)n_skip, tau, ws, device_sm_count(),
+                             static_cast<cudaStream_t>(stream)));
   return ACE_OK;
 }
 

@@ -53,21 +53,20 @@ cudaError_t launch_router_tc(const void* xs3, const void* wr, int T, int d, int 
 cudaError_t launch_router_logits(ace_dtype dt, const void* u, const float* inv_rms,
                                  const float* gamma, const void* wr, int T, int d, int E,
                                  int splitk, float* part, cudaStream_t s);
+struct ScanOut;
 cudaError_t launch_topk_mask(const float* part, int splitk, int T, int E, int k,
                              const float* bias, const float* amax, float tau, int renorm,
                              int32_t* idx, float* gate, float* score, uint8_t* keep,
                              uint32_t* bitmap, int32_t* hist, float* logits_out,
-                             uint32_t* status, cudaStream_t s);
-cudaError_t launch_scan(const int32_t* hist, int nchunk, int E, int tile_n, int max_tiles,
-                        int32_t* base, int32_t* counts, int32_t* offsets, int32_t* n_kept,
-                        int4* tiles, int32_t* n_tiles, cudaStream_t s);
-cudaError_t launch_scatter(ace_dtype dt, int T, int k, int E, int d, const int32_t* idx,
-                           const float* gate, const uint8_t* keep, const uint32_t* bitmap,
-                           const int32_t* base, const void* x, int32_t* slot_token,
-                           int32_t* slot_rank, float* slot_gate, int32_t* slot_of, void* xp,
-                           uint32_t* status, cudaStream_t s);
-cudaError_t launch_gather(ace_dtype dt, int cap, int d, const int32_t* n_kept,
-                          const int32_t* slot_token, const void* x, void* xp, cudaStream_t s);
+                             uint32_t* status, uint32_t* done_ctr, const ScanOut* so,
+                             cudaStream_t s);
+// Slot tables and the gathered rows Xp[pos] = x[t]; x rows are x_stride
+// elements apart.
+cudaError_t launch_scatter_gather(ace_dtype dt, int T, int k, int E, int d, const int32_t* idx,
+                                  const float* gate, const uint8_t* keep, const uint32_t* bitmap,
+                                  const int32_t* base, const void* x, size_t x_stride,
+                                  int32_t* slot_token, int32_t* slot_rank, float* slot_gate,
+                                  int32_t* slot_of, void* xp, uint32_t* status, cudaStream_t s);
 cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* xp, void* h,
                                  float* yslot, const int4* tiles, const int32_t* n_tiles,
                                  int max_tiles, const float* slot_gate, uint32_t* status,
@@ -87,6 +86,9 @@ size_t tables_workspace_size(const ace_layer& L);
 ace_status build_tables_impl(const ace_layer* layers, int n_layers, const ace_table_opts& o,
                              float* a_gsp, float* a_rcr, float* amax, float* sigma, void* ws,
                              size_t ws_bytes, cudaStream_t s);
+size_t tau_workspace_size();
+cudaError_t launch_tau_quantile(const float* score, int n_tok, int k, long long n_skip,
+                                float* tau, void* ws, int num_sms, cudaStream_t s);
 cudaError_t launch_combine(ace_dtype dt, int T, int k, int d, const int32_t* slot_of,
                            const float* yslot, void* y, cudaStream_t s);
 

@@ -1,6 +1,8 @@
 // route.cu -- the online routing half of the ACE MoE forward.
 //
 //   k_rmsnorm        x_t = RMSNorm(u_t) * gamma, the expert input, and 1/rms_t
+//                    (bf16 layers: x as three bf16 terms, the first of which
+//                    is the experts' bf16 input)
 //                    ([ACE] "Theoretical Foundation": x = xbar Gamma_l)
 //   k_router_logits  l_{t,e} = x_t . w_e, fp32 CUDA-core GEMM over a K split
 //                    (fp32 layers; bf16 layers use the tensor-core router in
@@ -18,16 +20,18 @@
 
 #include "ace_common.cuh"
 #include "ace_internal.h"
+#include "compact.cuh"
 
 namespace ace {
 
 // ------------------------------------------------------------------ RMSNorm
 // One warp per token, 16-byte loads and stores (d is a multiple of 64).
-// With xs3 given (bf16 layers), also writes the fp32 router input
+// x (nullable) receives x rounded to the storage type.  With xs3 given
+// (bf16 layers), the kernel writes the fp32 router input
 // xhat = u * (1/rms) * gamma as three bf16 terms hi + mid + lo, each the
 // rounding of what the previous terms leave, at xs3[t][0 | d | 2d + i]: the
 // operand of the tensor-core router, whose products with bf16 router rows
-// are then exact in fp32.
+// are then exact in fp32.  The hi term is bf16(x), the experts' input.
 template <typename T>
 __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn, int d,
                                                  const float* __restrict__ gamma, float eps,
@@ -64,7 +68,7 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn
       xf[c] = to_f(e[c]) * r * gamma[v * V + c];
       oe[c] = from_f<T>(xf[c]);
     }
-    xr[v] = o;
+    if (x != nullptr) xr[v] = o;
     if (xs3 != nullptr && V == 8) {
       uint4 oh, om, ol;
       __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(&oh);
@@ -192,8 +196,9 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
     const float* __restrict__ bias, const float* __restrict__ amax, float tau, int renorm,
     int32_t* __restrict__ idx, float* __restrict__ gate, float* __restrict__ score,
     uint8_t* __restrict__ keep, uint32_t* __restrict__ bitmap, int32_t* __restrict__ hist,
-    float* __restrict__ logits_out, uint32_t* status) {
+    float* __restrict__ logits_out, uint32_t* status, uint32_t* done_ctr, ScanOut so) {
   __shared__ uint32_t bm[kMaxE];
+  __shared__ int s_last;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int e = threadIdx.x; e < E; e += blockDim.x) bm[e] = 0u;
   __syncthreads();
@@ -255,17 +260,33 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
     bitmap[(size_t)c * E + e] = bm[e];
     hist[(size_t)c * E + e] = __popc(bm[e]);
   }
+  if (done_ctr == nullptr) return;
+  // the last CTA to finish runs the expert-offset scan over every chunk's
+  // histogram (each writer fences its stores before the arrival count)
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t prev;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(done_ctr) : "memory");
+    s_last = prev == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (s_last) scan_experts(hist, (int)gridDim.x, E, so);
 }
 
 cudaError_t launch_topk_mask(const float* part, int splitk, int T, int E, int k,
                              const float* bias, const float* amax, float tau, int renorm,
                              int32_t* idx, float* gate, float* score, uint8_t* keep,
                              uint32_t* bitmap, int32_t* hist, float* logits_out,
-                             uint32_t* status, cudaStream_t s) {
+                             uint32_t* status, uint32_t* done_ctr, const ScanOut* so,
+                             cudaStream_t s) {
   dim3 grid(cdiv(T, kChunk));
-#define ACE_TOPK(V)                                                                          \
-  k_topk_mask<V><<<grid, kChunk * 32, 0, s>>>(part, splitk, T, E, k, bias, amax, tau, renorm, idx,    \
-                                      gate, score, keep, bitmap, hist, logits_out, status)
+  const ScanOut sv = so ? *so : ScanOut{};
+  if (so == nullptr) done_ctr = nullptr;
+#define ACE_TOPK(V)                                                                         \
+  k_topk_mask<V><<<grid, kChunk * 32, 0, s>>>(part, splitk, T, E, k, bias, amax, tau, renorm, \
+                                              idx, gate, score, keep, bitmap, hist,           \
+                                              logits_out, status, done_ctr, sv)
   if (E <= 32) ACE_TOPK(1);
   else if (E <= 64) ACE_TOPK(2);
   else if (E <= 128) ACE_TOPK(4);
