@@ -166,15 +166,15 @@ def barrier(ws):
 
 
 # ----------------------------------------------------------- our workload
-def tau_quantile_host(score, n_skip):
-    """tau = c_(n+1) over the non-top-1 scores sorted ascending (quantile
-    mapping of the target skip count)."""
-    cand = np.sort(score[:, 1:].reshape(-1).astype(np.float64))
-    if n_skip <= 0:
-        return float(cand[0])
-    if n_skip >= cand.size:
-        return float("inf")
-    return float(cand[n_skip])
+def tau_on_device(score, n_skip, tws=None):
+    """Quantile mapping of the skip count to tau on the GPU (ace_tau_quantile);
+    returns a one-element device tensor."""
+    from token_dynamic_expert_b200 import ace
+    if tws is None:
+        tws = ace.alloc_workspace(ace.ace_tau_workspace_size(), score.device)
+    tau = torch.empty(1, dtype=torch.float32, device=score.device)
+    ace.ace_tau_quantile(score, n_skip, tau, tws)
+    return tau
 
 
 def setup_prefill(w, rate, device):
@@ -203,8 +203,7 @@ def setup_prefill(w, rate, device):
     ace.ace_moe_scores(L, u, score, ws)
     torch.cuda.synchronize()
     n_skip = int(np.floor(rate * (w.T * w.k if w.skip_of == "slots" else w.T * (w.k - 1)) + 0.5))
-    tau = tau_quantile_host(score.cpu().numpy(), n_skip)
-    tau32 = float(np.float32(tau)) if np.isfinite(tau) else float("inf")
+    tau32 = float(tau_on_device(score, n_skip).item())
     y = torch.empty_like(u)
     return dict(layer=layer, u=u, L=L, ws=ws, y=y, tau=tau32, amax=amax, tables=tables,
                 n_skip=n_skip)
@@ -392,18 +391,27 @@ def setup_decode(w, device, n_layers=None):
     pws = ace.alloc_workspace(ace.ace_workspace_size(full[0], pool), device)
     score = torch.empty(pool, w.k, dtype=torch.float32, device=device)
     n_skip = int(np.floor(w.skip * pool * w.k + 0.5))
-    taus = []
-    for l in range(nl):
-        up = workloads.make_tokens(w, T=pool, token_seed=2000 + l, device=device)
-        ace.ace_moe_scores(full[l], up, score, pws)
-        t = tau_quantile_host(score.cpu().numpy(), n_skip)
-        taus.append(float(np.float32(t)))
-    del pws
+    # threshold construction: per layer, the pool's scores and the quantile
+    # mapping of the skip count, both on the device (timed)
+    pools = [workloads.make_tokens(w, T=pool, token_seed=2000 + l, device=device)
+             for l in range(nl)]
+    tws = ace.alloc_workspace(ace.ace_tau_workspace_size(), device)
+    taus_dev = torch.empty(nl, dtype=torch.float32, device=device)
+    for rep in range(2):  # the first pass warms up; the second is timed
+        t0.record()
+        for l in range(nl):
+            ace.ace_moe_scores(full[l], pools[l], score, pws)
+            ace.ace_tau_quantile(score, n_skip, taus_dev[l:l + 1], tws)
+        t1.record()
+        torch.cuda.synchronize()
+    threshold_ms = t0.elapsed_time(t1)
+    taus = [float(t) for t in taus_dev.cpu().tolist()]
+    del pws, pools
     us = [workloads.make_tokens(w, T=w.T, token_seed=5000 + l, device=device) for l in range(nl)]
     ys = [torch.empty_like(x) for x in us]
     ws = ace.alloc_workspace(ace.ace_workspace_size(full[0], max(w.T, 1)), device)
     return dict(layers=layers, L=full, taus=taus, u=us, y=ys, ws=ws, amax=amax,
-                tables_ms=tables_ms, n_layers=nl)
+                tables_ms=tables_ms, threshold_ms=threshold_ms, n_layers=nl)
 
 
 def run_decode(args, w, ws_n, rank, local):
@@ -505,7 +513,11 @@ def run_decode(args, w, ws_n, rank, local):
         "kernels": {"step": {"achieved_gbs": step_gbs, "frac": step_gbs / pk["hbm_gbs"]},
                     "tables": {"layers": nl, "experts": w.E, "ms": st["tables_ms"],
                                "ms_per_layer": st["tables_ms"] / nl,
-                               "includes": "GSP Grams, power iteration (sigma, 200 steps), RCR"}},
+                               "includes": "GSP Grams, power iteration (sigma, 200 steps), RCR"},
+                    "thresholds": {"layers": nl, "pool_tokens": max(w.pool, 1),
+                                   "ms": st["threshold_ms"],
+                                   "includes": "per layer: ace_moe_scores over the pool, "
+                                               "ace_tau_quantile (radix select)"}},
         "clocks": clk.summary(),
         "e2e": {"value": ws_n * args.steps * nl * w.T / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
