@@ -428,21 +428,33 @@ void ora_rcr(int E, int d, int m, const double *gamma, const float *wr,
 /* expert is always retained ([ACE]; [NEWS] likewise).  "Low" is s < tau.     */
 /* Both forms are evaluated; the return value counts slots where the max rule */
 /* and the set intersection disagree (always 0 for a correct oracle).         */
+/* The pages' ablations replace the fusion rule ([ACE] "Fusion Strategy       */
+/* Ablation", Table 5: Min, Mean; "Component Ablation", Table 4: one view):   */
+/*   fusion 1  c = min(s^GSP, s^RCR), checked against the union of the sets  */
+/*   fusion 2  c = (s^GSP + s^RCR) / 2                                       */
+/*   fusion 3  c = s^GSP          fusion 4  c = s^RCR                        */
 /* ------------------------------------------------------------------------ */
 int ora_mask(int T, int k, const int *idx, const double *gate,
-             const double *A_gsp, const double *A_rcr, double tau,
+             const double *A_gsp, const double *A_rcr, double tau, int fusion,
              double *s_gsp, double *s_rcr, double *c, unsigned char *keep) {
   int disagree = 0;
   for (long s = 0; s < (long)T * k; ++s) {
     int e = idx[s];
     s_gsp[s] = gate[s] * A_gsp[e];
     s_rcr[s] = gate[s] * A_rcr[e];
-    c[s] = s_gsp[s] > s_rcr[s] ? s_gsp[s] : s_rcr[s];
+    int low_g = s_gsp[s] < tau, low_r = s_rcr[s] < tau;
+    switch (fusion) {
+      case 1: c[s] = s_gsp[s] < s_rcr[s] ? s_gsp[s] : s_rcr[s]; break;
+      case 2: c[s] = 0.5 * (s_gsp[s] + s_rcr[s]); break;
+      case 3: c[s] = s_gsp[s]; break;
+      case 4: c[s] = s_rcr[s]; break;
+      default: c[s] = s_gsp[s] > s_rcr[s] ? s_gsp[s] : s_rcr[s]; break;
+    }
     int rank = (int)(s % k);
-    int low_both = (s_gsp[s] < tau) && (s_rcr[s] < tau);
-    int skip_max = (c[s] < tau);
-    if (low_both != skip_max) ++disagree;
-    keep[s] = (unsigned char)(rank == 0 || !skip_max);
+    int skip = (c[s] < tau);
+    if (fusion == 0 && (low_g && low_r) != skip) ++disagree;
+    if (fusion == 1 && (low_g || low_r) != skip) ++disagree;
+    keep[s] = (unsigned char)(rank == 0 || !skip);
   }
   return disagree;
 }

@@ -39,7 +39,7 @@ def lib():
         L.ora_sigma_factors.argtypes = [i, i, i, _D, _F, _F, _F, i, _D]
         L.ora_gsp.argtypes = [i, i, i, _D, _F, _F, _F, i, i, d, _D, _D, _D, _D, _D]
         L.ora_rcr.argtypes = [i, i, i, _D, _F, _F, _F, _F, d, d, _D, _D, _D, _D]
-        L.ora_mask.argtypes = [i, i, _I, _D, _D, _D, d, _D, _D, _D, _U8]
+        L.ora_mask.argtypes = [i, i, _I, _D, _D, _D, d, i, _D, _D, _D, _U8]
         L.ora_mask.restype = i
         L.ora_compact.argtypes = [i, i, i, _I, _U8, _I, _I, _I, _I, _I]
         L.ora_compact.restype = i
@@ -151,7 +151,10 @@ def tables(layer, spectral=False, iters=200, rho=1.0, eps=1e-6):
     return dict(gsp=g, rcr=r, A_gsp=g["A"], A_rcr=r["A"], Amax=np.maximum(g["A"], r["A"]))
 
 
-def mask(idx, gate, A_gsp, A_rcr, tau):
+FUSIONS = {"max": 0, "min": 1, "mean": 2, "gsp": 3, "rcr": 4}
+
+
+def mask(idx, gate, A_gsp, A_rcr, tau, fusion="max"):
     idx = _np(idx, np.int32)
     gate = _np(gate, np.float64)
     A_gsp = _np(A_gsp, np.float64)
@@ -160,7 +163,8 @@ def mask(idx, gate, A_gsp, A_rcr, tau):
     s_gsp, s_rcr, c = (np.empty((T, k)) for _ in range(3))
     keep = np.empty((T, k), dtype=np.uint8)
     dis = lib().ora_mask(T, k, _p(idx, _I), _p(gate, _D), _p(A_gsp, _D), _p(A_rcr, _D),
-                         float(tau), _p(s_gsp, _D), _p(s_rcr, _D), _p(c, _D), _p(keep, _U8))
+                         float(tau), FUSIONS[fusion], _p(s_gsp, _D), _p(s_rcr, _D), _p(c, _D),
+                         _p(keep, _U8))
     return dict(s_gsp=s_gsp, s_rcr=s_rcr, c=c, keep=keep, disagree=int(dis))
 
 
@@ -218,13 +222,15 @@ def tau_quantile(c, n_skip):
     return float(cand[n_skip])
 
 
-def moe_forward(layer, u, tau, A_gsp, A_rcr, renorm=True, keep=None, eps_rms=1e-6, outputs=True):
-    """Whole layer: RMSNorm, router, top-k, scores, skip mask, compaction and
-    the gate-weighted combine of the kept slots.  ``keep`` overrides the mask
-    (to evaluate the outputs the GPU produced with its own mask)."""
+def moe_forward(layer, u, tau, A_gsp, A_rcr, renorm=True, keep=None, eps_rms=1e-6, outputs=True,
+                fusion="max"):
+    """Whole layer: RMSNorm, router, top-k, scores, skip mask (views fused by
+    ``fusion``), compaction and the gate-weighted combine of the kept slots.
+    ``keep`` overrides the mask (to evaluate the outputs the GPU produced with
+    its own mask)."""
     xbar, x = rmsnorm(u, layer["gamma"], eps_rms)
     logits, idx, gate = router(x, layer["wr"], layer.get("bias"), layer["k"], renorm)
-    mk = mask(idx, gate, A_gsp, A_rcr, tau)
+    mk = mask(idx, gate, A_gsp, A_rcr, tau, fusion)
     kp = mk["keep"] if keep is None else _np(keep, np.uint8)
     E = layer["wr"].shape[0]
     cp = compact(idx, kp, E)

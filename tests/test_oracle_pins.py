@@ -349,6 +349,42 @@ def test_mask_rules():
     assert prev_skips == T * (k - 1)                   # tau = 2 skips every non-top-1
 
 
+def test_fusion_ablation_rules():
+    """The pages' fusion ablation (Min, Mean against ACE's Max) and the single
+    views: set identities and closed forms, not the formulas retyped."""
+    rng = np.random.default_rng(16)
+    T, k, E = 300, 8, 16
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    g = np.sort(rng.dirichlet(np.ones(k), T), axis=1)[:, ::-1].copy()
+    A_gsp = rng.uniform(0.5, 1.5, E)
+    A_rcr = rng.uniform(0.5, 1.5, E)
+    low_g = g * A_gsp[idx]
+    low_r = g * A_rcr[idx]
+    for tau in [0.0, 0.05, 0.1, 0.2, 2.0]:
+        r = {f: oracle.mask(idx, g, A_gsp, A_rcr, tau, f) for f in oracle.FUSIONS}
+        sk = {f: v["keep"] == 0 for f, v in r.items()}
+        for v in r.values():
+            assert (v["keep"][:, 0] == 1).all()          # top-1 retained under every rule
+            assert v["disagree"] == 0
+        lg, lr = low_g < tau, low_r < tau
+        lg[:, 0] = lr[:, 0] = False
+        assert (sk["min"] == (lg | lr)).all()            # Min: either view low (union)
+        assert (sk["max"] == (lg & lr)).all()            # Max: both low (intersection)
+        assert (sk["gsp"] == lg).all() and (sk["rcr"] == lr).all()
+        assert not (sk["max"] & ~sk["mean"]).any()       # max-skips within mean-skips
+        assert not (sk["mean"] & ~sk["min"]).any()       # mean-skips within min-skips
+    # equal views: every rule is the same rule
+    same = {f: oracle.mask(idx, g, A_gsp, A_gsp, 0.1, f) for f in oracle.FUSIONS}
+    for f in oracle.FUSIONS:
+        assert np.array_equal(same[f]["keep"], same["max"]["keep"])
+        assert np.array_equal(same[f]["c"], same["gsp"]["c"])
+    # A^RCR = 3 A^GSP: mean = 2 s^GSP, min = s^GSP, max = s^RCR, exactly
+    m3 = {f: oracle.mask(idx, g, A_gsp, 3.0 * A_gsp, 0.1, f) for f in oracle.FUSIONS}
+    assert np.allclose(m3["mean"]["c"], 2.0 * m3["gsp"]["c"], rtol=1e-15, atol=0)
+    assert np.array_equal(m3["min"]["c"], m3["gsp"]["c"])
+    assert np.array_equal(m3["max"]["c"], m3["rcr"]["c"])
+
+
 def test_tau_quantile_skips_exactly_n():
     rng = np.random.default_rng(14)
     T, k = 100, 4
