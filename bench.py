@@ -166,6 +166,18 @@ def barrier(ws):
 
 
 # ----------------------------------------------------------- our workload
+def step_spread(t_steps, what):
+    """Median and max of the timed steps.  A step far above the median means
+    a kernel waited out its bounded wait (the status word only holds the last
+    call's flags), so the run is rejected rather than averaged."""
+    med = float(np.median(t_steps))
+    mx = float(np.max(t_steps))
+    if mx > 20.0 * med + 1.0:
+        raise RuntimeError("%s: a timed step took %.1f ms against a median of %.3f ms"
+                           % (what, mx, med))
+    return {"median_ms": med, "max_ms": mx}
+
+
 def tau_on_device(score, n_skip, tws=None):
     """Quantile mapping of the skip count to tau on the GPU (ace_tau_quantile);
     returns a one-element device tensor."""
@@ -264,6 +276,7 @@ def run_ours(args, w, rate, ws_n, rank, local):
         stream.synchronize()
     barrier(ws_n)
     t_steps = [a.elapsed_time(b) for a, b in evs]
+    spread = step_spread(t_steps, w.name)
     value, total_ms = replica_throughput(ws_n, args.steps, w.T, sum(t_steps))
     ms_step = total_ms / args.steps
     code, flags = ace.ace_read_status(st["ws"], stream=stream)
@@ -332,7 +345,7 @@ def run_ours(args, w, rate, ws_n, rank, local):
                    "skip_of": w.skip_of, "router_bias": w.bias, "tau": st["tau"],
                    "realised_skip": ss["skipped"] / (w.T * w.k), "kept_slots": S,
                    "touched_experts": touched, "tables": st["tables"],
-                   "parallelism": "replicas" if ws_n > 1 else "single",
+                   "parallelism": "replicas" if ws_n > 1 else "single", "step_ms": spread,
                    "launch": "forward captured in one CUDA graph, replayed per step",
                    "l2": "flushed before each timed step (256 MiB write), flush untimed"},
         "roofline": {"bound": "hbm", "achieved": gu_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -438,9 +451,8 @@ def run_decode(args, w, ws_n, rank, local):
             ace.ace_moe_forward(st["L"][l], st["u"][l], st["taus"][l], st["y"][l], st["ws"],
                                 stream=stream)
 
-    # plain launches: the cooperative decode kernel replays slowly from a
-    # CUDA graph at 8 tokens (observed on B200), and at these kernel lengths
-    # launch overhead is hidden by the queue anyway
+    # plain launches: at these kernel lengths the launch overhead is hidden
+    # by the queue (a CUDA graph of the 48 layers times the same)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
@@ -455,9 +467,13 @@ def run_decode(args, w, ws_n, rank, local):
             evs[i][1].record(stream)
         stream.synchronize()
     barrier(ws_n)
-    value, total_ms = replica_throughput(ws_n, args.steps, nl * w.T,
-                                         sum(a.elapsed_time(b) for a, b in evs))
+    t_steps = [a.elapsed_time(b) for a, b in evs]
+    spread = step_spread(t_steps, w.name)
+    value, total_ms = replica_throughput(ws_n, args.steps, nl * w.T, sum(t_steps))
     ms_step = total_ms / args.steps
+    code, flags = ace.ace_read_status(st["ws"], stream=stream)
+    if code != ace.ACE_OK:
+        raise RuntimeError("device status %s flags %#x" % (ace.ace_status_str(code), flags))
     # the decode kernel alone, per layer, events recorded by the library
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nl)]
     with torch.cuda.stream(stream):
@@ -501,7 +517,7 @@ def run_decode(args, w, ws_n, rank, local):
                    "mean_kept_slots": float(np.mean(kept)),
                    "mean_surviving_experts": float(np.mean(touched)),
                    "us_per_layer": ms_step * 1e3 / nl,
-                   "parallelism": "replicas" if ws_n > 1 else "single",
+                   "parallelism": "replicas" if ws_n > 1 else "single", "step_ms": spread,
                    "launch": "%d layer forwards per step, plain launches" % nl,
                    "l2": "weights of %d layers (%.1f GB) exceed L2; no flush" % (
                        nl, nl * 3 * w.E * w.d * w.m * 2 / 1e9)},

@@ -72,8 +72,22 @@ typedef enum { ACE_BF16 = 0, ACE_F32 = 1 } ace_dtype;
  * spectral norm (largest singular value, power iteration). */
 typedef enum { ACE_GSP_FRO = 0, ACE_GSP_SPECTRAL = 1 } ace_gsp_norm;
 
-/* Fusion of the two views into one score ([ACE] "3. Conservative Fusion"). */
-typedef enum { ACE_FUSE_MAX = 0 } ace_fusion;
+/* Fusion of the two views' scores s^GSP = g A^GSP(e), s^RCR = g A^RCR(e)
+ * into the score c that is compared with tau.  MAX is ACE's rule
+ * ([ACE] "3. Conservative Fusion": a slot is skipped only when both views
+ * call it low, i.e. the intersection of the two low sets).  The others are
+ * the pages' ablations: MIN (skipped when either view calls it low, the
+ * union) and MEAN (the arithmetic mean of the two scores) in the fusion
+ * ablation (Table 5), and a single view, GSP or RCR, in the component
+ * ablation (Table 4).  Gates are non-negative, so c = g F(A^GSP, A^RCR)(e)
+ * with F = max, min, mean, first or second. */
+typedef enum {
+  ACE_FUSE_MAX = 0,
+  ACE_FUSE_MIN = 1,
+  ACE_FUSE_MEAN = 2,
+  ACE_FUSE_GSP = 3,
+  ACE_FUSE_RCR = 4
+} ace_fusion;
 
 /* One MoE layer: shapes, weights (device) and its ACE table. */
 typedef struct {
@@ -88,20 +102,29 @@ typedef struct {
   const void* w_gate;      /* [E][m][d]                                    */
   const void* w_up;        /* [E][m][d]                                    */
   const void* w_down;      /* [E][d][m]                                    */
-  const float* amax;       /* [E] max(A^GSP, A^RCR) from ace_build_tables;
-                              NULL only for ace_moe_scores callers that want
-                              the raw gates (scores use 1.0 then)           */
+  const float* amax;       /* [E] max(A^GSP, A^RCR) from ace_build_tables,
+                              the table of ACE_FUSE_MAX; NULL only for
+                              callers that want the raw gates as scores
+                              (1.0 then), or that give a_gsp and a_rcr      */
+  const float* a_gsp;      /* [E] A^GSP, or NULL; needed by ACE_FUSE_MIN,
+                              _MEAN and _GSP                                */
+  const float* a_rcr;      /* [E] A^RCR, or NULL; needed by ACE_FUSE_MIN,
+                              _MEAN and _RCR                                */
 } ace_layer;
 
 /* Forward options. */
 typedef struct {
-  float tau;           /* skip threshold: slot i > 0 is skipped iff
-                          g_i * Amax[e_i] < tau ([ACE] "Conservative
+  float tau;           /* skip threshold: slot i > 0 is skipped iff its
+                          fused score c_i < tau ([ACE] "Conservative
                           Fusion"; tau comes from the caller, one per layer
                           and skip budget, [ACE] "Efficiency Results")    */
   int renorm_topk;     /* 1: gates renormalised over the top-k (the gate of
                           slot i is p_i / sum_topk p); 0: raw softmax p_i    */
-  ace_fusion fusion;   /* ACE_FUSE_MAX                                    */
+  ace_fusion fusion;   /* how c is formed (ace_fusion); MAX reads
+                          layer->amax when it is set, else
+                          max(a_gsp, a_rcr); the other rules read a_gsp
+                          and/or a_rcr and return ACE_ERR_INVALID_ARG when
+                          a table they need is NULL                       */
   float eps_rms;       /* RMSNorm epsilon (1e-6 in the shipped workloads)  */
 } ace_fwd_opts;
 
@@ -110,7 +133,7 @@ typedef struct {
 typedef struct {
   int32_t* topk_idx;       /* [T][k] expert of slot (t, i); i = 0 is top-1 */
   float* gate;             /* [T][k] gate g_{t,i}                          */
-  float* score;            /* [T][k] fused score c = g * Amax[e]           */
+  float* score;            /* [T][k] fused score c (opts->fusion)          */
   uint8_t* keep;           /* [T][k] 1 = kept, 0 = skipped                 */
   int32_t* expert_offsets; /* [E+1] first kept slot of each expert         */
   int32_t* slot_token;     /* [T*k] token of each kept slot (first n_kept)  */
@@ -156,7 +179,8 @@ ACE_API size_t ace_workspace_size(const ace_layer* layer, int max_tokens);
  *   the token's gate and scalar operations).
  *   Per token t: x_t = RMSNorm(u_t) * gamma; logits x_t . w_e (+ b_e); the
  *   top-k experts by logit (ties: lower index first); gates; scores
- *   c = g * Amax[e]; slot i is kept iff i == 0 or !(c < tau); the kept
+ *   c = g * F(A^GSP, A^RCR)(e) by opts->fusion (ACE: F = max, the table
+ *   layer->amax); slot i is kept iff i == 0 or !(c < tau); the kept
  *   slots are grouped by expert (then token), run through their SwiGLU
  *   experts, and y_t = sum over kept i, in rank order, of g_i f_{e_i}(x_t).
  *   Skipped slots drop out without re-normalising the others.
@@ -172,7 +196,8 @@ ACE_API ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T,
 
 /* ------------------------------------------------------------------------
  * ace_moe_scores -- only the routing half of the forward: fused scores
- *   c = g * Amax[e] (gate alone when layer->amax is NULL) of every slot,
+ *   c (opts->fusion; the gate alone under ACE_FUSE_MAX when layer->amax,
+ *   a_gsp and a_rcr are all NULL) of every slot,
  *   for building tau by quantile mapping ([ACE] "Efficiency Results",
  *   Table 6).  score (device) [T][k] fp32, column 0 = top-1 slot;
  *   topk_idx (device) [T][k] int32 or NULL.

@@ -41,25 +41,36 @@ def midpoint_tau(c, n_skip):
     return float(np.float32(0.5 * (cand[n_skip - 1] + cand[n_skip])))
 
 
-def gpu_layer(layer_cpu, amax32, device="cuda"):
+def _dev32(a, device):
+    if a is None:
+        return None
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+
+def gpu_layer(layer_cpu, amax32, device="cuda", views=None):
+    """Device copy of a layer and its ace_layer; views = (A_gsp, A_rcr) fp32
+    tables for the fusion rules that read them."""
     from token_dynamic_expert_b200 import ace
     g = {k: (v.to(device).contiguous() if torch.is_tensor(v) else v) for k, v in layer_cpu.items()}
-    g["amax"] = torch.from_numpy(np.ascontiguousarray(amax32, dtype=np.float32)).to(device)
+    g["amax"] = _dev32(amax32, device)
+    g["a_gsp"], g["a_rcr"] = (_dev32(v, device) for v in (views or (None, None)))
     c = ace.make_layer(g["gamma"], g["wr"], g["wg"], g["wu"], g["wd"], layer_cpu["k"],
-                       amax=g["amax"], router_bias=g["bias"])
+                       amax=g["amax"], router_bias=g["bias"], a_gsp=g["a_gsp"], a_rcr=g["a_rcr"])
     return g, c
 
 
-def run_gpu(layer_cpu, u_cpu, amax32, tau32, renorm=True, ws_tokens=None, stream=None):
+def run_gpu(layer_cpu, u_cpu, amax32, tau32, renorm=True, ws_tokens=None, stream=None,
+            fusion="max", views=None):
     from token_dynamic_expert_b200 import ace
-    g, c = gpu_layer(layer_cpu, amax32)
+    g, c = gpu_layer(layer_cpu, amax32, views=views)
     u = u_cpu.to("cuda").contiguous()
     T = u.shape[0]
     y = torch.full_like(u, float("nan"))
     ws = ace.alloc_workspace(ace.ace_workspace_size(c, ws_tokens or max(T, 1)))
     ws.fill_(0xFF)  # poison: reads of unwritten scratch show up as NaN
     dbg = ace.DebugOut(T, layer_cpu["k"], layer_cpu["E"])
-    ace.ace_moe_forward(c, u, tau32, y, ws, renorm=renorm, dbg=dbg.c, stream=stream)
+    ace.ace_moe_forward(c, u, tau32, y, ws, renorm=renorm, dbg=dbg.c, stream=stream,
+                        fusion=fusion)
     code, flags = ace.ace_read_status(ws, stream=stream)
     torch.cuda.synchronize()
     assert code == ace.ACE_OK and flags == 0, (ace.ace_status_str(code), flags)
@@ -81,12 +92,12 @@ def near_tie_tokens(logits, k, tol):
 
 
 def compare(layer_cpu, u_cpu, gpu, A_gsp32, A_rcr32, tau32, renorm=True, out_tokens=None,
-            y_tol=2e-2):
+            y_tol=2e-2, fusion="max"):
     """Compare the GPU forward with the oracle; returns a dict of the counts."""
     T = u_cpu.shape[0]
     k, E = layer_cpu["k"], layer_cpu["E"]
     ref = oracle.moe_forward(layer_cpu, u_cpu, tau32, A_gsp32, A_rcr32, renorm=renorm,
-                             outputs=False)
+                             outputs=False, fusion=fusion)
     assert ref["disagree"] == 0
     # logits: fp32 GEMM against the fp64 definition
     lerr = np.abs(gpu["logits"] - ref["logits"]).max() if T else 0.0
@@ -125,7 +136,8 @@ def compare(layer_cpu, u_cpu, gpu, A_gsp32, A_rcr32, tau32, renorm=True, out_tok
     toks = toks[exact_tokens[toks]] if T else toks
     if toks.size:
         sub = {**layer_cpu}
-        yref = oracle.moe_forward(sub, u_cpu[toks], tau32, A_gsp32, A_rcr32, renorm=renorm)["y"]
+        yref = oracle.moe_forward(sub, u_cpu[toks], tau32, A_gsp32, A_rcr32, renorm=renorm,
+                                  fusion=fusion)["y"]
         y = gpu["y"][toks]
         assert np.isfinite(y).all()
         num = np.abs(y - yref).max(axis=1)
@@ -137,8 +149,10 @@ def compare(layer_cpu, u_cpu, gpu, A_gsp32, A_rcr32, tau32, renorm=True, out_tok
     return res
 
 
-def setup_case(w, seed=0, token_seed=1000, T=None, tables="oracle", rate=None, renorm=True):
-    """Layer, tokens, fp32 tables and the midpoint threshold for a workload."""
+def setup_case(w, seed=0, token_seed=1000, T=None, tables="oracle", rate=None, renorm=True,
+               fusion="max"):
+    """Layer, tokens, fp32 tables and the midpoint threshold for a workload
+    (scores fused by ``fusion``)."""
     layer = workloads.make_layer(w, seed=seed)
     u = workloads.make_tokens(w, T=T, token_seed=token_seed)
     if tables == "oracle":
@@ -150,7 +164,8 @@ def setup_case(w, seed=0, token_seed=1000, T=None, tables="oracle", rate=None, r
     amax = np.maximum(A_gsp, A_rcr)
     rate = w.skip if rate is None else rate
     T_ = u.shape[0]
-    ref = oracle.moe_forward(layer, u, 0.0, A_gsp, A_rcr, renorm=renorm, outputs=False)
+    ref = oracle.moe_forward(layer, u, 0.0, A_gsp, A_rcr, renorm=renorm, outputs=False,
+                             fusion=fusion)
     n = oracle.n_skip_for(T_, w.k, rate, of=w.skip_of)
     tau = midpoint_tau(ref["c"], n)
     return layer, u, A_gsp, A_rcr, amax, tau, n

@@ -89,8 +89,9 @@ def test_forward_rejects_bad_calls(ace):
     assert _fwd(ace, L, ws=None) == ace.ACE_ERR_WORKSPACE
     assert _fwd(ace, L, ws=0x80010) == ace.ACE_ERR_WORKSPACE           # not 256-B aligned
     assert _fwd(ace, L, ws_bytes=1024) == ace.ACE_ERR_WORKSPACE        # too small
-    bad = ace.ace_fwd_opts(tau=0.1, renorm_topk=1, fusion=3, eps_rms=1e-6)
-    assert _fwd(ace, L, opts=bad) == ace.ACE_ERR_UNSUPPORTED
+    for f in (-1, 5):  # no such fusion rule
+        bad = ace.ace_fwd_opts(tau=0.1, renorm_topk=1, fusion=f, eps_rms=1e-6)
+        assert _fwd(ace, L, opts=bad) == ace.ACE_ERR_INVALID_ARG
     assert ace.lib().ace_moe_forward(ctypes.byref(L), 0x20000, 4, None, 0x40000, 0x80000,
                                      1 << 30, None, None) == ace.ACE_ERR_INVALID_ARG
 
@@ -135,3 +136,19 @@ def test_tau_quantile_rejects_bad_calls(ace):
     assert f(sc, 4, 8, 1, tau, ws, n - 1, None) == ace.ACE_ERR_WORKSPACE      # short
     assert f(sc, 4, 8, 1, tau, ws + 16, n, None) == ace.ACE_ERR_WORKSPACE     # misaligned
     assert f(sc, 4, 8, 1, tau, None, n, None) == ace.ACE_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("fusion,tables,ok", [
+    (1, {}, False), (1, dict(a_gsp=0x10000), False), (2, dict(a_rcr=0x10000), False),
+    (3, dict(a_rcr=0x10000), False), (4, dict(a_gsp=0x10000), False),
+    (3, dict(a_gsp=0x10002), False),                     # misaligned table
+    (1, dict(a_gsp=0x10000, a_rcr=0x10000), True), (3, dict(a_gsp=0x10000), True),
+    (4, dict(a_rcr=0x10000), True), (0, {}, True)])
+def test_fusion_rules_need_their_tables(ace, fusion, tables, ok):
+    """Each fusion rule reads the view tables it fuses; a missing one is an
+    argument error found before any launch.  Valid combinations get past
+    validation and stop at the (deliberately short) workspace."""
+    L = _fake_layer(ace, **tables)
+    opts = ace.ace_fwd_opts(tau=0.1, renorm_topk=1, fusion=fusion, eps_rms=1e-6)
+    want = ace.ACE_ERR_WORKSPACE if ok else ace.ACE_ERR_INVALID_ARG
+    assert _fwd(ace, L, opts=opts, ws_bytes=1024) == want

@@ -37,6 +37,28 @@ def _check(w, tables="oracle", rate=None, T=None, renorm=True, seed=0, y_tol=2e-
     return res, gpu
 
 
+# ------------------------------------------------------------ fusion rules
+@pytest.mark.parametrize("fusion", ["max", "max_views", "min", "mean", "gsp", "rcr"])
+@pytest.mark.parametrize("T", [300, 5])
+def test_fusion_rules(fusion, T):
+    """The pages' fusion ablation (min, mean) and single views (GSP, RCR)
+    next to ACE's max, through the prefill path (300 tokens) and the decode
+    kernel (5 tokens), with the view tables given separately; spread tables
+    so that the views disagree often."""
+    w = W("fusion", T=T, d=256, E=16, m=256, k=4, dtype="bf16", bias=False, skip=0.5,
+          skip_of="slots")
+    # "max_views": ACE's rule with no precomputed max table, only the views
+    rule = "max" if fusion == "max_views" else fusion
+    layer, u, A_gsp, A_rcr, amax, tau, n = setup_case(w, tables="spread", fusion=rule)
+    gpu = run_gpu(layer, u, amax if fusion == "max" else None, tau, fusion=rule,
+                  views=(A_gsp, A_rcr))
+    res = compare(layer, u, gpu, A_gsp, A_rcr, tau, fusion=rule)
+    print(fusion, T, res)
+    assert res["mask_mismatch"] == 0
+    if res["band"] == 0 and res["ties"] == 0:
+        assert int((gpu["keep"] == 0).sum()) == n
+
+
 def test_tiny_fp32_layer():
     """hidden 256, 8 experts of FFN 128, top-2, 64 tokens, fp32; tau skips
     50% of the non-top-1 slots."""
@@ -220,6 +242,37 @@ def test_full_shape_decode(T):
     res = compare(layer_cpu, u_cpu, gpu, A_gsp, A_rcr, tau)
     print("decode", T, res)
     assert res["compared_tokens"] == T
+
+
+@pytest.mark.parametrize("T", [8, 5, 1])
+def test_decode_back_to_back_launches(T):
+    """Hundreds of decode launches queued without a synchronisation, each
+    with its own workspace: every one finishes without a timeout flag and
+    gives the same output as a launch on an idle GPU.  (An odd copy ring once
+    let one phase-C warp group lap the other on a shared slot; those waits
+    timed out under back-to-back launches only.)"""
+    from token_dynamic_expert_b200 import ace
+    w = workloads.WORKLOADS["decode_bs8"].with_(T=T)
+    layer = workloads.make_layer(w, seed=5, device="cuda")
+    u = workloads.make_tokens(w, T=T, token_seed=91, device="cuda")
+    amax = torch.linspace(0.6, 1.4, w.E, device="cuda")
+    c = ace.make_layer(layer["gamma"], layer["wr"], layer["wg"], layer["wu"], layer["wd"], w.k,
+                       amax=amax, router_bias=layer["bias"])
+    nbytes = ace.ace_workspace_size(c, T)
+    tau = 0.08
+    y0 = torch.empty_like(u)
+    ws0 = ace.alloc_workspace(nbytes)
+    ace.ace_moe_forward(c, u, tau, y0, ws0)
+    assert ace.ace_read_status(ws0) == (ace.ACE_OK, 0)
+    n = 300
+    wss = [ace.alloc_workspace(nbytes) for _ in range(n)]
+    ys = torch.empty(n, T, w.d, dtype=u.dtype, device="cuda")
+    for i in range(n):
+        ace.ace_moe_forward(c, u, tau, ys[i], wss[i])
+    torch.cuda.synchronize()
+    bad = [i for i in range(n) if ace.ace_read_status(wss[i]) != (ace.ACE_OK, 0)]
+    assert bad == [], bad[:10]
+    assert torch.equal(ys, y0.unsqueeze(0).expand_as(ys))
 
 
 @pytest.mark.parametrize("tau", [-1.0, float("inf")])

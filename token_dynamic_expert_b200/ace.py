@@ -23,7 +23,9 @@ ACE_OK, ACE_ERR_INVALID_ARG, ACE_ERR_WORKSPACE, ACE_ERR_CUDA, ACE_ERR_UNSUPPORTE
     ACE_ERR_DEVICE_FAULT, ACE_ERR_TIMEOUT = range(7)
 ACE_BF16, ACE_F32 = 0, 1
 ACE_GSP_FRO, ACE_GSP_SPECTRAL = 0, 1
-ACE_FUSE_MAX = 0
+ACE_FUSE_MAX, ACE_FUSE_MIN, ACE_FUSE_MEAN, ACE_FUSE_GSP, ACE_FUSE_RCR = 0, 1, 2, 3, 4
+FUSIONS = {"max": ACE_FUSE_MAX, "min": ACE_FUSE_MIN, "mean": ACE_FUSE_MEAN, "gsp": ACE_FUSE_GSP,
+           "rcr": ACE_FUSE_RCR}
 ACE_FLAG_BAD_INDEX, ACE_FLAG_TIMEOUT, ACE_FLAG_OVERFLOW = 0x1, 0x2, 0x4
 
 _vp = ctypes.c_void_p
@@ -32,7 +34,8 @@ _vp = ctypes.c_void_p
 class ace_layer(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int), ("E", ctypes.c_int), ("m", ctypes.c_int), ("k", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("gamma", _vp), ("w_router", _vp), ("router_bias", _vp),
-                ("w_gate", _vp), ("w_up", _vp), ("w_down", _vp), ("amax", _vp)]
+                ("w_gate", _vp), ("w_up", _vp), ("w_down", _vp), ("amax", _vp), ("a_gsp", _vp),
+                ("a_rcr", _vp)]
 
 
 class ace_fwd_opts(ctypes.Structure):
@@ -126,17 +129,23 @@ def _dtype_code(t):
     raise TypeError("unsupported dtype %s" % t.dtype)
 
 
-def make_layer(gamma, w_router, w_gate, w_up, w_down, k, amax=None, router_bias=None):
+def make_layer(gamma, w_router, w_gate, w_up, w_down, k, amax=None, router_bias=None,
+               a_gsp=None, a_rcr=None):
     """Pack device tensors into an ``ace_layer``.  The caller keeps the tensors
     alive while the struct is in use."""
     E, d = w_router.shape
     m = w_gate.shape[1]
-    for t in (gamma, w_router, w_gate, w_up, w_down, amax, router_bias):
+    for t in (gamma, w_router, w_gate, w_up, w_down, amax, router_bias, a_gsp, a_rcr):
         if t is not None and not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
     return ace_layer(d=d, E=E, m=m, k=k, dtype=_dtype_code(w_router), gamma=_ptr(gamma),
                      w_router=_ptr(w_router), router_bias=_ptr(router_bias), w_gate=_ptr(w_gate),
-                     w_up=_ptr(w_up), w_down=_ptr(w_down), amax=_ptr(amax))
+                     w_up=_ptr(w_up), w_down=_ptr(w_down), amax=_ptr(amax), a_gsp=_ptr(a_gsp),
+                     a_rcr=_ptr(a_rcr))
+
+
+def _fusion(f):
+    return FUSIONS[f] if isinstance(f, str) else int(f)
 
 
 def ace_workspace_size(layer, max_tokens):
@@ -148,8 +157,9 @@ def alloc_workspace(nbytes, device="cuda"):
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def ace_moe_forward(layer, u, tau, y, ws, renorm=True, eps_rms=1e-6, dbg=None, stream=None):
-    opts = ace_fwd_opts(tau=float(tau), renorm_topk=int(bool(renorm)), fusion=ACE_FUSE_MAX,
+def ace_moe_forward(layer, u, tau, y, ws, renorm=True, eps_rms=1e-6, dbg=None, stream=None,
+                    fusion="max"):
+    opts = ace_fwd_opts(tau=float(tau), renorm_topk=int(bool(renorm)), fusion=_fusion(fusion),
                         eps_rms=float(eps_rms))
     code = _lib.ace_moe_forward(ctypes.byref(layer), _ptr(u), int(u.shape[0]), ctypes.byref(opts),
                                 _ptr(y), _ptr(ws), ws.numel(),
@@ -158,8 +168,9 @@ def ace_moe_forward(layer, u, tau, y, ws, renorm=True, eps_rms=1e-6, dbg=None, s
     return y
 
 
-def ace_moe_scores(layer, u, score, ws, topk_idx=None, renorm=True, eps_rms=1e-6, stream=None):
-    opts = ace_fwd_opts(tau=0.0, renorm_topk=int(bool(renorm)), fusion=ACE_FUSE_MAX,
+def ace_moe_scores(layer, u, score, ws, topk_idx=None, renorm=True, eps_rms=1e-6, stream=None,
+                   fusion="max"):
+    opts = ace_fwd_opts(tau=0.0, renorm_topk=int(bool(renorm)), fusion=_fusion(fusion),
                         eps_rms=float(eps_rms))
     code = _lib.ace_moe_scores(ctypes.byref(layer), _ptr(u), int(u.shape[0]), ctypes.byref(opts),
                                _ptr(score), _ptr(topk_idx), _ptr(ws), ws.numel(), _stream(stream))
@@ -167,10 +178,11 @@ def ace_moe_scores(layer, u, score, ws, topk_idx=None, renorm=True, eps_rms=1e-6
     return score
 
 
-def ace_moe_decode_noalloc(layer, u, tau, y, renorm=True, eps_rms=1e-6, stream=None):
+def ace_moe_decode_noalloc(layer, u, tau, y, renorm=True, eps_rms=1e-6, stream=None,
+                           fusion="max"):
     """Decode forward (1-8 tokens) with the library's fixed scratch array
     instead of a caller workspace; see include/ace.h."""
-    opts = ace_fwd_opts(tau=float(tau), renorm_topk=int(bool(renorm)), fusion=ACE_FUSE_MAX,
+    opts = ace_fwd_opts(tau=float(tau), renorm_topk=int(bool(renorm)), fusion=_fusion(fusion),
                         eps_rms=float(eps_rms))
     code = _lib.ace_moe_decode_noalloc(ctypes.byref(layer), _ptr(u), int(u.shape[0]),
                                        ctypes.byref(opts), _ptr(y), _stream(stream))

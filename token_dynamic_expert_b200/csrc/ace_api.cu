@@ -104,6 +104,24 @@ ace_status check_layer(const ace_layer* L, bool need_experts) {
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
+}  // namespace
+
+namespace ace {
+// The fusion rule is known and the tables it reads are present.
+ace_status check_fusion(const ace_layer& L, int fusion) {
+  const bool need_g = fusion == ACE_FUSE_MIN || fusion == ACE_FUSE_MEAN || fusion == ACE_FUSE_GSP;
+  const bool need_r = fusion == ACE_FUSE_MIN || fusion == ACE_FUSE_MEAN || fusion == ACE_FUSE_RCR;
+  if (fusion < ACE_FUSE_MAX || fusion > ACE_FUSE_RCR) return ACE_ERR_INVALID_ARG;
+  if ((need_g && !L.a_gsp) || (need_r && !L.a_rcr)) return ACE_ERR_INVALID_ARG;
+  if ((L.amax && !aligned(L.amax, 4)) || (L.a_gsp && !aligned(L.a_gsp, 4)) ||
+      (L.a_rcr && !aligned(L.a_rcr, 4)))
+    return ACE_ERR_INVALID_ARG;
+  return ACE_OK;
+}
+}  // namespace ace
+
+namespace {
+
 ace_status cuda_fail(cudaError_t e) {
   g_last_cuda_error = e;
   return ACE_ERR_CUDA;
@@ -148,7 +166,8 @@ ace_status run_routing(const ace_layer& L, const void* u, int T, const ace_fwd_o
   so.n_tiles = at<int32_t>(ws, ly.n_tiles);
   so.max_tiles = ly.max_tiles;
   so.tile_n = kTileN;
-  ACE_CK(launch_topk_mask(at<float>(ws, ly.part), splitk, T, L.E, L.k, L.router_bias, L.amax,
+  FuseTables ft{L.amax, L.a_gsp, L.a_rcr, (int)o.fusion};
+  ACE_CK(launch_topk_mask(at<float>(ws, ly.part), splitk, T, L.E, L.k, L.router_bias, ft,
                           o.tau, o.renorm_topk, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
                           at<float>(ws, ly.score), at<uint8_t>(ws, ly.keep),
                           at<uint32_t>(ws, ly.bitmap), at<int32_t>(ws, ly.hist), logits_dbg,
@@ -162,7 +181,8 @@ ace_status check_common(const ace_layer* layer, const void* u, int T, const ace_
   ace_status st = check_layer(layer, need_experts);
   if (st != ACE_OK) return st;
   if (!opts || T < 0) return ACE_ERR_INVALID_ARG;
-  if (opts->fusion != ACE_FUSE_MAX) return ACE_ERR_UNSUPPORTED;
+  st = check_fusion(*layer, opts->fusion);
+  if (st != ACE_OK) return st;
   if (T > 0 && (!u || !aligned(u, 16))) return ACE_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256)) return ACE_ERR_WORKSPACE;
   return ACE_OK;
@@ -244,7 +264,7 @@ ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T, const a
     // decode: one cooperative kernel streams the surviving experts' weights
     if (ev_b) ACE_CK(cudaEventRecord(ev_b, s));
     if (ev_m) ACE_CK(cudaEventRecord(ev_m, s));
-    ACE_CK(launch_decode(L, u, T, opts->tau, opts->renorm_topk, opts->eps_rms, y,
+    ACE_CK(launch_decode(L, (int)opts->fusion, u, T, opts->tau, opts->renorm_topk, opts->eps_rms, y,
                          at<float>(ws, ly.part), at<void>(ws, ly.h), at<int32_t>(ws, ly.idx),
                          at<float>(ws, ly.gate), at<float>(ws, ly.score), at<uint8_t>(ws, ly.keep),
                          at<int32_t>(ws, ly.offsets), at<int32_t>(ws, ly.slot_token),

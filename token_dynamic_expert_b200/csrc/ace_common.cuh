@@ -209,6 +209,30 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- fusion
+// The per-expert factor F(A^GSP, A^RCR)(e) of the fused score c = g F: the
+// gates are non-negative, so fusing the two views' scores g A^GSP and
+// g A^RCR by max / min / mean / one view equals fusing the tables.
+struct FuseTables {
+  const float* amax;   // max(A^GSP, A^RCR), or NULL
+  const float* a_gsp;  // or NULL
+  const float* a_rcr;  // or NULL
+  int fusion;          // ace_fusion
+};
+
+__device__ __forceinline__ float fused_factor(const FuseTables& f, int e) {
+  switch (f.fusion) {
+    case ACE_FUSE_MIN: return fminf(f.a_gsp[e], f.a_rcr[e]);
+    case ACE_FUSE_MEAN: return 0.5f * (f.a_gsp[e] + f.a_rcr[e]);
+    case ACE_FUSE_GSP: return f.a_gsp[e];
+    case ACE_FUSE_RCR: return f.a_rcr[e];
+    default:
+      if (f.amax) return f.amax[e];
+      if (f.a_gsp && f.a_rcr) return fmaxf(f.a_gsp[e], f.a_rcr[e]);
+      return 1.0f;
+  }
+}
+
 // ---------------------------------------------------------------- top-k
 // order-preserving map of a float to an unsigned key (larger float, larger key)
 __device__ __forceinline__ uint32_t fkey(float f) {

@@ -41,6 +41,7 @@ struct FwdLayout {
 FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms);
 
 int device_sm_count();
+ace_status check_fusion(const ace_layer& L, int fusion);
 
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
@@ -54,8 +55,9 @@ cudaError_t launch_router_logits(ace_dtype dt, const void* u, const float* inv_r
                                  const float* gamma, const void* wr, int T, int d, int E,
                                  int splitk, float* part, cudaStream_t s);
 struct ScanOut;
+struct FuseTables;
 cudaError_t launch_topk_mask(const float* part, int splitk, int T, int E, int k,
-                             const float* bias, const float* amax, float tau, int renorm,
+                             const float* bias, const FuseTables& ft, float tau, int renorm,
                              int32_t* idx, float* gate, float* score, uint8_t* keep,
                              uint32_t* bitmap, int32_t* hist, float* logits_out,
                              uint32_t* status, uint32_t* done_ctr, const ScanOut* so,
@@ -76,7 +78,8 @@ cudaError_t launch_experts_simt(const ace_layer& L, const void* xp, void* h, flo
                                 const float* slot_gate, cudaStream_t s);
 size_t decode_smem_bytes(int T, int d, int m, int k, int E, int num_sms);
 bool decode_fits(int T, int d, int m, int k, int E, int num_sms);
-cudaError_t launch_decode(const ace_layer& L, const void* u, int T, float tau, int renorm,
+cudaError_t launch_decode(const ace_layer& L, int fusion, const void* u, int T, float tau,
+                          int renorm,
                           float eps_rms, void* y, float* logits, void* h, int32_t* idx,
                           float* gate, float* score, uint8_t* keep, int32_t* offsets,
                           int32_t* slot_token, int32_t* slot_rank, int32_t* slot_of,

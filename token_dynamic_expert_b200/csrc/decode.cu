@@ -57,7 +57,7 @@ struct DecodeArgs {
   const __nv_bfloat16* wg;
   const __nv_bfloat16* wu;
   const __nv_bfloat16* wd;
-  const float* amax;
+  FuseTables ft;
   const __nv_bfloat16* u;
   __nv_bfloat16* y;
   int T, d, E, m, k;
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     }
     if (lane < k) {
       const float g = ex / denom;
-      const float sc = g * (a.amax ? a.amax[sel_e] : 1.0f);
+      const float sc = g * fused_factor(a.ft, sel_e);
       sh.t_idx[t * k + lane] = sel_e;
       sh.t_gate[t * k + lane] = g;
       sh.t_score[t * k + lane] = sc;
@@ -418,7 +418,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
 #endif
     }
   } else {
-    // two groups of 8 warps take alternate stages; in a group, warp
+    // two groups of 8 warps take alternate stages (the ring is even, so a
+    // slot always belongs to the same group); in a group, warp
     // 2r + mat reduces row r of the stage against W^gate (mat 0) or W^up
     // (mat 1) for every kept token of the row's expert.  The dots go to the
     // CTA's table; each warp releases the stage on its own.
@@ -602,7 +603,13 @@ static int ring_stages(int T, int d, int m, int k, int E, int num_sms) {
   const size_t avail = (size_t)kSmemBudget - sizeof(DecShared) - 1024 -
                        region_bytes(T, d, m, k, E, num_sms);
   int n = (int)(avail / kStageBytes);
-  return n > kRing ? kRing : n;
+  n = n > kRing ? kRing : n;
+  // even: phase C's two consumer groups take alternate stages, so with an
+  // even ring each slot belongs to one group, which waits on the slot's fills
+  // in order.  With an odd ring a slot alternates between the groups, and a
+  // group running a lap ahead would test the slot's full barrier for a parity
+  // that an older, already completed phase also has.
+  return n & ~1;
 }
 
 size_t decode_smem_bytes(int T, int d, int m, int k, int E, int num_sms) {
@@ -613,7 +620,7 @@ size_t decode_smem_bytes(int T, int d, int m, int k, int E, int num_sms) {
 bool decode_fits(int T, int d, int m, int k, int E, int num_sms) {
   if (T < 1 || T > kDecodeMaxT || d > 2048 || d % 32 != 0 || m % 8 != 0) return false;
   const int n = ring_stages(T, d, m, k, E, num_sms);
-  if (n < 3) return false;
+  if (n < 2) return false;
   if ((size_t)T * d * 4 > (size_t)n * kStageBytes) return false;  // the unrounded x
   const int rows = (d + num_sms - 1) / num_sms;                    // phase-D rows per CTA
   if (rows > kCompWarps) return false;
@@ -623,7 +630,8 @@ bool decode_fits(int T, int d, int m, int k, int E, int num_sms) {
   return decode_smem_bytes(T, d, m, k, E, num_sms) >= 1024 + hbytes + 2 * dstage;
 }
 
-cudaError_t launch_decode(const ace_layer& L, const void* u, int T, float tau, int renorm,
+cudaError_t launch_decode(const ace_layer& L, int fusion, const void* u, int T, float tau,
+                          int renorm,
                           float eps_rms, void* y, float* logits, void* h, int32_t* idx,
                           float* gate, float* score, uint8_t* keep, int32_t* offsets,
                           int32_t* slot_token, int32_t* slot_rank, int32_t* slot_of,
@@ -636,7 +644,10 @@ cudaError_t launch_decode(const ace_layer& L, const void* u, int T, float tau, i
   a.wg = (const __nv_bfloat16*)L.w_gate;
   a.wu = (const __nv_bfloat16*)L.w_up;
   a.wd = (const __nv_bfloat16*)L.w_down;
-  a.amax = L.amax;
+  a.ft.amax = L.amax;
+  a.ft.a_gsp = L.a_gsp;
+  a.ft.a_rcr = L.a_rcr;
+  a.ft.fusion = fusion;
   a.u = (const __nv_bfloat16*)u;
   a.y = (__nv_bfloat16*)y;
   a.T = T;

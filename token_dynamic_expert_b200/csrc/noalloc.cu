@@ -92,7 +92,7 @@ extern "C" ace_status ace_moe_decode_noalloc(const ace_layer* layer, const void*
   if (L.d <= 0 || L.E <= 0 || L.m <= 0 || L.k <= 0 || L.k > L.E || L.k > kMaxK)
     return ACE_ERR_INVALID_ARG;
   if (!L.gamma || !L.w_router || !L.w_gate || !L.w_up || !L.w_down) return ACE_ERR_INVALID_ARG;
-  if (opts->fusion != ACE_FUSE_MAX) return ACE_ERR_UNSUPPORTED;
+  if (check_fusion(L, (int)opts->fusion) != ACE_OK) return ACE_ERR_INVALID_ARG;
   const uintptr_t mis = reinterpret_cast<uintptr_t>(u) | reinterpret_cast<uintptr_t>(y) |
                         reinterpret_cast<uintptr_t>(L.w_router) |
                         reinterpret_cast<uintptr_t>(L.w_gate) |
@@ -116,7 +116,7 @@ extern "C" ace_status ace_moe_decode_noalloc(const ace_layer* layer, const void*
   // the status word and the grid-barrier counter must start at zero
   if (cudaMemsetAsync(w, 0, 256, s) != cudaSuccess) return ACE_ERR_CUDA;
   auto at = [&](size_t off) { return w + off; };
-  if (launch_decode(L, u, T, opts->tau, opts->renorm_topk, opts->eps_rms, y,
+  if (launch_decode(L, (int)opts->fusion, u, T, opts->tau, opts->renorm_topk, opts->eps_rms, y,
                     reinterpret_cast<float*>(at(ly.logits)), at(ly.h),
                     reinterpret_cast<int32_t*>(at(ly.idx)), reinterpret_cast<float*>(at(ly.gate)),
                     reinterpret_cast<float*>(at(ly.score)), at(ly.keep),

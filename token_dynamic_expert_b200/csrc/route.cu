@@ -193,7 +193,7 @@ cudaError_t launch_router_logits(ace_dtype dt, const void* u, const float* inv_r
 template <int V>
 __global__ void __launch_bounds__(1024) k_topk_mask(
     const float* __restrict__ part, int splitk, int Tn, int E, int k,
-    const float* __restrict__ bias, const float* __restrict__ amax, float tau, int renorm,
+    const float* __restrict__ bias, const FuseTables ft, float tau, int renorm,
     int32_t* __restrict__ idx, float* __restrict__ gate, float* __restrict__ score,
     uint8_t* __restrict__ keep, uint32_t* __restrict__ bitmap, int32_t* __restrict__ hist,
     float* __restrict__ logits_out, uint32_t* status, uint32_t* done_ctr, ScanOut so) {
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
     }
     if (lane < k) {
       const float g = ex / denom;
-      const float sc = g * (amax ? amax[my_e] : 1.0f);
+      const float sc = g * fused_factor(ft, my_e);
       const bool kept = (lane == 0) || !(sc < tau);
       const size_t o = (size_t)t * k + lane;
       idx[o] = my_e;
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
 }
 
 cudaError_t launch_topk_mask(const float* part, int splitk, int T, int E, int k,
-                             const float* bias, const float* amax, float tau, int renorm,
+                             const float* bias, const FuseTables& ft, float tau, int renorm,
                              int32_t* idx, float* gate, float* score, uint8_t* keep,
                              uint32_t* bitmap, int32_t* hist, float* logits_out,
                              uint32_t* status, uint32_t* done_ctr, const ScanOut* so,
@@ -284,7 +284,7 @@ cudaError_t launch_topk_mask(const float* part, int splitk, int T, int E, int k,
   const ScanOut sv = so ? *so : ScanOut{};
   if (so == nullptr) done_ctr = nullptr;
 #define ACE_TOPK(V)                                                                         \
-  k_topk_mask<V><<<grid, kChunk * 32, 0, s>>>(part, splitk, T, E, k, bias, amax, tau, renorm, \
+  k_topk_mask<V><<<grid, kChunk * 32, 0, s>>>(part, splitk, T, E, k, bias, ft, tau, renorm,   \
                                               idx, gate, score, keep, bitmap, hist,           \
                                               logits_out, status, done_ctr, sv)
   if (E <= 32) ACE_TOPK(1);
