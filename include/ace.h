@@ -15,6 +15,9 @@
  *   - The library allocates no device memory: scratch space is the caller's
  *     workspace `ws` of at least the size the matching *_workspace_size
  *     query returns, 256-byte aligned.
+ *   - Weight, gamma, activation and output pointers are 16-byte aligned
+ *     (the kernels move them in 16-byte vectors and bulk copies); tables
+ *     are 4-byte aligned.  A misaligned pointer is ACE_ERR_INVALID_ARG.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Work is enqueued asynchronously; nothing synchronises the
  *     host except ace_read_status.  No call allocates or synchronises, so

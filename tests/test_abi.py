@@ -69,7 +69,8 @@ def _fwd(ace, layer, T=4, u=0x20000, y=0x40000, ws=0x80000, ws_bytes=1 << 30, op
 
 @pytest.mark.parametrize("bad", [dict(d=0), dict(E=-1), dict(k=0), dict(k=9), dict(k=17, E=32),
                                  dict(dtype=7), dict(gamma=None), dict(w_router=None),
-                                 dict(w_gate=None), dict(w_down=None), dict(w_up=0x10008)])
+                                 dict(w_gate=None), dict(w_down=None), dict(w_up=0x10008),
+                                 dict(gamma=0x10004)])
 def test_forward_rejects_bad_layers(ace, bad):
     assert _fwd(ace, _fake_layer(ace, **bad)) == ace.ACE_ERR_INVALID_ARG
 

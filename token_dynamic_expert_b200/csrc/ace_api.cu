@@ -98,7 +98,7 @@ ace_status check_layer(const ace_layer* L, bool need_experts) {
       return ACE_ERR_INVALID_ARG;
     if (L->dtype == ACE_BF16 && (L->d % 128 != 0 || L->m % 128 != 0)) return ACE_ERR_UNSUPPORTED;
   }
-  if (!aligned(L->w_router, 16)) return ACE_ERR_INVALID_ARG;
+  if (!aligned(L->w_router, 16) || !aligned(L->gamma, 16)) return ACE_ERR_INVALID_ARG;
   return ACE_OK;
 }
 

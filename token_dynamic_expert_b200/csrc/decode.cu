@@ -34,7 +34,7 @@
 // prefetches from the producer warp's idle lanes, 2 bulk prefetches queued
 // after the phase-C copies.
 #ifndef ACE_DECODE_PREFETCH
-#define ACE_DECODE_PREFETCH 1
+#define ACE_DECODE_PREFETCH 2
 #endif
 
 namespace ace {
@@ -98,6 +98,9 @@ struct DecShared {
   int t_keep[kMaxSlots];
   int t_pos[kMaxSlots];
   float acc_d[kCompWarps][kDecodeMaxT];  // phase-D per-warp token sums
+  uint32_t tok_mask[kMaxE];    // per expert: bit t set when token t kept a slot of it
+  int e_base[kMaxE];           // per expert: its first slot
+  uint64_t in_bar;             // phase A: u, gamma and the router rows have landed
   int abort;
 };
 
@@ -185,9 +188,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const bool producer = warp == kCompWarps;
   const int nring = a.nring;
   uint8_t* ring = dsm;
-  float* xf = reinterpret_cast<float*>(dsm);  // phase A only, inside the ring
+  // phase A lives inside the ring: the unrounded x (fp32), then the staged
+  // inputs u (bf16), gamma (fp32) and the CTA's router rows (bf16)
+  float* xf = reinterpret_cast<float*>(dsm);
+  __nv_bfloat16* us = reinterpret_cast<__nv_bfloat16*>(dsm + (size_t)NT * d * 4);
+  float* gs = reinterpret_cast<float*>(dsm + (size_t)NT * d * 6);
+  __nv_bfloat16* wrs = reinterpret_cast<__nv_bfloat16*>(dsm + (size_t)NT * d * 6 + (size_t)d * 4);
   __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(dsm + a.region);  // bf16(x)
   float* part = reinterpret_cast<float*>(dsm + a.region + (size_t)NT * a.d * 2);
+  const int n_router_warps = (E + G - 1) / G;
+  // router rows of this CTA: experts blockIdx.x + G * r, r < n_mine
+  const int n_mine = (int)blockIdx.x < E ? min(n_router_warps, (E - 1 - (int)blockIdx.x) / G + 1) : 0;
   if (threadIdx.x == 0) {
     sh.abort = 0;
     for (int i = 0; i < kRing; ++i) {
@@ -196,54 +207,40 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       mbar_init(&sh.full_d[i], 1);
       mbar_init(&sh.empty_d[i], kCompWarps);
     }
+    mbar_init(&sh.in_bar, 1);
     fence_barrier_init();
+    // one round trip for every input of phase A
+    mbar_expect_tx(&sh.in_bar, (uint32_t)(NT * d * 2 + d * 4 + n_mine * d * 2));
+    bulk_g2s(us, a.u, (uint32_t)(NT * d * 2), &sh.in_bar);
+    bulk_g2s(gs, a.gamma, (uint32_t)(d * 4), &sh.in_bar);
+    for (int r = 0; r < n_mine; ++r)
+      bulk_g2s(wrs + (size_t)r * d, a.wr + (size_t)((int)blockIdx.x + G * r) * d,
+               (uint32_t)(d * 2), &sh.in_bar);
   }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) sh.tok_mask[e] = 0u;
   stamp(a, 0);
+  __syncthreads();  // barrier inits are visible
 
   // ---------------------------------------------------------- phase A
-  const int n_router_warps = (E + G - 1) / G;
-  const int rwarp = kCompWarps - 1 - warp;  // router warps count down from the last
-  const int my_e = (int)blockIdx.x + G * rwarp;
-  const bool router = warp < kCompWarps && rwarp < n_router_warps && my_e < E;
-  constexpr int kRV = 8;  // 16-byte chunks per lane of a router row (d <= 2048)
-  uint4 wrq[kRV];
-  if (router) {
-    const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + (size_t)my_e * d);
-#pragma unroll
-    for (int i = 0; i < kRV; ++i) {
-      const int v = lane + 32 * i;
-      wrq[i] = v < d / 8 ? __ldg(wrow + v) : make_uint4(0, 0, 0, 0);
-    }
-  }
-  if (warp < NT) {  // token warps: one pass, the row stays in registers
+  if (!wait_bar(&sh.in_bar, 0, a, sh)) return;
+  if (warp < NT) {  // token warps: x = u / rms(u) * gamma
     const int t = warp;
-    const uint4* ur = reinterpret_cast<const uint4*>(a.u + (size_t)t * d);
-    const float4* gp = reinterpret_cast<const float4*>(a.gamma);
-    constexpr int kUV = 8;  // d <= 2048
-    uint4 uq[kUV];
-#pragma unroll
-    for (int i = 0; i < kUV; ++i) {
-      const int v = lane + 32 * i;
-      uq[i] = v < d / 8 ? ur[v] : make_uint4(0, 0, 0, 0);
-    }
+    const uint4* ur = reinterpret_cast<const uint4*>(us + (size_t)t * d);
+    const float4* gp = reinterpret_cast<const float4*>(gs);
     float ss = 0.f;
-#pragma unroll
-    for (int i = 0; i < kUV; ++i) {
+    for (int v = lane; v < d / 8; v += 32) {
       float f[8];
-      bf16x8_to_f32(uq[i], f);
+      bf16x8_to_f32(ur[v], f);
 #pragma unroll
       for (int c = 0; c < 8; ++c) ss = fmaf(f[c], f[c], ss);
     }
     ss = warp_sum(ss);
     stamp(a, 7);
     const float r = 1.0f / sqrtf(ss / (float)d + a.eps_rms);
-#pragma unroll
-    for (int i = 0; i < kUV; ++i) {
-      const int v = lane + 32 * i;
-      if (v >= d / 8) continue;
+    for (int v = lane; v < d / 8; v += 32) {
       float f[8];
-      bf16x8_to_f32(uq[i], f);
-      const float4 g0 = __ldg(gp + 2 * v), g1 = __ldg(gp + 2 * v + 1);
+      bf16x8_to_f32(ur[v], f);
+      const float4 g0 = gp[2 * v], g1 = gp[2 * v + 1];
       const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
       float xv[8];
 #pragma unroll
@@ -260,16 +257,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   }
   __syncthreads();
   stamp(a, 1);
-  if (router) {
+  // router: warp w < n_mine (counting down from the last compute warp) dots
+  // its staged row with every token's x
+  const int rwarp = kCompWarps - 1 - warp;
+  if (warp < kCompWarps && rwarp < n_mine) {
+    const int my_e = (int)blockIdx.x + G * rwarp;
+    const uint4* wrow = reinterpret_cast<const uint4*>(wrs + (size_t)rwarp * d);
     float acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-#pragma unroll
-    for (int i = 0; i < kRV; ++i) {
-      const int v = lane + 32 * i;
-      if (v >= d / 8) continue;
+    for (int v = lane; v < d / 8; v += 32) {
       float w[8];
-      bf16x8_to_f32(wrq[i], w);
+      bf16x8_to_f32(wrow[v], w);
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
         float xv[8];
@@ -280,8 +279,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     }
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
-      const float s = warp_sum(acc[t]);
-      if (lane == 0) a.logits[(size_t)t * E + my_e] = s + (a.bias ? a.bias[my_e] : 0.f);
+      const float sm = warp_sum(acc[t]);
+      if (lane == 0) a.logits[(size_t)t * E + my_e] = sm + (a.bias ? a.bias[my_e] : 0.f);
     }
   }
   if (!grid_barrier(a, sh, 1)) return;
@@ -318,49 +317,66 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       sh.t_idx[t * k + lane] = sel_e;
       sh.t_gate[t * k + lane] = g;
       sh.t_score[t * k + lane] = sc;
-      sh.t_keep[t * k + lane] = (lane == 0) || !(sc < a.tau);
+      const bool kept = (lane == 0) || !(sc < a.tau);
+      sh.t_keep[t * k + lane] = kept;
+      if (kept) atomicOr(&sh.tok_mask[sel_e], 1u << t);  // distinct experts per token
     }
   }
   __syncthreads();
-  // slot position = number of kept slots with a smaller (expert, token) key
+  // counting sort of the kept slots by (expert, token): per-expert counts
+  // are the popcounts of the token masks; one warp scans them over experts
+  // (consecutive experts per lane) into first-slot bases and the list of
+  // distinct experts
   const int TK = NT * k;
+  if (warp == 0) {
+    const int per = (E + 31) / 32;
+    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+    int cnt = 0, nue = 0;
+    for (int e = e0; e < e1; ++e) {
+      const uint32_t mk = sh.tok_mask[e];
+      cnt += __popc(mk);
+      nue += mk != 0u;
+    }
+    int ci = cnt, ui = nue;  // inclusive scans over lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int c2 = __shfl_up_sync(0xffffffffu, ci, o);
+      const int u2 = __shfl_up_sync(0xffffffffu, ui, o);
+      if (lane >= o) {
+        ci += c2;
+        ui += u2;
+      }
+    }
+    int base = ci - cnt, ub = ui - nue;
+    for (int e = e0; e < e1; ++e) {
+      const uint32_t mk = sh.tok_mask[e];
+      sh.e_base[e] = base;
+      if (mk != 0u) {
+        sh.uexp[ub] = e;
+        sh.ufirst[ub] = base;
+        ++ub;
+      }
+      base += __popc(mk);
+    }
+    if (lane == 31) {
+      sh.n_slots = ci;
+      sh.n_uexp = ui;
+      sh.ufirst[ui] = ci;
+    }
+  }
+  __syncthreads();
   if ((int)threadIdx.x < TK) {
     const int s = threadIdx.x;
     int pos = -1;
     if (sh.t_keep[s]) {
-      const int key = sh.t_idx[s] * kDecodeMaxT + s / k;
-      pos = 0;
-      for (int o = 0; o < TK; ++o)
-        pos += (sh.t_keep[o] && sh.t_idx[o] * kDecodeMaxT + o / k < key) ? 1 : 0;
-      sh.slot_e[pos] = sh.t_idx[s];
-      sh.slot_t[pos] = s / k;
+      const int e = sh.t_idx[s], t = s / k;
+      pos = sh.e_base[e] + __popc(sh.tok_mask[e] & ((1u << t) - 1u));
+      sh.slot_e[pos] = e;
+      sh.slot_t[pos] = t;
       sh.slot_r[pos] = s % k;
       sh.slot_g[pos] = sh.t_gate[s];
     }
     sh.t_pos[s] = pos;
-  }
-  __syncthreads();
-  if (warp == 0) {  // slot count and distinct experts by ballots (TK <= 128)
-    int S = 0;
-    for (int b = 0; b < TK; b += 32)
-      S += __popc(__ballot_sync(0xffffffffu, b + lane < TK && sh.t_keep[b + lane]));
-    int nu = 0;
-    for (int b = 0; b < S; b += 32) {
-      const int s = b + lane;
-      const bool first = s < S && (s == 0 || sh.slot_e[s] != sh.slot_e[s - 1]);
-      const uint32_t mk = __ballot_sync(0xffffffffu, first);
-      if (first) {
-        const int at = nu + __popc(mk & ((1u << lane) - 1u));
-        sh.uexp[at] = sh.slot_e[s];
-        sh.ufirst[at] = s;
-      }
-      nu += __popc(mk);
-    }
-    if (lane == 0) {
-      sh.n_slots = S;
-      sh.n_uexp = nu;
-      sh.ufirst[nu] = S;
-    }
   }
   __syncthreads();
   stamp(a, 3);
@@ -567,11 +583,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       a.slot_token[threadIdx.x] = sh.slot_t[threadIdx.x];
       a.slot_rank[threadIdx.x] = sh.slot_r[threadIdx.x];
     }
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
-      int c = 0;  // first slot of expert >= e
-      for (int s = 0; s < S; ++s) c += sh.slot_e[s] < e;
-      a.offsets[e] = c;
-    }
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) a.offsets[e] = e < E ? sh.e_base[e] : S;
     if (threadIdx.x == 0) *a.n_kept = S;
   }
 }
@@ -621,7 +633,10 @@ bool decode_fits(int T, int d, int m, int k, int E, int num_sms) {
   if (T < 1 || T > kDecodeMaxT || d > 2048 || d % 32 != 0 || m % 8 != 0) return false;
   const int n = ring_stages(T, d, m, k, E, num_sms);
   if (n < 2) return false;
-  if ((size_t)T * d * 4 > (size_t)n * kStageBytes) return false;  // the unrounded x
+  // phase A inside the ring: x (fp32), u (bf16), gamma, the router rows
+  const size_t staged = (size_t)T * d * 6 + (size_t)d * 4 +
+                        (size_t)((E + num_sms - 1) / num_sms) * d * 2;
+  if (staged > (size_t)n * kStageBytes) return false;
   const int rows = (d + num_sms - 1) / num_sms;                    // phase-D rows per CTA
   if (rows > kCompWarps) return false;
   // phase D: h of every kept slot plus at least two stages of W^down rows

@@ -94,6 +94,7 @@ extern "C" ace_status ace_moe_decode_noalloc(const ace_layer* layer, const void*
   if (!L.gamma || !L.w_router || !L.w_gate || !L.w_up || !L.w_down) return ACE_ERR_INVALID_ARG;
   if (check_fusion(L, (int)opts->fusion) != ACE_OK) return ACE_ERR_INVALID_ARG;
   const uintptr_t mis = reinterpret_cast<uintptr_t>(u) | reinterpret_cast<uintptr_t>(y) |
+                        reinterpret_cast<uintptr_t>(L.gamma) |
                         reinterpret_cast<uintptr_t>(L.w_router) |
                         reinterpret_cast<uintptr_t>(L.w_gate) |
                         reinterpret_cast<uintptr_t>(L.w_up) | reinterpret_cast<uintptr_t>(L.w_down);
