@@ -30,13 +30,6 @@
 #include "ace_common.cuh"
 #include "ace_internal.h"
 
-// How the W^down rows of phase D reach L2 ahead of use: 0 none, 1 plain
-// prefetches from the producer warp's idle lanes, 2 bulk prefetches queued
-// after the phase-C copies.
-#ifndef ACE_DECODE_PREFETCH
-#define ACE_DECODE_PREFETCH 2
-#endif
-
 namespace ace {
 namespace {
 
@@ -97,10 +90,11 @@ struct DecShared {
   float t_score[kMaxSlots];
   int t_keep[kMaxSlots];
   int t_pos[kMaxSlots];
-  float acc_d[kCompWarps][kDecodeMaxT];  // phase-D per-warp token sums
   uint32_t tok_mask[kMaxE];    // per expert: bit t set when token t kept a slot of it
   int e_base[kMaxE];           // per expert: its first slot
+  float acc_d[kCompWarps][kDecodeMaxT];  // phase-D per-warp token sums
   uint64_t in_bar;             // phase A: u, gamma and the router rows have landed
+  uint64_t h_bar;              // phase D: h of the kept slots has landed
   int abort;
 };
 
@@ -208,6 +202,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       mbar_init(&sh.empty_d[i], kCompWarps);
     }
     mbar_init(&sh.in_bar, 1);
+    mbar_init(&sh.h_bar, 1);
     fence_barrier_init();
     // one round trip for every input of phase A
     mbar_expect_tx(&sh.in_bar, (uint32_t)(NT * d * 2 + d * 4 + n_mine * d * 2));
@@ -390,21 +385,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const int p1 = (int)(((long long)P * (blockIdx.x + 1)) / G);
   const int SR = max(1, min(kMaxStageRows, kStageBytes / (4 * d)));  // row pairs per stage
   const int nstage_c = (p1 - p0 + SR - 1) / SR;
+  // phase-D geometry (its first stages are filled while phase C ends)
+  const int nrows = i1 - i0;  // <= kCompWarps: output row i0 + w belongs to warp w
+  const uint32_t dbytes = (uint32_t)(nrows * m * 2);
+  const size_t hbytes = ((size_t)S * m * 2 + 1023) & ~(size_t)1023;
+  const uint32_t dstage = (dbytes + 1023u) & ~1023u;
+  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(dsm);
+  uint8_t* ring_d = dsm + hbytes;
+  const int nring_d =
+      dstage ? (int)min((size_t)kRing, (a.dyn_bytes - 1024 - hbytes) / dstage) : 1;
+  // stages that lie inside phase C's ring (free once its last stage is
+  // consumed), clear of bf16(x) and the dot table that phase C still reads
+  const int n_pre = (nrows > 0 && hbytes + dstage <= (size_t)a.region)
+                        ? min(min(nring_d, U), (int)(((size_t)a.region - hbytes) / dstage))
+                        : 0;
   if (producer) {
-    if (lane > 0) {
-#if ACE_DECODE_PREFETCH == 1
-      // lanes 1..31: the phase-D rows of every surviving expert into L2, by
-      // plain prefetches (bulk prefetches would queue ahead of the ring's
-      // copies in the CTA's copy engine)
-      const int lines = (i1 - i0) * m * 2 / 128;
-      for (int q = lane - 1; q < U * lines; q += 31) {
-        const int ui = q / lines, ln = q - ui * lines;
-        const char* p =
-            reinterpret_cast<const char*>(a.wd + ((size_t)sh.uexp[ui] * d + i0) * m) + ln * 128;
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-      }
-#endif
-    } else {
+    if (lane == 0) {
       for (int st = 0; st < nstage_c; ++st) {
         const int slot = st % nring;
         if (!wait_bar(&sh.empty_c[slot], ((st / nring) & 1) ^ 1u, a, sh)) break;
@@ -423,15 +419,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
           p += run;
         }
       }
-#if ACE_DECODE_PREFETCH == 2
-      if (i0 < i1)  // the phase-D rows, after every ring copy of this CTA
-        for (int ui = 0; ui < U; ++ui) {
-          const char* p = reinterpret_cast<const char*>(a.wd + ((size_t)sh.uexp[ui] * d + i0) * m);
-          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p),
-                       "r"((uint32_t)((i1 - i0) * m * 2))
-                       : "memory");
+      if (n_pre > 0) {
+        // once every phase-C stage is consumed, the first W^down stages go in
+        bool ok = true;
+        for (int st = max(0, nstage_c - nring); st < nstage_c && ok; ++st)
+          ok = wait_bar(&sh.empty_c[st % nring], (st / nring) & 1, a, sh);
+        for (int ui = 0; ui < n_pre && ok; ++ui) {
+          mbar_expect_tx(&sh.full_d[ui], dbytes);
+          bulk_g2s(ring_d + (size_t)ui * dstage, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m,
+                   dbytes, &sh.full_d[ui]);
         }
-#endif
+      }
     }
   } else {
     // two groups of 8 warps take alternate stages (the ring is even, so a
@@ -495,37 +493,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       a.h[(size_t)(s0 + x) * m + j] = __float2bfloat16_rn(silu(gs) * us);
     }
   }
+  // h is read back by bulk copies (the async proxy) after the grid barrier
+  asm volatile("fence.proxy.async.global;" ::: "memory");
   stamp(a, 4);
   if (!grid_barrier(a, sh, 2)) return;
   stamp(a, 5);
 
   // ---------------------------------------------------------- phase D
-  // shared memory: h of the kept slots, then a ring of stages that each hold
-  // the CTA's output rows of one surviving expert's W^down
-  const int nrows = i1 - i0;  // <= kCompWarps: output row i0 + w belongs to warp w
-  const uint32_t dbytes = (uint32_t)(nrows * m * 2);
-  const size_t hbytes = ((size_t)S * m * 2 + 1023) & ~(size_t)1023;
-  const uint32_t dstage = (dbytes + 1023u) & ~1023u;
-  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(dsm);
-  uint8_t* ring_d = dsm + hbytes;
-  const int nring_d =
-      dstage ? (int)min((size_t)kRing, (a.dyn_bytes - 1024 - hbytes) / dstage) : 1;
-  for (int q = threadIdx.x; q < S * m / 8; q += blockDim.x)
-    reinterpret_cast<uint4*>(hs)[q] = reinterpret_cast<const uint4*>(a.h)[q];
-  __syncthreads();
+  // shared memory: h of the kept slots (one bulk copy), then a ring of
+  // stages that each hold the CTA's output rows of one surviving expert's
+  // W^down; the first n_pre stages were issued at the end of phase C
   if (nrows > 0) {
     if (producer) {
-      if (lane == 0)
-        for (int ui = 0; ui < U; ++ui) {
+      if (lane == 0) {
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        mbar_expect_tx(&sh.h_bar, (uint32_t)(S * m * 2));
+        bulk_g2s(hs, a.h, (uint32_t)(S * m * 2), &sh.h_bar);
+        for (int ui = n_pre; ui < U; ++ui) {
           const int slot = ui % nring_d;
           if (!wait_bar(&sh.empty_d[slot], ((ui / nring_d) & 1) ^ 1u, a, sh)) break;
           mbar_expect_tx(&sh.full_d[slot], dbytes);
           bulk_g2s(ring_d + (size_t)slot * dstage, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m,
                    dbytes, &sh.full_d[slot]);
         }
+      }
     } else {
       if (lane < NT) sh.acc_d[warp][lane] = 0.f;
       __syncwarp();
+      if (!wait_bar(&sh.h_bar, 0, a, sh)) return;
       for (int ui = 0; ui < U; ++ui) {
         const int slot = ui % nring_d;
         if (!wait_bar(&sh.full_d[slot], (ui / nring_d) & 1, a, sh)) break;
