@@ -542,6 +542,105 @@ def run_decode(args, w, ws_n, rank, local):
     }
 
 
+def run_stack(args, w, ws_n, rank, local):
+    """The 48 layers chained through ace_moe_stack_forward: one step is one
+    pass of T tokens through every layer (a per-token latency of the MoE
+    layers), captured once in a CUDA graph and replayed per step."""
+    from token_dynamic_expert_b200 import ace
+    dev = torch.device("cuda", local)
+    st = setup_decode(w, dev, n_layers=args.layers)
+    nl = st["n_layers"]
+    stream = torch.cuda.Stream(dev)
+    u, y = st["u"][0], torch.empty_like(st["u"][0])
+    ws = ace.alloc_workspace(ace.ace_stack_workspace_size(st["L"], w.T), dev)
+    # the chain's own routing, layer by layer (untimed): surviving experts
+    lws = ace.alloc_workspace(ace.ace_workspace_size(st["L"][0], w.T), dev)
+    x, touched, kept = u, [], []
+    for l in range(nl):
+        dbg = ace.DebugOut(w.T, w.k, w.E, dev)
+        out = torch.empty_like(u)
+        ace.ace_moe_forward(st["L"][l], x, st["taus"][l], out, lws, dbg=dbg.c)
+        off = dbg.expert_offsets.cpu().numpy()
+        touched.append(int((np.diff(off) > 0).sum()))
+        kept.append(int(dbg.n_kept.item()))
+        x = out
+    ace.ace_moe_stack_forward(st["L"], u, st["taus"], y, ws, stream=stream)
+    stream.synchronize()
+    if not torch.equal(y, x):
+        raise RuntimeError("stack output differs from the layer-by-layer chain")
+    with torch.cuda.stream(stream):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            ace.ace_moe_stack_forward(st["L"], u, st["taus"], y, ws, stream=stream)
+        for _ in range(args.warmup):
+            g.replay()
+    stream.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(ws_n)
+    with ClockSampler(local) as clk, torch.cuda.stream(stream):
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            g.replay()
+            evs[i][1].record(stream)
+        stream.synchronize()
+    barrier(ws_n)
+    t_steps = [a.elapsed_time(b) for a, b in evs]
+    spread = step_spread(t_steps, w.name)
+    value, total_ms = replica_throughput(ws_n, args.steps, w.T, sum(t_steps))
+    ms_step = total_ms / args.steps
+    code, flags = ace.ace_read_status(ws, stream=stream)
+    if code != ace.ACE_OK:
+        raise RuntimeError("device status %s flags %#x" % (ace.ace_status_str(code), flags))
+    del g
+    pk = peaks()
+    surv = sum(touched) * 3 * w.d * w.m * 2
+    router = nl * w.E * w.d * 2
+    gbs = (surv + router) / (ms_step / 1e3) / 1e9
+    # e2e: host tokens in, host outputs back, the plain API call
+    u_host = u.cpu().pin_memory()
+    y_host = torch.empty_like(u_host).pin_memory()
+    e2e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            e2e[i][0].record(stream)
+            u.copy_(u_host, non_blocking=True)
+            ace.ace_moe_stack_forward(st["L"], u, st["taus"], y, ws, stream=stream)
+            y_host.copy_(y, non_blocking=True)
+            e2e[i][1].record(stream)
+        stream.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e), ws_n)
+    nbytes = w.T * w.d * 2
+    return {
+        "metric": METRIC, "value": value,
+        "unit": "tokens/s (through all %d chained MoE layers)" % nl,
+        "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) weights, N(0,1) tokens)",
+        "config": {"workload": w.name, "tokens_per_step": w.T, "layers": nl, "hidden": w.d,
+                   "experts": w.E, "expert_ffn": w.m, "top_k": w.k, "skip_rate": w.skip,
+                   "tau": "per layer, quantile of a %d-token pool" % w.pool,
+                   "mean_kept_slots": float(np.mean(kept)),
+                   "mean_surviving_experts": float(np.mean(touched)),
+                   "us_per_layer": ms_step * 1e3 / nl, "tpot_proxy_ms": ms_step,
+                   "parallelism": "replicas" if ws_n > 1 else "single", "step_ms": spread,
+                   "launch": "ace_moe_stack_forward captured in one CUDA graph",
+                   "l2": "weights of %d layers (%.1f GB) exceed L2; no flush" % (
+                       nl, nl * 3 * w.E * w.d * w.m * 2 / 1e9)},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                     "kernel": "k_decode x %d layers (whole step)" % nl,
+                     "algorithmic_bytes": surv + router, "kernel_ms": ms_step,
+                     "peak_source": pk["source"]},
+        "clocks": clk.summary(),
+        "e2e": {"value": ws_n * args.steps * w.T / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+                "launch": "plain API call per step"},
+        "gpu_launches": nl * args.steps,
+    }
+
+
 # ---------------------------------------------------------- CPU baselines
 def _oracle_inputs(st):
     """Host copies in the oracle's input types (converted once, untimed)."""
@@ -604,16 +703,20 @@ def run_reference(args, w, rate):
         oracle.moe_forward(layer, u[:n], tau, amax, amax)
     dt = time.perf_counter() - t0
     val = args.steps * n / dt
-    return {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+    unit, sample = "tokens/s", "%d of %d tokens per step" % (n, w.T)
+    if w.name.startswith("stack"):  # one layer timed; the chain costs layers times as much
+        val /= w.layers
+        unit = "tokens/s (through all %d chained MoE layers)" % w.layers
+        sample += "; one layer timed, the %d-layer rate is its rate / %d" % (w.layers, w.layers)
+    return {"metric": METRIC, "value": val, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "tokens": w.T, "hidden": w.d, "experts": w.E,
                        "expert_ffn": w.m, "top_k": w.k, "skip_rate": rate},
-            "cpu_baseline": {"value": val, "unit": "tokens/s", "kind": "oracle",
-                             "cores": oracle.threads(),
-                             "sample": "%d of %d tokens per step" % (n, w.T)},
-            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+            "cpu_baseline": {"value": val, "unit": unit, "kind": "oracle",
+                             "cores": oracle.threads(), "sample": sample},
+            "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
@@ -624,7 +727,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="prefill_1024",
                     choices=["prefill_1024", "prefill_8192_e256", "sweep_4096", "decode_bs1",
-                             "decode_bs8"])
+                             "decode_bs8", "stack_bs1", "stack_bs8"])
     ap.add_argument("--rate", type=float, default=None, help="override the skip rate")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -644,8 +747,9 @@ def main():
 
     from token_dynamic_expert_b200 import build as _b  # noqa: F401  (the .so ships prebuilt)
     ws_n, rank, local = dist_setup(args.gpus)
-    if args.workload.startswith("decode"):
-        out = run_decode(args, w, ws_n, rank, local)
+    if args.workload.startswith("decode") or args.workload.startswith("stack"):
+        run = run_decode if args.workload.startswith("decode") else run_stack
+        out = run(args, w, ws_n, rank, local)
         if rank == 0:
             print(json.dumps(out), flush=True)
         if ws_n > 1:

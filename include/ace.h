@@ -198,6 +198,33 @@ ACE_API ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T,
                            size_t ws_bytes, ace_debug_out* dbg, void* stream);
 
 /* ------------------------------------------------------------------------
+ * ace_stack_workspace_size -- bytes of workspace ace_moe_stack_forward
+ *   needs for the n_layers layers (same d and dtype) and up to max_tokens
+ *   tokens; 0 for invalid layers.
+ * ---------------------------------------------------------------------- */
+ACE_API size_t ace_stack_workspace_size(const ace_layer* layers, int n_layers, int max_tokens);
+
+/* ------------------------------------------------------------------------
+ * ace_moe_stack_forward -- n_layers MoE layers in sequence, the output of
+ *   each the input of the next (u_{l+1} = y_l), as in a decode step through
+ *   the model's MoE layers ([ACE] "Efficiency Results", Table 7: the
+ *   per-token latency over every layer).  The paper has no entry point of
+ *   its own for this; it is the layer forward repeated, each layer with its
+ *   own options opts[l] (tau per layer).  Every layer's forward is exactly
+ *   ace_moe_forward's (same kernels, same results), so the stack equals
+ *   n_layers calls with the outputs fed back.  The intermediate
+ *   activations alternate between two [T][d] buffers inside ws; u (device)
+ *   [T][d] is only read, y (device) [T][d] receives the last layer's
+ *   output; they must not overlap.  The status word (ace_read_status on
+ *   ws) holds the flags of every layer of the call.  Asynchronous; no
+ *   allocation, no synchronisation, so it can be captured in a CUDA graph.
+ *   Argument errors (any layer's) return before anything is launched.
+ * ---------------------------------------------------------------------- */
+ACE_API ace_status ace_moe_stack_forward(const ace_layer* layers, int n_layers, const void* u,
+                                         int T, const ace_fwd_opts* opts, void* y, void* ws,
+                                         size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * ace_moe_scores -- only the routing half of the forward: fused scores
  *   c (opts->fusion; the gate alone under ACE_FUSE_MAX when layer->amax,
  *   a_gsp and a_rcr are all NULL) of every slot,

@@ -153,3 +153,26 @@ def test_fusion_rules_need_their_tables(ace, fusion, tables, ok):
     opts = ace.ace_fwd_opts(tau=0.1, renorm_topk=1, fusion=fusion, eps_rms=1e-6)
     want = ace.ACE_ERR_WORKSPACE if ok else ace.ACE_ERR_INVALID_ARG
     assert _fwd(ace, L, opts=opts, ws_bytes=1024) == want
+
+
+def test_stack_rejects_bad_calls(ace):
+    Ls = (ace.ace_layer * 3)(_fake_layer(ace), _fake_layer(ace), _fake_layer(ace))
+    opts = (ace.ace_fwd_opts * 3)(*[ace.ace_fwd_opts(tau=0.1, renorm_topk=1, fusion=0,
+                                                     eps_rms=1e-6)] * 3)
+    f = ace.lib().ace_moe_stack_forward
+    ok = dict(u=0x20000, y=0x40000, ws=0x80000, nb=1 << 30)
+    assert ace.lib().ace_stack_workspace_size(Ls, 3, 8) >= 2 * 8 * 256 * 2
+    assert ace.lib().ace_stack_workspace_size(Ls, 0, 8) == 0
+    assert f(Ls, 0, ok["u"], 4, opts, ok["y"], ok["ws"], ok["nb"], None) == ace.ACE_ERR_INVALID_ARG
+    assert f(Ls, 3, ok["u"], 4, None, ok["y"], ok["ws"], ok["nb"], None) == ace.ACE_ERR_INVALID_ARG
+    assert f(Ls, 3, ok["u"], 4, opts, ok["u"] + 64, ok["ws"], ok["nb"], None) == \
+        ace.ACE_ERR_INVALID_ARG                                        # u and y overlap
+    assert f(Ls, 3, ok["u"], 4, opts, ok["y"], ok["ws"], 1024, None) == ace.ACE_ERR_WORKSPACE
+    assert f(Ls, 3, ok["u"], 4, opts, ok["y"], ok["ws"] + 16, ok["nb"], None) == \
+        ace.ACE_ERR_WORKSPACE
+    bad = (ace.ace_layer * 3)(_fake_layer(ace), _fake_layer(ace, d=512), _fake_layer(ace))
+    assert f(bad, 3, ok["u"], 4, opts, ok["y"], ok["ws"], ok["nb"], None) == \
+        ace.ACE_ERR_INVALID_ARG                                        # layers of different d
+    opts[2].fusion = 1                                                 # min without view tables
+    assert f(Ls, 3, ok["u"], 4, opts, ok["y"], ok["ws"], ok["nb"], None) == \
+        ace.ACE_ERR_INVALID_ARG

@@ -72,6 +72,11 @@ _lib.ace_tables_workspace_size.restype = ctypes.c_size_t
 _lib.ace_build_tables.argtypes = [_P(ace_layer), ctypes.c_int, _P(ace_table_opts), _vp, _vp, _vp,
                                   _vp, _vp, ctypes.c_size_t, _vp]
 _lib.ace_build_tables.restype = ctypes.c_int
+_lib.ace_stack_workspace_size.argtypes = [_P(ace_layer), ctypes.c_int, ctypes.c_int]
+_lib.ace_stack_workspace_size.restype = ctypes.c_size_t
+_lib.ace_moe_stack_forward.argtypes = [_P(ace_layer), ctypes.c_int, _vp, ctypes.c_int,
+                                       _P(ace_fwd_opts), _vp, _vp, ctypes.c_size_t, _vp]
+_lib.ace_moe_stack_forward.restype = ctypes.c_int
 _lib.ace_tau_workspace_size.argtypes = []
 _lib.ace_tau_workspace_size.restype = ctypes.c_size_t
 _lib.ace_tau_quantile.argtypes = [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp,
@@ -187,6 +192,26 @@ def ace_moe_decode_noalloc(layer, u, tau, y, renorm=True, eps_rms=1e-6, stream=N
     code = _lib.ace_moe_decode_noalloc(ctypes.byref(layer), _ptr(u), int(u.shape[0]),
                                        ctypes.byref(opts), _ptr(y), _stream(stream))
     _check(code, "ace_moe_decode_noalloc")
+    return y
+
+
+def ace_stack_workspace_size(layers, max_tokens):
+    arr = (ace_layer * len(layers))(*layers)
+    return int(_lib.ace_stack_workspace_size(arr, len(layers), int(max_tokens)))
+
+
+def ace_moe_stack_forward(layers, u, taus, y, ws, renorm=True, eps_rms=1e-6, stream=None,
+                          fusion="max"):
+    """len(layers) layers in sequence, each output the next input; taus[l]
+    is layer l's threshold.  See include/ace.h."""
+    n = len(layers)
+    arr = (ace_layer * n)(*layers)
+    opts = (ace_fwd_opts * n)(*[ace_fwd_opts(tau=float(t), renorm_topk=int(bool(renorm)),
+                                             fusion=_fusion(fusion), eps_rms=float(eps_rms))
+                                for t in taus])
+    code = _lib.ace_moe_stack_forward(arr, n, _ptr(u), int(u.shape[0]), opts, _ptr(y), _ptr(ws),
+                                      ws.numel(), _stream(stream))
+    _check(code, "ace_moe_stack_forward")
     return y
 
 

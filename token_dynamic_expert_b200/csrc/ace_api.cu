@@ -234,9 +234,15 @@ size_t ace_workspace_size(const ace_layer* layer, int max_tokens) {
   return fwd_layout(*layer, max_tokens, device_sm_count()).total;
 }
 
-ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T, const ace_fwd_opts* opts,
-                           void* y, void* ws, size_t ws_bytes, ace_debug_out* dbg,
-                           void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The forward of one layer.  keep_status: leave the status word as it is
+// (a layer of a stack adds its flags to those of the layers before it).
+ace_status forward_impl(const ace_layer* layer, const void* u, int T, const ace_fwd_opts* opts,
+                        void* y, void* ws, size_t ws_bytes, ace_debug_out* dbg, void* stream,
+                        bool keep_status) {
   ace_status st = check_common(layer, u, T, opts, ws, true);
   if (st != ACE_OK) return st;
   if (T > 0 && (!y || !aligned(y, 16))) return ACE_ERR_INVALID_ARG;
@@ -253,7 +259,10 @@ ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T, const a
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // status word (offset 0), the decode kernel's grid-barrier words (byte 64)
   // and the routing CTAs' completion count (byte 128)
-  ACE_CK(cudaMemsetAsync(at<void>(ws, ly.status), 0, 256, s));
+  if (keep_status)
+    ACE_CK(cudaMemsetAsync(at<uint8_t>(ws, ly.status) + 64, 0, 192, s));
+  else
+    ACE_CK(cudaMemsetAsync(at<void>(ws, ly.status), 0, 256, s));
   if (T == 0) return ACE_OK;
   cudaEvent_t ev_b = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_begin) : nullptr;
   cudaEvent_t ev_m = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_mid) : nullptr;
@@ -291,6 +300,83 @@ ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T, const a
     if (dbg->logits && decode &&
         !cp(dbg->logits, ly.part, (size_t)T * L.E * 4))
       return ACE_ERR_CUDA;
+  }
+  return ACE_OK;
+}
+
+// Stack workspace: [the largest layer workspace | activations A | B], each
+// 256-byte aligned; the layer workspace starts at 0 so its status word is
+// the stack's.
+struct StackLayout {
+  size_t layer_ws, act0, act1, total;
+};
+
+bool stack_layout(const ace_layer* layers, int n, int max_tokens, int num_sms, StackLayout* o) {
+  if (!layers || n < 1 || max_tokens < 0) return false;
+  size_t lw = 0;
+  for (int l = 0; l < n; ++l) {
+    if (check_layer(&layers[l], true) != ACE_OK) return false;
+    if (layers[l].d != layers[0].d || layers[l].dtype != layers[0].dtype) return false;
+    const size_t b = fwd_layout(layers[l], max_tokens, num_sms).total;
+    if (b > lw) lw = b;
+  }
+  const size_t act = align_up((size_t)(max_tokens > 0 ? max_tokens : 1) * layers[0].d *
+                                  esize(layers[0].dtype), 256);
+  o->layer_ws = align_up(lw, 256);
+  o->act0 = o->layer_ws;
+  o->act1 = o->act0 + act;
+  o->total = o->act1 + act;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T, const ace_fwd_opts* opts,
+                           void* y, void* ws, size_t ws_bytes, ace_debug_out* dbg,
+                           void* stream) {
+  return forward_impl(layer, u, T, opts, y, ws, ws_bytes, dbg, stream, false);
+}
+
+size_t ace_stack_workspace_size(const ace_layer* layers, int n_layers, int max_tokens) {
+  StackLayout ly;
+  if (!stack_layout(layers, n_layers, max_tokens, device_sm_count(), &ly)) return 0;
+  return ly.total;
+}
+
+ace_status ace_moe_stack_forward(const ace_layer* layers, int n_layers, const void* u, int T,
+                                 const ace_fwd_opts* opts, void* y, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  if (!layers || n_layers < 1 || !opts || T < 0) return ACE_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256)) return ACE_ERR_WORKSPACE;
+  for (int l = 0; l < n_layers; ++l) {
+    if (check_layer(&layers[l], true) != ACE_OK) return check_layer(&layers[l], true);
+    if (layers[l].d != layers[0].d || layers[l].dtype != layers[0].dtype)
+      return ACE_ERR_INVALID_ARG;
+    const ace_status fs = check_fusion(layers[l], opts[l].fusion);
+    if (fs != ACE_OK) return fs;
+  }
+  if (T > 0 && (!u || !y || !aligned(u, 16) || !aligned(y, 16))) return ACE_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)T * layers[0].d * esize(layers[0].dtype);
+  if (T > 0) {
+    const uint8_t *ub = (const uint8_t*)u, *yb = (const uint8_t*)y;
+    if (ub < yb + bytes && yb < ub + bytes) return ACE_ERR_INVALID_ARG;
+  }
+  StackLayout ly;
+  if (!stack_layout(layers, n_layers, T, device_sm_count(), &ly)) return ACE_ERR_INVALID_ARG;
+  if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ACE_CK(cudaMemsetAsync(ws, 0, 4, s));  // the status word, once for the stack
+  if (T == 0) return ACE_OK;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const void* in = u;
+  for (int l = 0; l < n_layers; ++l) {
+    void* out = l == n_layers - 1 ? y : base + ((l & 1) ? ly.act1 : ly.act0);
+    const ace_status st = forward_impl(&layers[l], in, T, &opts[l], out, ws, ly.layer_ws, nullptr,
+                                       stream, true);
+    if (st != ACE_OK) return st;
+    in = out;
   }
   return ACE_OK;
 }

@@ -65,6 +65,12 @@ WORKLOADS = {
                            bias=False, skip=0.6, skip_of="slots", layers=48, pool=4096),
     "decode_bs8": Workload("decode_bs8", T=8, d=2048, E=128, m=768, k=8, dtype="bf16",
                            bias=False, skip=0.6, skip_of="slots", layers=48, pool=4096),
+    # the same 48 layers chained (each layer's output the next one's input):
+    # one step is a token step through the model's MoE layers
+    "stack_bs1": Workload("stack_bs1", T=1, d=2048, E=128, m=768, k=8, dtype="bf16",
+                          bias=False, skip=0.6, skip_of="slots", layers=48, pool=4096),
+    "stack_bs8": Workload("stack_bs8", T=8, d=2048, E=128, m=768, k=8, dtype="bf16",
+                          bias=False, skip=0.6, skip_of="slots", layers=48, pool=4096),
     # wider pool: 256 experts of FFN 512, 4 x 2048 tokens, router bias N(0,1)
     # (skewed expert load), 50% skip
     "prefill_8192_e256": Workload("prefill_8192_e256", T=8192, d=2048, E=256, m=512, k=8,
