@@ -427,6 +427,33 @@ def setup_decode(w, device, n_layers=None):
                 tables_ms=tables_ms, threshold_ms=threshold_ms, n_layers=nl)
 
 
+DECODE_PHASES = ["start", "x ready", "barrier 1", "slots", "gate/up done", "barrier 2", "end",
+                 "rms sum (token 0)"]
+
+
+def decode_phases(st, w, stream, reps=5):
+    """The decode kernel's per-CTA phase stamps (the debug trace of
+    ace_moe_forward), layer 0, L2 flushed before each of `reps` launches:
+    median over CTAs of each stamp, in microseconds from the first CTA's
+    start, from the last launch."""
+    from token_dynamic_expert_b200 import ace
+    import ctypes
+    dev = st["u"][0].device
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    tr = torch.zeros(nsm, 8, dtype=torch.int64, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            flush.fill_(1)
+            dbg = ace.ace_debug_out(trace=ctypes.c_void_p(tr.data_ptr()))
+            ace.ace_moe_forward(st["L"][0], st["u"][0], st["taus"][0], st["y"][0], st["ws"],
+                                dbg=dbg, stream=stream)
+        stream.synchronize()
+    t = tr.cpu().numpy().astype(np.float64)
+    rel = (t - t[:, 0].min()) / 1e3
+    return {n: round(float(np.median(rel[:, i])), 2) for i, n in enumerate(DECODE_PHASES)}
+
+
 def run_decode(args, w, ws_n, rank, local):
     from token_dynamic_expert_b200 import ace
     dev = torch.device("cuda", local)
@@ -488,6 +515,7 @@ def run_decode(args, w, ws_n, rank, local):
     router = nl * w.E * w.d * 2
     kernel_gbs = (surv + router) / (k_ms / 1e3) / 1e9
     step_gbs = (surv + router) / (ms_step / 1e3) / 1e9
+    phases = decode_phases(st, w, stream) if args.trace else None
     # e2e: host tokens in, host outputs back, every layer, plain API calls
     u_host = [x.cpu().pin_memory() for x in st["u"]]
     y_host = [torch.empty_like(x).pin_memory() for x in u_host]
@@ -530,6 +558,7 @@ def run_decode(args, w, ws_n, rank, local):
                     "tables": {"layers": nl, "experts": w.E, "ms": st["tables_ms"],
                                "ms_per_layer": st["tables_ms"] / nl,
                                "includes": "GSP Grams, power iteration (sigma, 200 steps), RCR"},
+                    **({"decode_phases_us": phases} if phases else {}),
                     "thresholds": {"layers": nl, "pool_tokens": max(w.pool, 1),
                                    "ms": st["threshold_ms"],
                                    "includes": "per layer: ace_moe_scores over the pool, "
@@ -733,6 +762,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="decode: number of layers (default: the workload's 48)")
+    ap.add_argument("--trace", action="store_true",
+                    help="decode: add the decode kernel's phase timeline (debug trace)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     w = workloads.WORKLOADS[args.workload]
