@@ -11,11 +11,13 @@
 //   phase B  every CTA, redundantly: top-k, gates, ACE scores and the skip
 //            mask ([ACE] "3. Conservative Fusion", top-1 always kept), the
 //            kept slots sorted by (expert, token), the distinct experts
-//   phase C  gate/up ([ACE] eq. f): the CTA's contiguous share of the
-//            surviving (expert, row) pairs streams through a shared-memory
+//   phase C  gate/up ([ACE] eq. f): the surviving (expert, row) pairs, in
+//            stages of 4 row pairs that the CTAs take from a grid-wide
+//            counter as their rings free up, stream through a shared-memory
 //            ring by TMA bulk copies issued from a producer warp; 16 warps
-//            form h = SiLU(x W^gate) (.) x W^up for the expert's kept tokens;
-//            meanwhile the W^down rows the CTA will need go to L2
+//            form h = SiLU(x W^gate) (.) x W^up for the expert's kept tokens
+//            and write it out; once the ring drains, the first W^down stages
+//            of phase D are issued
 //   -- grid barrier --
 //   phase D  down + combine: the CTA's output rows of every surviving
 //            expert's W^down stream through the ring; warp w owns output row
@@ -95,6 +97,9 @@ struct DecShared {
   float acc_d[kCompWarps][kDecodeMaxT];  // phase-D per-warp token sums
   uint64_t in_bar;             // phase A: u, gamma and the router rows have landed
   uint64_t h_bar;              // phase D: h of the kept slots has landed
+  int slot_stage[kRing];       // phase C: the stage a ring slot holds (-1: no more)
+  float xchg[2][kMaxStageRows][2 * kDecodeMaxT];  // phase C: second half-row dots
+  uint64_t xfull[2][kMaxStageRows], xempty[2][kMaxStageRows];  // ... and their handover
   int abort;
 };
 
@@ -189,7 +194,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   float* gs = reinterpret_cast<float*>(dsm + (size_t)NT * d * 6);
   __nv_bfloat16* wrs = reinterpret_cast<__nv_bfloat16*>(dsm + (size_t)NT * d * 6 + (size_t)d * 4);
   __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(dsm + a.region);  // bf16(x)
-  float* part = reinterpret_cast<float*>(dsm + a.region + (size_t)NT * a.d * 2);
   const int n_router_warps = (E + G - 1) / G;
   // router rows of this CTA: experts blockIdx.x + G * r, r < n_mine
   const int n_mine = (int)blockIdx.x < E ? min(n_router_warps, (E - 1 - (int)blockIdx.x) / G + 1) : 0;
@@ -203,6 +207,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     }
     mbar_init(&sh.in_bar, 1);
     mbar_init(&sh.h_bar, 1);
+    for (int g = 0; g < 2; ++g)
+      for (int r = 0; r < kMaxStageRows; ++r) {
+        mbar_init(&sh.xfull[g][r], 1);
+        mbar_init(&sh.xempty[g][r], 1);
+      }
     fence_barrier_init();
     // one round trip for every input of phase A
     mbar_expect_tx(&sh.in_bar, (uint32_t)(NT * d * 2 + d * 4 + n_mine * d * 2));
@@ -381,10 +390,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const int rows_per_cta = (d + G - 1) / G;  // phase-D output rows per CTA (<= 16)
   const int i0 = min(d, (int)blockIdx.x * rows_per_cta), i1 = min(d, i0 + rows_per_cta);
   const int P = U * m;  // surviving (expert, row) pairs
-  const int p0 = (int)(((long long)P * blockIdx.x) / G);
-  const int p1 = (int)(((long long)P * (blockIdx.x + 1)) / G);
   const int SR = max(1, min(kMaxStageRows, kStageBytes / (4 * d)));  // row pairs per stage
-  const int nstage_c = (p1 - p0 + SR - 1) / SR;
+  const int n_stages = (P + SR - 1) / SR;
   // phase-D geometry (its first stages are filled while phase C ends)
   const int nrows = i1 - i0;  // <= kCompWarps: output row i0 + w belongs to warp w
   const uint32_t dbytes = (uint32_t)(nrows * m * 2);
@@ -395,16 +402,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const int nring_d =
       dstage ? (int)min((size_t)kRing, (a.dyn_bytes - 1024 - hbytes) / dstage) : 1;
   // stages that lie inside phase C's ring (free once its last stage is
-  // consumed), clear of bf16(x) and the dot table that phase C still reads
+  // consumed), clear of bf16(x) that phase C still reads
   const int n_pre = (nrows > 0 && hbytes + dstage <= (size_t)a.region)
                         ? min(min(nring_d, U), (int)(((size_t)a.region - hbytes) / dstage))
                         : 0;
   if (producer) {
     if (lane == 0) {
-      for (int st = 0; st < nstage_c; ++st) {
-        const int slot = st % nring;
-        if (!wait_bar(&sh.empty_c[slot], ((st / nring) & 1) ^ 1u, a, sh)) break;
-        const int pa = p0 + st * SR, pb = min(p1, pa + SR);
+      // stages are taken from a grid-wide counter as the ring frees up, so
+      // CTAs that run ahead take more of them
+      uint32_t* stage_ctr = a.bar_count + 1;
+      int ls = 0;  // this CTA's stages so far
+      bool ok = true;
+      for (;; ++ls) {
+        const int slot = ls % nring;
+        if (!(ok = wait_bar(&sh.empty_c[slot], ((ls / nring) & 1) ^ 1u, a, sh))) break;
+        const int gst = (int)atomicAdd(stage_ctr, 1u);
+        if (gst >= n_stages) break;
+        sh.slot_stage[slot] = gst;
+        const int pa = gst * SR, pb = min(P, pa + SR);
         mbar_expect_tx(&sh.full_c[slot], (uint32_t)((pb - pa) * d * 4));
         uint8_t* sg = ring + slot * kStageBytes;
         uint8_t* su = sg + kStageBytes / 2;
@@ -419,10 +434,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
           p += run;
         }
       }
-      if (n_pre > 0) {
+      // end marks for both consumer groups: this CTA's stages ls and ls + 1
+      for (int e = 0; e < 2 && ok; ++e) {
+        const int slot = (ls + e) % nring;
+        if (e == 1) ok = wait_bar(&sh.empty_c[slot], (((ls + 1) / nring) & 1) ^ 1u, a, sh);
+        if (ok) {
+          sh.slot_stage[slot] = -1;
+          mbar_arrive(&sh.full_c[slot]);
+        }
+      }
+      if (ok && n_pre > 0) {
         // once every phase-C stage is consumed, the first W^down stages go in
-        bool ok = true;
-        for (int st = max(0, nstage_c - nring); st < nstage_c && ok; ++st)
+        for (int st = max(0, ls - nring); st < ls && ok; ++st)
           ok = wait_bar(&sh.empty_c[st % nring], (st / nring) & 1, a, sh);
         for (int ui = 0; ui < n_pre && ok; ++ui) {
           mbar_expect_tx(&sh.full_d[ui], dbytes);
@@ -433,66 +456,92 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     }
   } else {
     // two groups of 8 warps take alternate stages (the ring is even, so a
-    // slot always belongs to the same group); in a group, warp
-    // 2r + mat reduces row r of the stage against W^gate (mat 0) or W^up
-    // (mat 1) for every kept token of the row's expert.  The dots go to the
-    // CTA's table; each warp releases the stage on its own.
+    // slot always belongs to the same group).  In a group, warps 2r and
+    // 2r + 1 take row pair r of the stage, each over half of the hidden
+    // size, for every kept token of the pair's expert: the gate and up dots.
+    // The second warp hands its halves over through shared memory; the
+    // first forms h = SiLU(gate) * up and writes it.
     const int grp = warp >> 3, wi = warp & 7;
-    const int rpos = wi >> 1, mat = wi & 1;
-    const int nv = d / 8;
-    for (int st = grp; st < nstage_c; st += 2) {
-      const int slot = st % nring;
-      if (!wait_bar(&sh.full_c[slot], (st / nring) & 1, a, sh)) break;
-      const int pa = p0 + st * SR, nr = min(p1, pa + SR) - pa;
-      if (rpos < nr) {
-        const int p = pa + rpos;
-        const int ui = p / m;
-        const int s0 = sh.ufirst[ui], s1 = sh.ufirst[ui + 1];
-        const uint4* wrow = reinterpret_cast<const uint4*>(
-            ring + slot * kStageBytes + mat * (kStageBytes / 2) + (size_t)rpos * d * 2);
-        float* trow = part + (size_t)(p - p0) * NT * 2;
-        for (int sg = s0; sg < s1; sg += 4) {  // the expert's kept tokens, 4 at a time
-          const int nt = min(4, s1 - sg);
-          const uint4* xt[4];
+    const int r = wi >> 1, half = wi & 1;
+    const int hv = d / 16;  // 16-byte chunks per half row
+    uint32_t kx = 0;        // handovers of this warp pair so far
+    for (int ls = grp;; ls += 2) {
+      const int slot = ls % nring;
+      if (!wait_bar(&sh.full_c[slot], (ls / nring) & 1, a, sh)) break;
+      const int gst = sh.slot_stage[slot];
+      if (gst < 0) break;
+      const int pa = gst * SR, nr = min(P, pa + SR) - pa;
+      if (r < nr) {
+        const int p = pa + r;
+        const int ui = p / m, j = p - ui * m;
+        const int s0 = sh.ufirst[ui], nt = sh.ufirst[ui + 1] - s0;  // <= NT
+        const uint4* wg =
+            reinterpret_cast<const uint4*>(ring + slot * kStageBytes + (size_t)r * d * 2) +
+            half * hv;
+        const uint4* wu = reinterpret_cast<const uint4*>(ring + slot * kStageBytes +
+                                                         kStageBytes / 2 + (size_t)r * d * 2) +
+                          half * hv;
+        int xo[NT];  // each kept token's row of bf16(x), in 16-byte chunks
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            xt[q] = reinterpret_cast<const uint4*>(xb + (size_t)sh.slot_t[sg + min(q, nt - 1)] * d);
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
-          for (int c = lane; c < nv; c += 32) {
-            float w8[8];
-            bf16x8_to_f32(wrow[c], w8);
+        for (int q = 0; q < NT; ++q) xo[q] = (q < nt ? sh.slot_t[s0 + q] : 0) * (d / 8) + half * hv;
+        float ga[NT], ua[NT];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (q >= nt) break;
+        for (int q = 0; q < NT; ++q) ga[q] = ua[q] = 0.f;
+        const uint4* xq = reinterpret_cast<const uint4*>(xb);
+        for (int c = lane; c < hv; c += 32) {
+          float w1[8], w2[8];
+          bf16x8_to_f32(wg[c], w1);
+          bf16x8_to_f32(wu[c], w2);
+#pragma unroll
+          for (int q = 0; q < NT; ++q) {
+            if (q < nt) {
               float xv[8];
-              bf16x8_to_f32(xt[q][c], xv);
+              bf16x8_to_f32(xq[xo[q] + c], xv);
 #pragma unroll
-              for (int cc = 0; cc < 8; ++cc) acc[q] = fmaf(w8[cc], xv[cc], acc[q]);
+              for (int cc = 0; cc < 8; ++cc) {
+                ga[q] = fmaf(w1[cc], xv[cc], ga[q]);
+                ua[q] = fmaf(w2[cc], xv[cc], ua[q]);
+              }
             }
           }
+        }
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (q >= nt) break;
-            const float r = warp_sum(acc[q]);
-            if (lane == 0) trow[(sg - s0 + q) * 2 + mat] = r;
+        for (int q = 0; q < NT; ++q) {
+          if (q < nt) {
+            ga[q] = warp_sum(ga[q]);
+            ua[q] = warp_sum(ua[q]);
           }
         }
+        float* xg = &sh.xchg[grp][r][0];
+        if (half == 1) {  // hand the second half over (one buffer per pair)
+          if (!wait_bar(&sh.xempty[grp][r], (kx & 1u) ^ 1u, a, sh)) break;
+          if (lane == 0) {
+#pragma unroll
+            for (int q = 0; q < NT; ++q)
+              if (q < nt) {
+                xg[q] = ga[q];
+                xg[kDecodeMaxT + q] = ua[q];
+              }
+            mbar_arrive(&sh.xfull[grp][r]);
+          }
+        } else {
+          if (!wait_bar(&sh.xfull[grp][r], kx & 1u, a, sh)) break;
+#pragma unroll
+          for (int q = 0; q < NT; ++q)
+            if (q < nt && lane == q) {
+              const float g = ga[q] + xg[q], uu = ua[q] + xg[kDecodeMaxT + q];
+              a.h[(size_t)(s0 + q) * m + j] = __float2bfloat16_rn(silu(g) * uu);
+            }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.xempty[grp][r]);
+        }
+        ++kx;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.empty_c[slot]);
     }
   }
-  __syncthreads();  // every (row, kept token) gate and up dot is in the table
-  for (int q = threadIdx.x; q < (p1 - p0) * NT; q += blockDim.x) {
-    const int r = q / NT, x = q - r * NT;
-    const int p = p0 + r;
-    const int ui = p / m, j = p - ui * m;
-    const int s0 = sh.ufirst[ui], s1 = sh.ufirst[ui + 1];
-    if (s0 + x < s1) {
-      const float gs = part[(size_t)q * 2], us = part[(size_t)q * 2 + 1];
-      a.h[(size_t)(s0 + x) * m + j] = __float2bfloat16_rn(silu(gs) * us);
-    }
-  }
+  __syncthreads();  // every kept slot's h of this CTA's stages is written
   // h is read back by bulk copies (the async proxy) after the grid barrier
   asm volatile("fence.proxy.async.global;" ::: "memory");
   stamp(a, 4);
@@ -597,13 +646,11 @@ cudaError_t launch_nt(cudaLaunchConfig_t& cfg, const DecodeArgs& a, size_t smem)
 
 }  // namespace
 
-// Dynamic shared memory: [ring of nring 32 KB stages | bf16(x) [T][d] |
-// phase-C dot table (rows of the CTA's share x T x 2 floats)].  The unrounded
-// fp32 x of phase A lives inside the ring.
+// Dynamic shared memory: [ring of nring 32 KB stages | bf16(x) [T][d]].  The
+// unrounded fp32 x and the staged inputs of phase A live inside the ring.
 static size_t region_bytes(int T, int d, int m, int k, int E, int num_sms) {
-  const int umax = E < T * k ? E : T * k;
-  const size_t rows = ((size_t)umax * m + num_sms - 1) / num_sms + 1;
-  return (size_t)T * d * 2 + rows * T * 2 * 4;
+  (void)m, (void)k, (void)E, (void)num_sms;
+  return (size_t)T * d * 2;  // bf16(x)
 }
 
 static int ring_stages(int T, int d, int m, int k, int E, int num_sms) {
