@@ -37,7 +37,8 @@ namespace {
 
 constexpr int kCompWarps = 16;                      // compute warps
 constexpr int kDecThreads = (kCompWarps + 1) * 32;  // + one producer warp
-constexpr int kRing = 6;                            // most stages of the copy ring
+constexpr int kRing = 6;                            // most stages of the phase-C ring
+constexpr int kRingD = 8;                           // most stages of the phase-D ring
 constexpr int kStageBytes = 32 * 1024;              // bytes per stage
 constexpr int kSmemBudget = 226 * 1024;             // dynamic + static shared memory
 constexpr int kMaxStageRows = 4;                    // (gate, up) row pairs per phase-C stage
@@ -78,7 +79,7 @@ struct DecodeArgs {
 };
 
 struct DecShared {
-  uint64_t full_c[kRing], empty_c[kRing], full_d[kRing], empty_d[kRing];
+  uint64_t full_c[kRing], empty_c[kRing], full_d[kRingD], empty_d[kRingD];
   int n_slots;                 // kept slots
   int n_uexp;                  // distinct experts among them
   int slot_e[kMaxSlots];
@@ -94,7 +95,7 @@ struct DecShared {
   int t_pos[kMaxSlots];
   uint32_t tok_mask[kMaxE];    // per expert: bit t set when token t kept a slot of it
   int e_base[kMaxE];           // per expert: its first slot
-  float acc_d[kCompWarps][kDecodeMaxT];  // phase-D per-warp token sums
+  float acc_d[2][kCompWarps][kDecodeMaxT];  // phase D: per group, row and token
   uint64_t in_bar;             // phase A: u, gamma and the router rows have landed
   uint64_t h_bar;              // phase D: h of the kept slots has landed
   int slot_stage[kRing];       // phase C: the stage a ring slot holds (-1: no more)
@@ -202,8 +203,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sh.full_c[i], 1);
       mbar_init(&sh.empty_c[i], kCompWarps / 2);
+    }
+    for (int i = 0; i < kRingD; ++i) {
       mbar_init(&sh.full_d[i], 1);
-      mbar_init(&sh.empty_d[i], kCompWarps);
+      mbar_init(&sh.empty_d[i], kCompWarps / 2);
     }
     mbar_init(&sh.in_bar, 1);
     mbar_init(&sh.h_bar, 1);
@@ -399,8 +402,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const uint32_t dstage = (dbytes + 1023u) & ~1023u;
   __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(dsm);
   uint8_t* ring_d = dsm + hbytes;
+  // even, like phase C's ring: the two consumer groups take alternate stages
   const int nring_d =
-      dstage ? (int)min((size_t)kRing, (a.dyn_bytes - 1024 - hbytes) / dstage) : 1;
+      dstage ? (int)min((size_t)kRingD, (a.dyn_bytes - 1024 - hbytes) / dstage) & ~1 : 2;
   // stages that lie inside phase C's ring (free once its last stage is
   // consumed), clear of bf16(x) that phase C still reads
   const int n_pre = (nrows > 0 && hbytes + dstage <= (size_t)a.region)
@@ -567,16 +571,26 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         }
       }
     } else {
-      if (lane < NT) sh.acc_d[warp][lane] = 0.f;
+      // two groups of 8 warps take alternate experts (the phase-D ring is
+      // even, so a slot always belongs to one group); warp wl of a group owns
+      // the CTA's output rows wl and wl + 8 and sums, per token, g * (h W^down)
+      // over its group's experts in ascending order
+      const int grp = warp >> 3, wl = warp & 7;
+      if (lane < NT) {
+        sh.acc_d[grp][wl][lane] = 0.f;
+        sh.acc_d[grp][wl + 8][lane] = 0.f;
+      }
       __syncwarp();
-      if (!wait_bar(&sh.h_bar, 0, a, sh)) return;
-      for (int ui = 0; ui < U; ++ui) {
+      bool ok = wait_bar(&sh.h_bar, 0, a, sh);
+      for (int ui = grp; ok && ui < U; ui += 2) {
         const int slot = ui % nring_d;
-        if (!wait_bar(&sh.full_d[slot], (ui / nring_d) & 1, a, sh)) break;
-        if (warp < nrows) {
-          const int s0 = sh.ufirst[ui], s1 = sh.ufirst[ui + 1];
+        if (!(ok = wait_bar(&sh.full_d[slot], (ui / nring_d) & 1, a, sh))) break;
+        const int s0 = sh.ufirst[ui], s1 = sh.ufirst[ui + 1];
+        for (int rr = 0; rr < 2; ++rr) {
+          const int row = wl + 8 * rr;
+          if (row >= nrows) continue;
           const uint4* wrow =
-              reinterpret_cast<const uint4*>(ring_d + (size_t)slot * dstage + (size_t)warp * m * 2);
+              reinterpret_cast<const uint4*>(ring_d + (size_t)slot * dstage + (size_t)row * m * 2);
           for (int sg = s0; sg < s1; sg += 4) {  // the expert's kept tokens, 4 at a time
             const int nt = min(4, s1 - sg);
             float dot[4] = {0.f, 0.f, 0.f, 0.f};
@@ -598,7 +612,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
               const float r = warp_sum(dot[q]);
               if (lane == 0) {
                 const int t = sh.slot_t[sg + q];
-                sh.acc_d[warp][t] = fmaf(sh.slot_g[sg + q], r, sh.acc_d[warp][t]);
+                sh.acc_d[grp][row][t] = fmaf(sh.slot_g[sg + q], r, sh.acc_d[grp][row][t]);
               }
             }
           }
@@ -606,11 +620,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.empty_d[slot]);
       }
-      __syncwarp();
-      if (warp < nrows && lane < NT)
-        a.y[(size_t)lane * d + i0 + warp] = __float2bfloat16_rn(sh.acc_d[warp][lane]);
     }
   }
+  __syncthreads();  // both groups' sums are in
+  if (warp < nrows && lane < NT)
+    a.y[(size_t)lane * d + i0 + warp] =
+        __float2bfloat16_rn(sh.acc_d[0][warp][lane] + sh.acc_d[1][warp][lane]);
   stamp(a, 6);
 
   // debug / compaction outputs (CTA 0, off the critical path)
@@ -666,9 +681,11 @@ static int ring_stages(int T, int d, int m, int k, int E, int num_sms) {
   return n & ~1;
 }
 
+// All the shared memory a CTA can have: phase C uses its ring and bf16(x),
+// phase D the whole of it (h, then as many W^down stages as fit).
 size_t decode_smem_bytes(int T, int d, int m, int k, int E, int num_sms) {
-  return 1024 + (size_t)ring_stages(T, d, m, k, E, num_sms) * kStageBytes +
-         region_bytes(T, d, m, k, E, num_sms);
+  (void)T, (void)d, (void)m, (void)k, (void)E, (void)num_sms;
+  return (size_t)kSmemBudget - sizeof(DecShared);
 }
 
 bool decode_fits(int T, int d, int m, int k, int E, int num_sms) {
