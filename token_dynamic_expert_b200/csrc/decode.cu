@@ -586,33 +586,45 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         const int slot = ui % nring_d;
         if (!(ok = wait_bar(&sh.full_d[slot], (ui / nring_d) & 1, a, sh))) break;
         const int s0 = sh.ufirst[ui], s1 = sh.ufirst[ui + 1];
-        for (int rr = 0; rr < 2; ++rr) {
-          const int row = wl + 8 * rr;
-          if (row >= nrows) continue;
-          const uint4* wrow =
-              reinterpret_cast<const uint4*>(ring_d + (size_t)slot * dstage + (size_t)row * m * 2);
+        // both rows of the warp in one pass: the h chunks are loaded once
+        // and the two rows' loads and reductions overlap
+        if (wl < nrows) {
+          const bool two = wl + 8 < nrows;
+          const uint4* w0 =
+              reinterpret_cast<const uint4*>(ring_d + (size_t)slot * dstage + (size_t)wl * m * 2);
+          const uint4* w1 = w0 + (two ? 8 * m / 8 : 0);
           for (int sg = s0; sg < s1; sg += 4) {  // the expert's kept tokens, 4 at a time
             const int nt = min(4, s1 - sg);
-            float dot[4] = {0.f, 0.f, 0.f, 0.f};
+            float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
             for (int c = lane; c < m / 8; c += 32) {
-              float w8[8];
-              bf16x8_to_f32(wrow[c], w8);
+              float a8[8], b8[8];
+              bf16x8_to_f32(w0[c], a8);
+              bf16x8_to_f32(w1[c], b8);
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 if (q >= nt) break;
                 float hv[8];
                 bf16x8_to_f32(reinterpret_cast<const uint4*>(hs + (size_t)(sg + q) * m)[c], hv);
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) dot[q] = fmaf(w8[cc], hv[cc], dot[q]);
+                for (int cc = 0; cc < 8; ++cc) {
+                  d0[q] = fmaf(a8[cc], hv[cc], d0[q]);
+                  d1[q] = fmaf(b8[cc], hv[cc], d1[q]);
+                }
               }
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               if (q >= nt) break;
-              const float r = warp_sum(dot[q]);
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) {
+                d0[q] += __shfl_xor_sync(0xffffffffu, d0[q], o);
+                d1[q] += __shfl_xor_sync(0xffffffffu, d1[q], o);
+              }
               if (lane == 0) {
                 const int t = sh.slot_t[sg + q];
-                sh.acc_d[grp][row][t] = fmaf(sh.slot_g[sg + q], r, sh.acc_d[grp][row][t]);
+                const float gq = sh.slot_g[sg + q];
+                sh.acc_d[grp][wl][t] = fmaf(gq, d0[q], sh.acc_d[grp][wl][t]);
+                if (two) sh.acc_d[grp][wl + 8][t] = fmaf(gq, d1[q], sh.acc_d[grp][wl + 8][t]);
               }
             }
           }
