@@ -43,6 +43,7 @@ constexpr int kStageBytes = 32 * 1024;              // bytes per stage
 constexpr int kSmemBudget = 226 * 1024;             // dynamic + static shared memory
 constexpr int kMaxStageRows = 4;                    // (gate, up) row pairs per phase-C stage
 constexpr int kMaxSlots = kDecodeMaxT * kMaxK;
+constexpr int kEndStages = 4;  // >= kCompWarps / (row pairs per stage) (4 pairs at d = 2048)
 // phase-C dot table: [row of the CTA's share][kept token of the row's
 // expert][gate, up], in dynamic shared memory after bf16(x)
 
@@ -99,8 +100,8 @@ struct DecShared {
   uint64_t in_bar;             // phase A: u, gamma and the router rows have landed
   uint64_t h_bar;              // phase D: h of the kept slots has landed
   int slot_stage[kRing];       // phase C: the stage a ring slot holds (-1: no more)
-  float xchg[2][kMaxStageRows][2 * kDecodeMaxT];  // phase C: second half-row dots
-  uint64_t xfull[2][kMaxStageRows], xempty[2][kMaxStageRows];  // ... and their handover
+  int slot_gen[kRing];         // phase C: the CTA's stage number a slot was last claimed for
+  int item_ctr;                // phase C: next (stage, row pair) item of this CTA
   int abort;
 };
 
@@ -200,9 +201,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const int n_mine = (int)blockIdx.x < E ? min(n_router_warps, (E - 1 - (int)blockIdx.x) / G + 1) : 0;
   if (threadIdx.x == 0) {
     sh.abort = 0;
+    const int sr = max(1, min(kMaxStageRows, kStageBytes / (4 * d)));  // items per stage
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sh.full_c[i], 1);
-      mbar_init(&sh.empty_c[i], kCompWarps / 2);
+      mbar_init(&sh.empty_c[i], sr);
     }
     for (int i = 0; i < kRingD; ++i) {
       mbar_init(&sh.full_d[i], 1);
@@ -210,11 +212,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     }
     mbar_init(&sh.in_bar, 1);
     mbar_init(&sh.h_bar, 1);
-    for (int g = 0; g < 2; ++g)
-      for (int r = 0; r < kMaxStageRows; ++r) {
-        mbar_init(&sh.xfull[g][r], 1);
-        mbar_init(&sh.xempty[g][r], 1);
-      }
+    sh.item_ctr = 0;
+    for (int i = 0; i < kRing; ++i) sh.slot_gen[i] = -1;
     fence_barrier_init();
     // one round trip for every input of phase A
     mbar_expect_tx(&sh.in_bar, (uint32_t)(NT * d * 2 + d * 4 + n_mine * d * 2));
@@ -423,6 +422,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         const int gst = (int)atomicAdd(stage_ctr, 1u);
         if (gst >= n_stages) break;
         sh.slot_stage[slot] = gst;
+        *(volatile int*)&sh.slot_gen[slot] = ls;
         const int pa = gst * SR, pb = min(P, pa + SR);
         mbar_expect_tx(&sh.full_c[slot], (uint32_t)((pb - pa) * d * 4));
         uint8_t* sg = ring + slot * kStageBytes;
@@ -438,12 +438,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
           p += run;
         }
       }
-      // end marks for both consumer groups: this CTA's stages ls and ls + 1
-      for (int e = 0; e < 2 && ok; ++e) {
-        const int slot = (ls + e) % nring;
-        if (e == 1) ok = wait_bar(&sh.empty_c[slot], (((ls + 1) / nring) & 1) ^ 1u, a, sh);
+      // end marks: every compute warp draws at most one item past the last
+      // stage, so the next kCompWarps / SR stages (at most the ring) carry none
+      for (int e = 0; e < kEndStages && ok; ++e) {
+        const int st = ls + e, slot = st % nring;
+        if (e > 0) ok = wait_bar(&sh.empty_c[slot], ((st / nring) & 1) ^ 1u, a, sh);
         if (ok) {
           sh.slot_stage[slot] = -1;
+          *(volatile int*)&sh.slot_gen[slot] = st;
           mbar_arrive(&sh.full_c[slot]);
         }
       }
@@ -459,18 +461,33 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       }
     }
   } else {
-    // two groups of 8 warps take alternate stages (the ring is even, so a
-    // slot always belongs to the same group).  In a group, warps 2r and
-    // 2r + 1 take row pair r of the stage, each over half of the hidden
-    // size, for every kept token of the pair's expert: the gate and up dots.
-    // The second warp hands its halves over through shared memory; the
-    // first forms h = SiLU(gate) * up and writes it.
-    const int grp = warp >> 3, wi = warp & 7;
-    const int r = wi >> 1, half = wi & 1;
-    const int hv = d / 16;  // 16-byte chunks per half row
-    uint32_t kx = 0;        // handovers of this warp pair so far
-    for (int ls = grp;; ls += 2) {
+    // Items are (stage, row pair), drawn in order from a CTA counter by
+    // whichever warp is free: the warp forms the pair's gate and up dots
+    // over the whole hidden size for every kept token of its expert and
+    // writes h = SiLU(gate) * up.  A warp may draw an item of a stage one
+    // lap ahead of the ring, so it first waits for the producer to have
+    // claimed the slot for that stage (slot_gen), then for the data.
+    const int nvc = d / 8;  // 16-byte chunks per row
+    const uint4* xq = reinterpret_cast<const uint4*>(xb);
+    for (;;) {
+      int it = 0;
+      if (lane == 0) it = atomicAdd(&sh.item_ctr, 1);
+      it = __shfl_sync(0xffffffffu, it, 0);
+      const int ls = it / SR, r = it - ls * SR;
       const int slot = ls % nring;
+      {
+        bool claimed = true;
+        const uint64_t t0 = global_ns();
+        while (*(volatile int*)&sh.slot_gen[slot] != ls) {
+          if (sh.abort || global_ns() - t0 > kWaitLimitNs) {
+            if (!sh.abort) raise_flag(a.status, ACE_FLAG_TIMEOUT);
+            sh.abort = 1;
+            claimed = false;
+            break;
+          }
+        }
+        if (!claimed) break;
+      }
       if (!wait_bar(&sh.full_c[slot], (ls / nring) & 1, a, sh)) break;
       const int gst = sh.slot_stage[slot];
       if (gst < 0) break;
@@ -480,19 +497,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         const int ui = p / m, j = p - ui * m;
         const int s0 = sh.ufirst[ui], nt = sh.ufirst[ui + 1] - s0;  // <= NT
         const uint4* wg =
-            reinterpret_cast<const uint4*>(ring + slot * kStageBytes + (size_t)r * d * 2) +
-            half * hv;
+            reinterpret_cast<const uint4*>(ring + slot * kStageBytes + (size_t)r * d * 2);
         const uint4* wu = reinterpret_cast<const uint4*>(ring + slot * kStageBytes +
-                                                         kStageBytes / 2 + (size_t)r * d * 2) +
-                          half * hv;
+                                                         kStageBytes / 2 + (size_t)r * d * 2);
         int xo[NT];  // each kept token's row of bf16(x), in 16-byte chunks
 #pragma unroll
-        for (int q = 0; q < NT; ++q) xo[q] = (q < nt ? sh.slot_t[s0 + q] : 0) * (d / 8) + half * hv;
+        for (int q = 0; q < NT; ++q) xo[q] = (q < nt ? sh.slot_t[s0 + q] : 0) * nvc;
         float ga[NT], ua[NT];
 #pragma unroll
         for (int q = 0; q < NT; ++q) ga[q] = ua[q] = 0.f;
-        const uint4* xq = reinterpret_cast<const uint4*>(xb);
-        for (int c = lane; c < hv; c += 32) {
+        for (int c = lane; c < nvc; c += 32) {
           float w1[8], w2[8];
           bf16x8_to_f32(wg[c], w1);
           bf16x8_to_f32(wu[c], w2);
@@ -512,34 +526,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
 #pragma unroll
         for (int q = 0; q < NT; ++q) {
           if (q < nt) {
-            ga[q] = warp_sum(ga[q]);
-            ua[q] = warp_sum(ua[q]);
-          }
-        }
-        float* xg = &sh.xchg[grp][r][0];
-        if (half == 1) {  // hand the second half over (one buffer per pair)
-          if (!wait_bar(&sh.xempty[grp][r], (kx & 1u) ^ 1u, a, sh)) break;
-          if (lane == 0) {
 #pragma unroll
-            for (int q = 0; q < NT; ++q)
-              if (q < nt) {
-                xg[q] = ga[q];
-                xg[kDecodeMaxT + q] = ua[q];
-              }
-            mbar_arrive(&sh.xfull[grp][r]);
-          }
-        } else {
-          if (!wait_bar(&sh.xfull[grp][r], kx & 1u, a, sh)) break;
-#pragma unroll
-          for (int q = 0; q < NT; ++q)
-            if (q < nt && lane == q) {
-              const float g = ga[q] + xg[q], uu = ua[q] + xg[kDecodeMaxT + q];
-              a.h[(size_t)(s0 + q) * m + j] = __float2bfloat16_rn(silu(g) * uu);
+            for (int o = 16; o > 0; o >>= 1) {
+              ga[q] += __shfl_xor_sync(0xffffffffu, ga[q], o);
+              ua[q] += __shfl_xor_sync(0xffffffffu, ua[q], o);
             }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.xempty[grp][r]);
+            if (lane == q) a.h[(size_t)(s0 + q) * m + j] = __float2bfloat16_rn(silu(ga[q]) * ua[q]);
+          }
         }
-        ++kx;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.empty_c[slot]);
@@ -703,7 +697,7 @@ size_t decode_smem_bytes(int T, int d, int m, int k, int E, int num_sms) {
 bool decode_fits(int T, int d, int m, int k, int E, int num_sms) {
   if (T < 1 || T > kDecodeMaxT || d > 2048 || d % 32 != 0 || m % 8 != 0) return false;
   const int n = ring_stages(T, d, m, k, E, num_sms);
-  if (n < 2) return false;
+  if (n < kEndStages) return false;  // the end marks take kEndStages distinct slots
   // phase A inside the ring: x (fp32), u (bf16), gamma, the router rows
   const size_t staged = (size_t)T * d * 6 + (size_t)d * 4 +
                         (size_t)((E + num_sms - 1) / num_sms) * d * 2;
