@@ -51,8 +51,11 @@ def profiled_traffic(workload):
     with open(os.path.join(ROOT, path), "rb") as f:
         cur = hashlib.sha1(f.read()).hexdigest()[:12]
     return nbytes if cur == sha else None
-# rmsnorm, router GEMM, top-k/mask (+ offset scan), scatter+gather, gate/up, down, combine
-KERNELS_PER_FORWARD = 7
+# status clear, rmsnorm, router GEMM, top-k/mask (+ offset scan), scatter+gather, gate/up,
+# down, combine
+KERNELS_PER_FORWARD = 8
+# per decode layer: status clear, the decode kernel
+KERNELS_PER_DECODE_LAYER = 2
 
 
 # ----------------------------------------------------------------- helpers
@@ -567,7 +570,7 @@ def run_decode(args, w, ws_n, rank, local):
         "e2e": {"value": ws_n * args.steps * nl * w.T / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
                 "launch": "plain API calls, no graph"},
-        "gpu_launches": nl * args.steps,
+        "gpu_launches": KERNELS_PER_DECODE_LAYER * nl * args.steps,
     }
 
 
@@ -666,7 +669,7 @@ def run_stack(args, w, ws_n, rank, local):
         "e2e": {"value": ws_n * args.steps * w.T / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
                 "launch": "plain API call per step"},
-        "gpu_launches": nl * args.steps,
+        "gpu_launches": (KERNELS_PER_DECODE_LAYER * nl + 1) * args.steps,
     }
 
 

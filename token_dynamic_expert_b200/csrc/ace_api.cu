@@ -8,6 +8,18 @@
 
 namespace ace {
 
+// Zeroes n 32-bit words.  A kernel rather than cudaMemsetAsync: inside a CUDA
+// graph a memset node before a kernel node costs ~3 us of dependency
+// latency on B200, a kernel node ~1 us.
+__global__ void k_clear_words(uint32_t* p, int n) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) p[i] = 0u;
+}
+
+cudaError_t launch_clear_words(void* p, int n_words, cudaStream_t s) {
+  k_clear_words<<<1, 64, 0, s>>>(static_cast<uint32_t*>(p), n_words);
+  return cudaGetLastError();
+}
+
 int device_sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -260,9 +272,9 @@ ace_status forward_impl(const ace_layer* layer, const void* u, int T, const ace_
   // status word (offset 0), the decode kernel's grid-barrier words (byte 64)
   // and the routing CTAs' completion count (byte 128)
   if (keep_status)
-    ACE_CK(cudaMemsetAsync(at<uint8_t>(ws, ly.status) + 64, 0, 192, s));
+    ACE_CK(launch_clear_words(at<uint8_t>(ws, ly.status) + 64, 48, s));
   else
-    ACE_CK(cudaMemsetAsync(at<void>(ws, ly.status), 0, 256, s));
+    ACE_CK(launch_clear_words(at<void>(ws, ly.status), 64, s));
   if (T == 0) return ACE_OK;
   cudaEvent_t ev_b = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_begin) : nullptr;
   cudaEvent_t ev_m = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_mid) : nullptr;
@@ -367,7 +379,7 @@ ace_status ace_moe_stack_forward(const ace_layer* layers, int n_layers, const vo
   if (!stack_layout(layers, n_layers, T, device_sm_count(), &ly)) return ACE_ERR_INVALID_ARG;
   if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ACE_CK(cudaMemsetAsync(ws, 0, 4, s));  // the status word, once for the stack
+  ACE_CK(launch_clear_words(ws, 1, s));  // the status word, once for the stack
   if (T == 0) return ACE_OK;
   uint8_t* base = static_cast<uint8_t*>(ws);
   const void* in = u;
@@ -392,7 +404,7 @@ ace_status ace_moe_scores(const ace_layer* layer, const void* u, int T, const ac
   const FwdLayout ly = fwd_layout(L, T, num_sms);
   if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ACE_CK(cudaMemsetAsync(at<void>(ws, ly.status), 0, 256, s));
+  ACE_CK(launch_clear_words(at<void>(ws, ly.status), 64, s));
   if (T == 0) return ACE_OK;
   st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, false, s);
   if (st != ACE_OK) return st;

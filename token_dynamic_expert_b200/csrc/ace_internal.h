@@ -41,6 +41,8 @@ struct FwdLayout {
 FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms);
 
 int device_sm_count();
+// Zeroes n_words 32-bit words on the stream (the status block of a call).
+cudaError_t launch_clear_words(void* p, int n_words, cudaStream_t s);
 ace_status check_fusion(const ace_layer& L, int fusion);
 
 // ---------------------------------------------------------------- launchers

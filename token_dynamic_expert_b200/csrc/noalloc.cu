@@ -115,7 +115,7 @@ extern "C" ace_status ace_moe_decode_noalloc(const ace_layer* layer, const void*
   uint8_t* w = static_cast<uint8_t*>(base);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the status word and the grid-barrier counter must start at zero
-  if (cudaMemsetAsync(w, 0, 256, s) != cudaSuccess) return ACE_ERR_CUDA;
+  if (launch_clear_words(w, 64, s) != cudaSuccess) return ACE_ERR_CUDA;
   auto at = [&](size_t off) { return w + off; };
   if (launch_decode(L, (int)opts->fusion, u, T, opts->tau, opts->renorm_topk, opts->eps_rms, y,
                     reinterpret_cast<float*>(at(ly.logits)), at(ly.h),
