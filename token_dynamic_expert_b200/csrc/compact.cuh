@@ -1,7 +1,7 @@
 // compact.cuh -- the expert-offset scan of the compaction, as a block-level
 // device routine run by the last routing CTA to finish.
 //
-// From the per-(32-token chunk, expert) kept-slot histogram it forms the
+// From the per-(expert, 32-token chunk) kept-slot histogram it forms the
 // per-expert counts, the exclusive offsets over experts (kept slots ordered
 // by expert, then token), the per-(chunk, expert) base positions and the list
 // of expert GEMM tiles (expert, first slot, rows <= tile_n) in expert order.
@@ -49,53 +49,83 @@ struct ScanOut {
   int max_tiles, tile_n;
 };
 
-// Whole-CTA routine (every thread calls it; blockDim.x a multiple of 32 and
-// at least E).  hist is read with L2-coherent loads: other CTAs wrote it.
+// Whole-CTA routine (every thread calls it; blockDim.x a multiple of 32, at
+// least E, at most 1024).  hist is expert-major, [E][nchunk], and read with
+// L2-coherent loads (other CTAs wrote it); base is chunk-major, [nchunk][E].
+// A warp takes four experts at a time: their chunk counts are summed (pass 1)
+// and, once the offsets over experts are known, scanned over the chunks in
+// segments of 32 (pass 2).
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
 __device__ __forceinline__ void scan_experts(const int32_t* hist, int nchunk, int E,
                                              const ScanOut& o) {
   __shared__ int s_warp[32];
-  int tpe = 1;  // threads per expert (a power of two that divides 32)
-  while (tpe < 32 && tpe * 2 * E <= (int)blockDim.x) tpe *= 2;
-  const int e = threadIdx.x / tpe, g = threadIdx.x % tpe;
-  const bool active = e < E;
-  const int per = (nchunk + tpe - 1) / tpe;
-  const int cb = min(nchunk, g * per), ce = min(nchunk, cb + per);
-  int local = 0;
-  if (active)
-    for (int c = cb; c < ce; ++c) local += __ldcg(hist + (size_t)c * E + e);
-  // prefix inside the expert's group of tpe consecutive lanes
-  int incl = local;
-  for (int sh = 1; sh < tpe; sh <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, incl, sh, tpe);
-    if (g >= sh) incl += n;
-  }
-  const int excl_in_group = incl - local;
-  const int cnt = __shfl_sync(0xffffffffu, incl, tpe - 1, tpe);
-  int total, total_tiles;
-  const int off = block_excl_scan((active && g == 0) ? cnt : 0, s_warp, &total);
-  const int ntile = (active && g == 0) ? (cnt + o.tile_n - 1) / o.tile_n : 0;
-  const int toff = block_excl_scan(ntile, s_warp, &total_tiles);
-  const int off_e = __shfl_sync(0xffffffffu, off, 0, tpe);
-  if (active) {
-    int run = off_e + excl_in_group;
-    for (int c = cb; c < ce; ++c) {
-      o.base[(size_t)c * E + e] = run;
-      run += __ldcg(hist + (size_t)c * E + e);
-    }
-    if (g == 0) {
-      o.counts[e] = cnt;
-      o.offsets[e] = off;
-      for (int q = 0; q < ntile; ++q) {
-        if (toff + q < o.max_tiles)
-          o.tiles[toff + q] =
-              make_int4(e, off + q * o.tile_n, min(o.tile_n, cnt - q * o.tile_n), 0);
+  __shared__ int s_cnt[1024], s_off[1024];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  constexpr int kEpw = 4;  // experts a warp handles at once
+  // pass 1: per-expert counts
+  for (int eb = warp; eb < E; eb += kEpw * nw) {
+    int acc[kEpw] = {0, 0, 0, 0};
+#pragma unroll 2
+    for (int c = lane; c < nchunk; c += 32)
+#pragma unroll
+      for (int j = 0; j < kEpw; ++j) {
+        const int e = eb + j * nw;
+        if (e < E) acc[j] += __ldcg(hist + (size_t)e * nchunk + c);
       }
+#pragma unroll
+    for (int j = 0; j < kEpw; ++j) {
+#pragma unroll
+      for (int sh = 16; sh > 0; sh >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], sh);
+      const int e = eb + j * nw;
+      if (lane == 0 && e < E) s_cnt[e] = acc[j];
     }
   }
-  if (threadIdx.x == 0) {
+  __syncthreads();
+  // offsets over experts and the tile list
+  const int t = threadIdx.x;
+  const int cnt = t < E ? s_cnt[t] : 0;
+  int total, total_tiles;
+  const int off = block_excl_scan(cnt, s_warp, &total);
+  const int ntile = t < E ? (cnt + o.tile_n - 1) / o.tile_n : 0;
+  const int toff = block_excl_scan(ntile, s_warp, &total_tiles);
+  if (t < E) {
+    s_off[t] = off;
+    o.counts[t] = cnt;
+    o.offsets[t] = off;
+    for (int q = 0; q < ntile; ++q)
+      if (toff + q < o.max_tiles)
+        o.tiles[toff + q] = make_int4(t, off + q * o.tile_n, min(o.tile_n, cnt - q * o.tile_n), 0);
+  }
+  if (t == 0) {
     o.offsets[E] = total;
     *o.n_kept = total;
     *o.n_tiles = min(total_tiles, o.max_tiles);
+  }
+  __syncthreads();
+  // pass 2: base[c][e] = offset of e + kept slots of e in chunks before c
+  for (int eb = warp; eb < E; eb += kEpw * nw) {
+    int carry[kEpw];
+#pragma unroll
+    for (int j = 0; j < kEpw; ++j) carry[j] = eb + j * nw < E ? s_off[eb + j * nw] : 0;
+    for (int c0 = 0; c0 < nchunk; c0 += 32) {
+      const int c = c0 + lane;
+#pragma unroll
+      for (int j = 0; j < kEpw; ++j) {
+        const int e = eb + j * nw;
+        const int v = (e < E && c < nchunk) ? __ldcg(hist + (size_t)e * nchunk + c) : 0;
+        const int incl = warp_incl_scan(v, lane);
+        if (e < E && c < nchunk) o.base[(size_t)c * E + e] = carry[j] + incl - v;
+        carry[j] += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
   }
 }
 

@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     bitmap[(size_t)c * E + e] = bm[e];
-    hist[(size_t)c * E + e] = __popc(bm[e]);
+    hist[(size_t)e * gridDim.x + c] = __popc(bm[e]);  // expert-major
   }
   if (done_ctr == nullptr) return;
   // the last CTA to finish runs the expert-offset scan over every chunk's
