@@ -68,13 +68,15 @@ def test_noalloc_rejects_what_it_cannot_serve():
              ctypes.c_void_p(y.data_ptr()), s) == ace.ACE_ERR_INVALID_ARG
     assert f(ctypes.byref(L), ctypes.c_void_p(u.data_ptr()), 4, ctypes.byref(opts),
              ctypes.c_void_p(u.data_ptr()), s) == ace.ACE_ERR_INVALID_ARG  # u, y overlap
-    big = workloads.Workload("big", T=8, d=2048, E=512, m=1024, k=16, dtype="bf16", bias=False,
+    # A layer whose scratch exceeds the fixed array: 8 tokens x top-16 x FFN 4096 bf16
+    # intermediates are 1 MiB.  Its buffers are real and of its own shape, so nothing
+    # would be read out of bounds even if the call were (wrongly) accepted.
+    big = workloads.Workload("big", T=8, d=256, E=32, m=4096, k=16, dtype="bf16", bias=False,
                              skip=0.5, skip_of="slots")
-    # 8 x 16 x 1024 bf16 intermediates alone exceed the fixed scratch
-    Lb = ace.ace_layer(d=big.d, E=big.E, m=big.m, k=big.k, dtype=ace.ACE_BF16,
-                       gamma=layer["gamma"].data_ptr(), w_router=layer["wr"].data_ptr(),
-                       router_bias=None, w_gate=layer["wg"].data_ptr(),
-                       w_up=layer["wu"].data_ptr(), w_down=layer["wd"].data_ptr(), amax=None)
-    assert f(ctypes.byref(Lb), ctypes.c_void_p(u.data_ptr()), 8, ctypes.byref(opts),
-             ctypes.c_void_p(y.data_ptr()), s) == ace.ACE_ERR_UNSUPPORTED
+    lb = workloads.make_layer(big, seed=3, device="cuda")
+    Lb = ace.make_layer(lb["gamma"], lb["wr"], lb["wg"], lb["wu"], lb["wd"], big.k)
+    ub = torch.zeros(8, big.d, dtype=torch.bfloat16, device="cuda")
+    yb = torch.zeros_like(ub)
+    assert f(ctypes.byref(Lb), ctypes.c_void_p(ub.data_ptr()), 8, ctypes.byref(opts),
+             ctypes.c_void_p(yb.data_ptr()), s) == ace.ACE_ERR_UNSUPPORTED
     torch.cuda.synchronize()
