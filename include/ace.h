@@ -146,7 +146,9 @@ typedef struct {
   /* Optional cudaEvent_t handles (passed as void*) recorded on the call's
    * stream right before the gate/up expert GEMM, between it and the down
    * GEMM, and right after the down GEMM: live kernel timing for profilers
-   * and benchmarks.  NULL = not recorded. */
+   * and benchmarks.  When both GEMMs run as one kernel (small slot tiles:
+   * T k < 128 E), "mid" is recorded after that kernel, like "end".  NULL =
+   * not recorded. */
   void* ev_experts_begin;
   void* ev_experts_mid;
   void* ev_experts_end;

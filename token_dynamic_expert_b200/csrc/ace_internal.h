@@ -33,7 +33,7 @@ int router_splits_for(const ace_layer& L, int T, int num_sms);
 // Byte offsets of the forward's scratch arrays inside the caller's
 // workspace.  Everything is sized for max_tokens and no skipping.
 struct FwdLayout {
-  size_t status, part, inv_rms, x, xs3, idx, gate, score, keep, bitmap, hist, base, counts,
+  size_t status, part, inv_rms, x, xs3, tile_done, idx, gate, score, keep, bitmap, hist, base, counts,
       offsets, n_kept, tiles, n_tiles, slot_token, slot_rank, slot_gate, slot_of, xp, h,
       yslot, total;
   int max_tokens, part_floats, max_tiles;
@@ -75,6 +75,12 @@ cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* 
                                  float* yslot, const int4* tiles, const int32_t* n_tiles,
                                  int max_tiles, const float* slot_gate, uint32_t* status,
                                  int num_sms, cudaStream_t s, cudaEvent_t ev_mid);
+// Both expert GEMMs in one persistent kernel (bf16 layers): gate/up items
+// first, then down items, each down item waiting for its tile's h rows.
+cudaError_t launch_experts_fused(const ace_layer& L, int cap_slots, const void* xp, void* h,
+                                 float* yslot, const int4* tiles, const int32_t* n_tiles,
+                                 int max_tiles, const float* slot_gate, uint32_t* tile_done,
+                                 uint32_t* status, int num_sms, cudaStream_t s);
 cudaError_t launch_experts_simt(const ace_layer& L, const void* xp, void* h, float* yslot,
                                 const int4* tiles, const int32_t* n_tiles, int max_tiles,
                                 const float* slot_gate, cudaStream_t s);

@@ -46,6 +46,7 @@ struct ScanOut {
   int32_t* n_kept;   // [1]
   int4* tiles;       // [max_tiles]
   int32_t* n_tiles;  // [1]
+  uint32_t* tile_done;  // [max_tiles] or NULL: per-tile counters, zeroed here
   int max_tiles, tile_n;
 };
 
@@ -109,6 +110,8 @@ __device__ __forceinline__ void scan_experts(const int32_t* hist, int nchunk, in
     *o.n_kept = total;
     *o.n_tiles = min(total_tiles, o.max_tiles);
   }
+  if (o.tile_done)
+    for (int i = t; i < o.max_tiles; i += blockDim.x) o.tile_done[i] = 0u;
   __syncthreads();
   // pass 2: base[c][e] = offset of e + kept slots of e in chunks before c
   for (int eb = warp; eb < E; eb += kEpw * nw) {
