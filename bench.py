@@ -41,6 +41,8 @@ METRIC = "MoE-layer tokens/s (prefill, decode) at skip rate; % of tensor/HBM roo
 PROFILED_TRAFFIC = {
     ("prefill_1024", "gateup"): ("token_dynamic_expert_b200/csrc/experts_sm100.cu", "06d17ea9eed8",
                                  825441792),
+    ("prefill_1024", "fused"): ("token_dynamic_expert_b200/csrc/experts_fused_sm100.cu",
+                                "f2148741ed71", 1228692480),
 }
 
 
