@@ -54,9 +54,9 @@ def profiled_traffic(workload, kernel):
     with open(os.path.join(ROOT, path), "rb") as f:
         cur = hashlib.sha1(f.read()).hexdigest()[:12]
     return nbytes if cur == sha else None
-# status clear, rmsnorm, router GEMM, top-k/mask (+ offset scan), scatter+gather, gate/up,
-# down, combine
-KERNELS_PER_FORWARD = 8
+# status clear, rmsnorm, router GEMM, top-k/mask (+ offset scan), scatter+gather, the expert
+# GEMMs (one fused launch for small slot tiles, else gate/up and down), combine
+KERNELS_PER_FORWARD = {True: 7, False: 8}
 # per decode layer: status clear, the decode kernel
 KERNELS_PER_DECODE_LAYER = 2
 
@@ -378,7 +378,7 @@ def run_ours(args, w, rate, ws_n, rank, local):
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
                 "d2h_bytes_per_step": nbytes, "launch": "plain API calls, no graph"},
-        "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+        "gpu_launches": KERNELS_PER_FORWARD[fused] * args.steps,
     }
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w, st, rate)
