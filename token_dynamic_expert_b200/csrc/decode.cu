@@ -12,8 +12,9 @@
 //            mask ([ACE] "3. Conservative Fusion", top-1 always kept), the
 //            kept slots sorted by (expert, token), the distinct experts
 //   phase C  gate/up ([ACE] eq. f): the surviving (expert, row) pairs, in
-//            stages of 4 row pairs that the CTAs take from a grid-wide
-//            counter as their rings free up, stream through a shared-memory
+//            stages of 4 row pairs (a fixed first lap per CTA, then stages
+//            the CTAs take from a grid-wide counter as their rings free up),
+//            stream through a shared-memory
 //            ring by TMA bulk copies issued from a producer warp; 16 warps
 //            form h = SiLU(x W^gate) (.) x W^up for the expert's kept tokens
 //            and write it out; once the ring drains, the first W^down stages
@@ -95,6 +96,7 @@ struct DecShared {
   int t_keep[kMaxSlots];
   int t_pos[kMaxSlots];
   uint32_t tok_mask[kMaxE];    // per expert: bit t set when token t kept a slot of it
+  float fac[kMaxE];            // per expert: the fused table factor F(A^GSP, A^RCR)
   int e_base[kMaxE];           // per expert: its first slot
   float acc_d[2][kCompWarps][kDecodeMaxT];  // phase D: per group, row and token
   uint64_t in_bar;             // phase A: u, gamma and the router rows have landed
@@ -228,6 +230,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   __syncthreads();  // barrier inits are visible
 
   // ---------------------------------------------------------- phase A
+  // the fused table factors, read while the inputs are in flight (by the
+  // last warps, so the token warps start normalising as soon as u lands);
+  // phase B then looks them up in shared memory
+  for (int e = kDecThreads - 1 - (int)threadIdx.x; e < E; e += kDecThreads)
+    sh.fac[e] = fused_factor(a.ft, e);
   if (!wait_bar(&sh.in_bar, 0, a, sh)) return;
   if (warp < NT) {  // token warps: x = u / rms(u) * gamma
     const int t = warp;
@@ -319,7 +326,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     }
     if (lane < k) {
       const float g = ex / denom;
-      const float sc = g * fused_factor(a.ft, sel_e);
+      const float sc = g * sh.fac[sel_e];
       sh.t_idx[t * k + lane] = sel_e;
       sh.t_gate[t * k + lane] = g;
       sh.t_score[t * k + lane] = sc;
@@ -411,16 +418,39 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
                         : 0;
   if (producer) {
     if (lane == 0) {
-      // stages are taken from a grid-wide counter as the ring frees up, so
-      // CTAs that run ahead take more of them
+      // The ring's first lap takes the fixed stages blockIdx.x + G * ls, so
+      // it is issued at once.  Later stages come from a grid-wide counter as
+      // the ring frees up (CTAs that run ahead take more of them), numbered
+      // from G * nring on; each is claimed two stages before it is issued, so
+      // the atomic's round trip overlaps the wait for a free slot.  The two
+      // pending claims alternate (even and odd stages after the first lap)
+      // and a CTA's claims increase in the order it makes them: when the
+      // claim in use is past the last stage, so is the one still pending.
       uint32_t* stage_ctr = a.bar_count + 1;
+      const int dyn0 = G * nring;
+      int claim_even = 0, claim_odd = 0;
       int ls = 0;  // this CTA's stages so far
       bool ok = true;
       for (;; ++ls) {
         const int slot = ls % nring;
         if (!(ok = wait_bar(&sh.empty_c[slot], ((ls / nring) & 1) ^ 1u, a, sh))) break;
-        const int gst = (int)atomicAdd(stage_ctr, 1u);
-        if (gst >= n_stages) break;
+        int gst;
+        if (ls < nring) {
+          gst = (int)blockIdx.x + G * ls;
+          if (gst >= n_stages) break;
+          if (ls == nring - 1) {
+            claim_even = (int)atomicAdd(stage_ctr, 1u);
+            claim_odd = (int)atomicAdd(stage_ctr, 1u);
+          }
+        } else if (((ls - nring) & 1) == 0) {
+          gst = dyn0 + claim_even;
+          if (gst >= n_stages) break;
+          claim_even = (int)atomicAdd(stage_ctr, 1u);
+        } else {
+          gst = dyn0 + claim_odd;
+          if (gst >= n_stages) break;
+          claim_odd = (int)atomicAdd(stage_ctr, 1u);
+        }
         sh.slot_stage[slot] = gst;
         *(volatile int*)&sh.slot_gen[slot] = ls;
         const int pa = gst * SR, pb = min(P, pa + SR);
