@@ -15,10 +15,12 @@
 //            stages of 4 row pairs (a fixed first lap per CTA, then stages
 //            the CTAs take from a grid-wide counter as their rings free up),
 //            stream through a shared-memory
-//            ring by TMA bulk copies issued from a producer warp; 16 warps
-//            form h = SiLU(x W^gate) (.) x W^up for the expert's kept tokens
-//            and write it out; once the ring drains, the first W^down stages
-//            of phase D are issued
+//            ring by TMA bulk copies issued from a producer warp; free
+//            compute warps take a whole stage (3+ tokens: tensor-core dots
+//            of every token with its 8 rows) or one row pair of it (1-2
+//            tokens: CUDA-core dots) and write h = SiLU(x W^gate) (.) x W^up
+//            for the tokens that kept the expert; once the ring drains, the
+//            first W^down stages of phase D are issued
 //   -- grid barrier --
 //   phase D  down + combine: the CTA's output rows of every surviving
 //            expert's W^down stream through the ring; warp w owns output row
@@ -28,6 +30,7 @@
 // spin; the launch is cooperative so every CTA is resident.  Every mbarrier
 // wait is bounded as well.  Numerics follow the prefill path: fp32 router on
 // the unrounded x, experts on bf16(x), h rounded to bf16, fp32 sums.
+#include <limits.h>
 #include <math.h>
 
 #include "ace_common.cuh"
@@ -40,13 +43,17 @@ constexpr int kCompWarps = 16;                      // compute warps
 constexpr int kDecThreads = (kCompWarps + 1) * 32;  // + one producer warp
 constexpr int kRing = 6;                            // most stages of the phase-C ring
 constexpr int kRingD = 8;                           // most stages of the phase-D ring
-constexpr int kStageBytes = 32 * 1024;              // bytes per stage
 constexpr int kSmemBudget = 226 * 1024;             // dynamic + static shared memory
-constexpr int kMaxStageRows = 4;                    // (gate, up) row pairs per phase-C stage
+constexpr int kStagePairs = 4;                      // (gate, up) row pairs per phase-C stage
+constexpr int kStageRows = 2 * kStagePairs;         // staged rows: 4 gate, then 4 up
 constexpr int kMaxSlots = kDecodeMaxT * kMaxK;
-constexpr int kEndStages = 4;  // >= kCompWarps / (row pairs per stage) (4 pairs at d = 2048)
-// phase-C dot table: [row of the CTA's share][kept token of the row's
-// expert][gate, up], in dynamic shared memory after bf16(x)
+
+// Bytes between the rows of bf16(x) and between the staged weight rows of a
+// phase-C stage: 2d, plus 64 when 2d is a multiple of 128, so that rows n and
+// n + 1 start 64 bytes apart modulo 128 and the 16-byte loads of a quarter
+// warp (two rows, four consecutive 16-byte pieces of each) hit distinct banks.
+__host__ __device__ constexpr int row_stride(int d) { return 2 * d + ((2 * d) % 128 == 0 ? 64 : 0); }
+constexpr int kStageBytes = kStageRows * row_stride(2048);  // bytes per ring slot (d <= 2048)
 
 struct DecodeArgs {
   const float* gamma;
@@ -103,7 +110,8 @@ struct DecShared {
   uint64_t h_bar;              // phase D: h of the kept slots has landed
   int slot_stage[kRing];       // phase C: the stage a ring slot holds (-1: no more)
   int slot_gen[kRing];         // phase C: the CTA's stage number a slot was last claimed for
-  int item_ctr;                // phase C: next (stage, row pair) item of this CTA
+  int item_ctr;                // phase C: the CTA's next stage number to hand to a warp
+  int n_ls;                    // phase C: the CTA's stage count, once known (else INT_MAX)
   int abort;
 };
 
@@ -157,6 +165,23 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const D
   return mbar_wait(bar, parity, a.status, &sh.abort);
 }
 
+// Waits until the producer has claimed ring slot `slot` for the CTA's stage
+// `ls` (true), or has published a stage count at or below ls (false); false
+// as well when the bounded wait runs out (ACE_FLAG_TIMEOUT) or the CTA aborted.
+__device__ bool await_stage(const DecodeArgs& a, DecShared& sh, int slot, int ls) {
+  const uint64_t t0 = global_ns();
+  while (*(volatile int*)&sh.slot_gen[slot] != ls) {
+    if (ls >= *(volatile int*)&sh.n_ls) return false;
+    if (*(volatile int*)&sh.abort || global_ns() - t0 > kWaitLimitNs) {
+      if (!*(volatile int*)&sh.abort) raise_flag(a.status, ACE_FLAG_TIMEOUT);
+      sh.abort = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
+}
+
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& q, float (&f)[8]) {
   const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
 #pragma unroll
@@ -175,6 +200,17 @@ __device__ __forceinline__ void lds8(const float* p, float (&f)[8]) {
 }
 
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
+
+// c += A * B for one m16n8k16 tile, bf16 operands, fp32 accumulators; A's
+// rows 8 .. 15 are zero (fragments a1, a3), so c[2], c[3] stay zero
+__device__ __forceinline__ void mma_bf16_m16n8k16(float (&c)[4], uint32_t a0, uint32_t a2,
+                                                  uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
 
 
 
@@ -203,10 +239,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const int n_mine = (int)blockIdx.x < E ? min(n_router_warps, (E - 1 - (int)blockIdx.x) / G + 1) : 0;
   if (threadIdx.x == 0) {
     sh.abort = 0;
-    const int sr = max(1, min(kMaxStageRows, kStageBytes / (4 * d)));  // items per stage
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sh.full_c[i], 1);
-      mbar_init(&sh.empty_c[i], sr);
+      mbar_init(&sh.empty_c[i], NT > 2 ? 1 : kStagePairs);  // the stage's items
     }
     for (int i = 0; i < kRingD; ++i) {
       mbar_init(&sh.full_d[i], 1);
@@ -215,6 +250,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     mbar_init(&sh.in_bar, 1);
     mbar_init(&sh.h_bar, 1);
     sh.item_ctr = 0;
+    sh.n_ls = INT_MAX;
     for (int i = 0; i < kRing; ++i) sh.slot_gen[i] = -1;
     fence_barrier_init();
     // one round trip for every input of phase A
@@ -265,7 +301,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       __nv_bfloat16* bp = reinterpret_cast<__nv_bfloat16*>(&bq);
 #pragma unroll
       for (int c = 0; c < 8; ++c) bp[c] = __float2bfloat16_rn(xv[c]);
-      reinterpret_cast<uint4*>(xb + (size_t)t * d)[v] = bq;
+      reinterpret_cast<uint4*>(xb + (size_t)t * (row_stride(d) / 2))[v] = bq;
     }
   }
   __syncthreads();
@@ -399,8 +435,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const int rows_per_cta = (d + G - 1) / G;  // phase-D output rows per CTA (<= 16)
   const int i0 = min(d, (int)blockIdx.x * rows_per_cta), i1 = min(d, i0 + rows_per_cta);
   const int P = U * m;  // surviving (expert, row) pairs
-  const int SR = max(1, min(kMaxStageRows, kStageBytes / (4 * d)));  // row pairs per stage
-  const int n_stages = (P + SR - 1) / SR;
+  const int n_stages = P / kStagePairs;  // m % 8 == 0: a stage never spans two experts
+  const int rs = row_stride(d);
   // phase-D geometry (its first stages are filled while phase C ends)
   const int nrows = i1 - i0;  // <= kCompWarps: output row i0 + w belongs to warp w
   const uint32_t dbytes = (uint32_t)(nrows * m * 2);
@@ -453,32 +489,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         }
         sh.slot_stage[slot] = gst;
         *(volatile int*)&sh.slot_gen[slot] = ls;
-        const int pa = gst * SR, pb = min(P, pa + SR);
-        mbar_expect_tx(&sh.full_c[slot], (uint32_t)((pb - pa) * d * 4));
-        uint8_t* sg = ring + slot * kStageBytes;
-        uint8_t* su = sg + kStageBytes / 2;
-        for (int p = pa; p < pb;) {  // runs of consecutive rows of one expert
-          const int ui = p / m, j = p - ui * m;
-          const int run = min(pb - p, m - j);
-          const size_t off = ((size_t)sh.uexp[ui] * m + j) * d;
-          bulk_g2s(sg + (size_t)(p - pa) * d * 2, a.wg + off, (uint32_t)(run * d * 2),
+        // rows j0 .. j0 + 3 of W^gate, then of W^up, one padded row each
+        const int pa = gst * kStagePairs, ui = pa / m, j0 = pa - ui * m;
+        const size_t off = ((size_t)sh.uexp[ui] * m + j0) * d;
+        mbar_expect_tx(&sh.full_c[slot], (uint32_t)(kStageRows * d * 2));
+        uint8_t* sg = ring + (size_t)slot * kStageBytes;
+        for (int n = 0; n < kStagePairs; ++n) {
+          bulk_g2s(sg + (size_t)n * rs, a.wg + off + (size_t)n * d, (uint32_t)(d * 2),
                    &sh.full_c[slot]);
-          bulk_g2s(su + (size_t)(p - pa) * d * 2, a.wu + off, (uint32_t)(run * d * 2),
-                   &sh.full_c[slot]);
-          p += run;
+          bulk_g2s(sg + (size_t)(n + kStagePairs) * rs, a.wu + off + (size_t)n * d,
+                   (uint32_t)(d * 2), &sh.full_c[slot]);
         }
       }
-      // end marks: every compute warp draws at most one item past the last
-      // stage, so the next kCompWarps / SR stages (at most the ring) carry none
-      for (int e = 0; e < kEndStages && ok; ++e) {
-        const int st = ls + e, slot = st % nring;
-        if (e > 0) ok = wait_bar(&sh.empty_c[slot], ((st / nring) & 1) ^ 1u, a, sh);
-        if (ok) {
-          sh.slot_stage[slot] = -1;
-          *(volatile int*)&sh.slot_gen[slot] = st;
-          mbar_arrive(&sh.full_c[slot]);
-        }
-      }
+      // the CTA's stage count: warps that drew a stage number at or past it leave
+      *(volatile int*)&sh.n_ls = ls;
       if (ok && n_pre > 0) {
         // once every phase-C stage is consumed, the first W^down stages go in
         for (int st = max(0, ls - nring); st < ls && ok; ++st)
@@ -491,82 +515,123 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       }
     }
   } else {
-    // Items are (stage, row pair), drawn in order from a CTA counter by
-    // whichever warp is free: the warp forms the pair's gate and up dots
-    // over the whole hidden size for every kept token of its expert and
-    // writes h = SiLU(gate) * up.  A warp may draw an item of a stage one
-    // lap ahead of the ring, so it first waits for the producer to have
-    // claimed the slot for that stage (slot_gen), then for the data.
-    const int nvc = d / 8;  // 16-byte chunks per row
-    const uint4* xq = reinterpret_cast<const uint4*>(xb);
+    // Items are drawn in order from a CTA counter by whichever warp is free.
+    // A warp may draw an item of a stage up to a ring lap ahead, so it first
+    // waits until the producer has claimed the slot for that stage
+    // (slot_gen) or has published the CTA's stage count (n_ls), then for the
+    // data.  Two forms of item, by token count:
+    //  * NT >= 3: a whole stage.  The warp forms on the tensor cores
+    //    (m16n8k16, bf16 operands, fp32 accumulation) the dots of the call's
+    //    tokens (MMA rows; rows NT .. 15 are zero) with the stage's 8 rows
+    //    (MMA columns: 4 gate, 4 up) over the whole hidden size.  In each
+    //    32-wide block of the hidden size, lane (g, q) holds the elements
+    //    8q .. 8q + 7 of token g's bf16(x) and of staged row g; the block's
+    //    two MMAs take elements 8q + {0..3} and 8q + {4..7} as the k of their
+    //    fragments, the same permutation of the block's 32 k on both
+    //    operands, so each MMA sums exact products of matching elements.
+    //    One warp per stage keeps several stages in work at once, so the
+    //    ring turns over at the rate the weights arrive.
+    //  * NT <= 2: one (gate, up) row pair of a stage, dotted on the CUDA
+    //    cores with each kept token of the pair's expert; the four pairs of
+    //    a stage go to four warps, which finishes a stage sooner when a CTA
+    //    has only a few.
+    // Either way the warp writes h = SiLU(gate) * up for the tokens that
+    // kept the stage's expert.
+    constexpr int kItems = NT > 2 ? 1 : kStagePairs;  // items per stage
+    const int g = lane >> 2, q = lane & 3;
+    const int nblk = d / 32;
+    const uint8_t* xrow = reinterpret_cast<const uint8_t*>(xb) + (size_t)g * rs + 16 * q;
     for (;;) {
       int it = 0;
       if (lane == 0) it = atomicAdd(&sh.item_ctr, 1);
       it = __shfl_sync(0xffffffffu, it, 0);
-      const int ls = it / SR, r = it - ls * SR;
+      const int ls = it / kItems, r = it - ls * kItems;
       const int slot = ls % nring;
-      {
-        bool claimed = true;
-        const uint64_t t0 = global_ns();
-        while (*(volatile int*)&sh.slot_gen[slot] != ls) {
-          if (sh.abort || global_ns() - t0 > kWaitLimitNs) {
-            if (!sh.abort) raise_flag(a.status, ACE_FLAG_TIMEOUT);
-            sh.abort = 1;
-            claimed = false;
-            break;
-          }
-        }
-        if (!claimed) break;
-      }
+      if (!await_stage(a, sh, slot, ls)) break;
       if (!wait_bar(&sh.full_c[slot], (ls / nring) & 1, a, sh)) break;
       const int gst = sh.slot_stage[slot];
-      if (gst < 0) break;
-      const int pa = gst * SR, nr = min(P, pa + SR) - pa;
-      if (r < nr) {
-        const int p = pa + r;
+      const uint8_t* stage = ring + (size_t)slot * kStageBytes;
+      if constexpr (NT > 2) {
+        (void)r;
+        const uint8_t* wrow = stage + (size_t)g * rs + 16 * q;
+        float c[4][4];  // four accumulators (blocks mod 4), so the MMA chains overlap
+#pragma unroll
+        for (int j = 0; j < 4; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.f;
+        for (int b0 = 0; b0 < nblk; b0 += 4) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int blk = b0 + j;
+            if (blk < nblk) {
+              uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+              if (g < NT) xv = *reinterpret_cast<const uint4*>(xrow + blk * 64);
+              const uint4 wv = *reinterpret_cast<const uint4*>(wrow + blk * 64);
+              mma_bf16_m16n8k16(c[j], xv.x, xv.y, wv.x, wv.y);
+              mma_bf16_m16n8k16(c[j], xv.z, xv.w, wv.z, wv.w);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty_c[slot]);  // the warp's reads of the slot are done
+        // token g with staged rows 2q, 2q + 1: gate rows of pairs 2q, 2q + 1
+        // on lanes q = 0, 1; the matching up rows (4 + 2q, 5 + 2q) two lanes up
+        const float d0 = (c[0][0] + c[1][0]) + (c[2][0] + c[3][0]);
+        const float d1 = (c[0][1] + c[1][1]) + (c[2][1] + c[3][1]);
+        const float u0 = __shfl_down_sync(0xffffffffu, d0, 2);
+        const float u1 = __shfl_down_sync(0xffffffffu, d1, 2);
+        if (q < 2 && g < NT) {
+          const int pa = gst * kStagePairs, ui = pa / m, j0 = pa - ui * m;
+          const uint32_t mk = sh.tok_mask[sh.uexp[ui]];
+          if ((mk >> g) & 1u) {
+            const int si = sh.ufirst[ui] + __popc(mk & ((1u << g) - 1u));
+            __nv_bfloat16* hp = a.h + (size_t)si * m + j0 + 2 * q;
+            hp[0] = __float2bfloat16_rn(silu(d0) * u0);
+            hp[1] = __float2bfloat16_rn(silu(d1) * u1);
+          }
+        }
+      } else {
+        const int p = gst * kStagePairs + r;
         const int ui = p / m, j = p - ui * m;
         const int s0 = sh.ufirst[ui], nt = sh.ufirst[ui + 1] - s0;  // <= NT
-        const uint4* wg =
-            reinterpret_cast<const uint4*>(ring + slot * kStageBytes + (size_t)r * d * 2);
-        const uint4* wu = reinterpret_cast<const uint4*>(ring + slot * kStageBytes +
-                                                         kStageBytes / 2 + (size_t)r * d * 2);
+        const uint4* wg = reinterpret_cast<const uint4*>(stage + (size_t)r * rs);
+        const uint4* wu = reinterpret_cast<const uint4*>(stage + (size_t)(r + kStagePairs) * rs);
+        const uint4* xq = reinterpret_cast<const uint4*>(xb);
         int xo[NT];  // each kept token's row of bf16(x), in 16-byte chunks
 #pragma unroll
-        for (int q = 0; q < NT; ++q) xo[q] = (q < nt ? sh.slot_t[s0 + q] : 0) * nvc;
+        for (int t = 0; t < NT; ++t) xo[t] = (t < nt ? sh.slot_t[s0 + t] : 0) * (rs / 16);
         float ga[NT], ua[NT];
 #pragma unroll
-        for (int q = 0; q < NT; ++q) ga[q] = ua[q] = 0.f;
-        for (int c = lane; c < nvc; c += 32) {
+        for (int t = 0; t < NT; ++t) ga[t] = ua[t] = 0.f;
+        for (int cc = lane; cc < d / 8; cc += 32) {
           float w1[8], w2[8];
-          bf16x8_to_f32(wg[c], w1);
-          bf16x8_to_f32(wu[c], w2);
+          bf16x8_to_f32(wg[cc], w1);
+          bf16x8_to_f32(wu[cc], w2);
 #pragma unroll
-          for (int q = 0; q < NT; ++q) {
-            if (q < nt) {
+          for (int t = 0; t < NT; ++t) {
+            if (t < nt) {
               float xv[8];
-              bf16x8_to_f32(xq[xo[q] + c], xv);
+              bf16x8_to_f32(xq[xo[t] + cc], xv);
 #pragma unroll
-              for (int cc = 0; cc < 8; ++cc) {
-                ga[q] = fmaf(w1[cc], xv[cc], ga[q]);
-                ua[q] = fmaf(w2[cc], xv[cc], ua[q]);
+              for (int e = 0; e < 8; ++e) {
+                ga[t] = fmaf(w1[e], xv[e], ga[t]);
+                ua[t] = fmaf(w2[e], xv[e], ua[t]);
               }
             }
           }
         }
 #pragma unroll
-        for (int q = 0; q < NT; ++q) {
-          if (q < nt) {
+        for (int t = 0; t < NT; ++t) {
+          if (t < nt) {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
-              ga[q] += __shfl_xor_sync(0xffffffffu, ga[q], o);
-              ua[q] += __shfl_xor_sync(0xffffffffu, ua[q], o);
+              ga[t] += __shfl_xor_sync(0xffffffffu, ga[t], o);
+              ua[t] += __shfl_xor_sync(0xffffffffu, ua[t], o);
             }
-            if (lane == q) a.h[(size_t)(s0 + q) * m + j] = __float2bfloat16_rn(silu(ga[q]) * ua[q]);
+            if (lane == t) a.h[(size_t)(s0 + t) * m + j] = __float2bfloat16_rn(silu(ga[t]) * ua[t]);
           }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty_c[slot]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.empty_c[slot]);
     }
   }
   __syncthreads();  // every kept slot's h of this CTA's stages is written
@@ -701,20 +766,17 @@ cudaError_t launch_nt(cudaLaunchConfig_t& cfg, const DecodeArgs& a, size_t smem)
 // unrounded fp32 x and the staged inputs of phase A live inside the ring.
 static size_t region_bytes(int T, int d, int m, int k, int E, int num_sms) {
   (void)m, (void)k, (void)E, (void)num_sms;
-  return (size_t)T * d * 2;  // bf16(x)
+  return (size_t)T * row_stride(d);  // bf16(x), padded rows
 }
 
 static int ring_stages(int T, int d, int m, int k, int E, int num_sms) {
   const size_t avail = (size_t)kSmemBudget - sizeof(DecShared) - 1024 -
                        region_bytes(T, d, m, k, E, num_sms);
-  int n = (int)(avail / kStageBytes);
-  n = n > kRing ? kRing : n;
-  // even: phase C's two consumer groups take alternate stages, so with an
-  // even ring each slot belongs to one group, which waits on the slot's fills
-  // in order.  With an odd ring a slot alternates between the groups, and a
-  // group running a lap ahead would test the slot's full barrier for a parity
-  // that an older, already completed phase also has.
-  return n & ~1;
+  const int n = (int)(avail / kStageBytes);
+  // any depth: a warp waits on a slot's full barrier only once the producer
+  // has claimed the slot for the warp's stage (the slot's earlier fill is
+  // then complete and consumed), so no wait can see an older phase
+  return n > kRing ? kRing : n;
 }
 
 // All the shared memory a CTA can have: phase C uses its ring and bf16(x),
@@ -727,7 +789,7 @@ size_t decode_smem_bytes(int T, int d, int m, int k, int E, int num_sms) {
 bool decode_fits(int T, int d, int m, int k, int E, int num_sms) {
   if (T < 1 || T > kDecodeMaxT || d > 2048 || d % 32 != 0 || m % 8 != 0) return false;
   const int n = ring_stages(T, d, m, k, E, num_sms);
-  if (n < kEndStages) return false;  // the end marks take kEndStages distinct slots
+  if (n < 2) return false;
   // phase A inside the ring: x (fp32), u (bf16), gamma, the router rows
   const size_t staged = (size_t)T * d * 6 + (size_t)d * 4 +
                         (size_t)((E + num_sms - 1) / num_sms) * d * 2;
