@@ -222,7 +222,7 @@ def test_full_prefill_8192_e256_skewed():
 
 
 # ------------------------------------------------------------------ decode
-@pytest.mark.parametrize("T", [1, 3, 8])
+@pytest.mark.parametrize("T", [1, 2, 3, 8])
 def test_full_shape_decode(T):
     """T <= 8 runs the cooperative decode kernel: Qwen3-30B-A3B layer shape,
     every token's routing, mask, slot order and output compared."""
@@ -273,6 +273,21 @@ def test_decode_back_to_back_launches(T):
     bad = [i for i in range(n) if ace.ace_read_status(wss[i]) != (ace.ACE_OK, 0)]
     assert bad == [], bad[:10]
     assert torch.equal(ys, y0.unsqueeze(0).expand_as(ys))
+
+
+@pytest.mark.parametrize("T,d", [(2, 288), (6, 288), (3, 96), (7, 2048)])
+def test_decode_item_forms_and_strides(T, d):
+    """Both forms of the decode kernel's gate/up items: row pairs on the CUDA
+    cores below 3 tokens, whole stages on the tensor cores from 3.  The hidden
+    sizes cover staged rows that need no padding (2d = 576 is 64 modulo 128)
+    and an MMA block count that leaves the unrolled group of four part empty
+    (d = 96: 3 blocks of 32)."""
+    w = W("dec_forms", T=T, d=d, E=32, m=128, k=8, dtype="bf16", bias=True, skip=0.5,
+          skip_of="slots")
+    layer, u, A_gsp, A_rcr, amax, tau, _ = setup_case(w, tables="spread")
+    gpu = run_gpu(layer, u, amax, tau)
+    res = compare(layer, u, gpu, A_gsp, A_rcr, tau)
+    assert res["compared_tokens"] >= T - 1  # run_gpu has checked the status word
 
 
 @pytest.mark.parametrize("tau", [-1.0, float("inf")])
