@@ -110,7 +110,7 @@ struct DecShared {
   uint64_t h_bar;              // phase D: h of the kept slots has landed
   int slot_stage[kRing];       // phase C: the stage a ring slot holds (-1: no more)
   int slot_gen[kRing];         // phase C: the CTA's stage number a slot was last claimed for
-  int item_ctr;                // phase C: the CTA's next stage number to hand to a warp
+  int item_ctr;                // phase C: the CTA's next item (a stage, or a stage's row pair)
   int n_ls;                    // phase C: the CTA's stage count, once known (else INT_MAX)
   int abort;
 };
@@ -444,7 +444,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const uint32_t dstage = (dbytes + 1023u) & ~1023u;
   __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(dsm);
   uint8_t* ring_d = dsm + hbytes;
-  // even, like phase C's ring: the two consumer groups take alternate stages
+  // even: phase D's two consumer groups take alternate experts, so each slot
+  // belongs to one group, which waits on the slot's fills in order
   const int nring_d =
       dstage ? (int)min((size_t)kRingD, (a.dyn_bytes - 1024 - hbytes) / dstage) & ~1 : 2;
   // stages that lie inside phase C's ring (free once its last stage is
