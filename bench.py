@@ -311,13 +311,20 @@ def run_ours(args, w, rate, ws_n, rank, local):
     # small slot tiles: both GEMMs run as one kernel and the library records
     # "mid" after it ("mid" = "end"): the dominant kernel is then the fused one
     fused = dn_ms < 0.02 * gu_ms
+    # algorithmic bytes (the method's): the touched experts' weights and the
+    # layer's input X and output Y; the design's own intermediates (gathered
+    # rows, h, per-slot outputs) are reported beside them
+    x_bytes = w.T * d * 2
     if fused:
         kname = "k_experts_fused (gate/up + SiLU and down GEMMs, one launch)"
-        k_bytes, k_ms = gu_bytes + dn_bytes, gu_ms + dn_ms
+        k_bytes, k_ms = touched * 3 * m * d * 2 + 2 * x_bytes, gu_ms + dn_ms
+        k_bytes_incl = gu_bytes + dn_bytes
     else:
         kname = "k_experts<0> (gate/up GEMM + SiLU)"
-        k_bytes, k_ms = gu_bytes, gu_ms
+        k_bytes, k_ms = touched * 2 * m * d * 2 + x_bytes, gu_ms
+        k_bytes_incl = gu_bytes
     k_gbs = k_bytes / (k_ms / 1e3) / 1e9
+    k_gbs_incl = k_bytes_incl / (k_ms / 1e3) / 1e9
     dn_gbs = dn_bytes / (dn_ms / 1e3) / 1e9 if not fused else None
     flops = S * 2 * d * 3 * m
     layer_bytes = touched * 3 * d * m * 2 + w.T * d * 2 * 2 + w.E * d * 2
@@ -358,15 +365,19 @@ def run_ours(args, w, rate, ws_n, rank, local):
         "config": {"workload": w.name, "tokens": w.T, "hidden": w.d, "experts": w.E,
                    "expert_ffn": w.m, "top_k": w.k, "skip_rate": rate,
                    "skip_of": w.skip_of, "router_bias": w.bias, "tau": st["tau"],
-                   "realised_skip": ss["skipped"] / (w.T * w.k), "kept_slots": S,
-                   "touched_experts": touched, "tables": st["tables"],
-                   "parallelism": "replicas" if ws_n > 1 else "single", "step_ms": spread,
+                   "parallelism": "replicas" if ws_n > 1 else "single",
                    "launch": "forward captured in one CUDA graph, replayed per step",
                    "l2": "flushed before each timed step (256 MiB write), flush untimed"},
+        "workload_stats": {"realised_skip": ss["skipped"] / (w.T * w.k), "kept_slots": S,
+                           "touched_experts": touched, "tables": st["tables"],
+                           "step_ms": spread},
         "roofline": {"bound": "hbm", "achieved": k_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": k_gbs / pk["hbm_gbs"],
                      "traffic": profiled_traffic(w.name, "fused" if fused else "gateup"),
                      "kernel": kname, "algorithmic_bytes": k_bytes, "kernel_ms": k_ms,
+                     "algorithmic": "touched experts' weights + X in + Y out",
+                     "bytes_incl_intermediates": k_bytes_incl,
+                     "frac_incl_intermediates": k_gbs_incl / pk["hbm_gbs"],
                      "peak_source": pk["source"]},
         "kernels": {
             "down": ({"fused": True} if fused else
@@ -706,31 +717,62 @@ def _oracle_inputs(st):
     return layer, u, amax
 
 
-def cpu_baseline(w, st, rate, target_s=12.0):
+def oracle_pass_size(layer, u, tau, amax, budget_s):
+    """Tokens per oracle pass: the whole batch, or the prefix of it that the
+    oracle finishes in about budget_s seconds (from a 4-token probe)."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.moe_forward(layer, u[:4], tau, amax, amax)
+    per_tok = (time.perf_counter() - t0) / 4
+    return int(max(4, min(u.shape[0], budget_s / max(per_tok, 1e-9))))
+
+
+def oracle_passes(layer, u, tau, amax, n, passes, warm=1):
+    """Seconds of each of `passes` oracle forwards over the first n tokens,
+    after `warm` untimed ones.  Both oracle timings of this script (the
+    cpu_baseline leg and the reference arm) run through here, under one
+    condition: torch's own CPU thread pool is held at one thread meanwhile,
+    so the host cores belong to the oracle's threads."""
+    import oracle
+    nt = torch.get_num_threads()
+    torch.set_num_threads(1)
+    try:
+        for _ in range(warm):
+            oracle.moe_forward(layer, u[:n], tau, amax, amax)
+        times = []
+        for _ in range(passes):
+            t0 = time.perf_counter()
+            oracle.moe_forward(layer, u[:n], tau, amax, amax)
+            times.append(time.perf_counter() - t0)
+    finally:
+        torch.set_num_threads(nt)
+    return times
+
+
+def cpu_baseline(w, st, rate, target_s=12.0, pass_budget_s=6.0):
     """The oracle as it stands on the host cores, on a bounded sample of the
-    same workload: whole passes over the batch's tokens (or a prefix of them)
-    until about target_s seconds of CPU work."""
+    same workload: one warm-up pass, then whole passes over the batch's
+    tokens (or the prefix that fits pass_budget_s) until about target_s
+    seconds of CPU work."""
     import oracle
     layer, u, amax = _oracle_inputs(st)
-    n = min(w.T, 64)
-    t0 = time.perf_counter()
-    oracle.moe_forward(layer, u[:n], st["tau"], amax, amax)
-    per_tok = (time.perf_counter() - t0) / n
-    n = int(max(8, min(w.T, target_s / max(per_tok, 1e-9))))
-    done, t0 = 0, time.perf_counter()
-    while True:
-        oracle.moe_forward(layer, u[:n], st["tau"], amax, amax)
-        done += n
-        dt = time.perf_counter() - t0
-        if dt >= target_s or done >= 64 * w.T:
-            break
-    return {"value": done / dt, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
-            "sample": "%d tokens (passes over the first %d of the batch's %d; fp64 forward incl. "
-                      "routing, mask and combine), %.1f s" % (done, n, w.T, dt)}
+    n = oracle_pass_size(layer, u, st["tau"], amax, pass_budget_s)
+    t1 = oracle_passes(layer, u, st["tau"], amax, n, 1, warm=1)[0]
+    passes = int(max(1, min(64, target_s / max(t1, 1e-9)) - 1))
+    times = [t1] + oracle_passes(layer, u, st["tau"], amax, n, passes, warm=0)
+    dt = sum(times)
+    return {"value": len(times) * n / dt, "unit": "tokens/s", "cores": oracle.threads(),
+            "kind": "oracle",
+            "sample": "%d passes over the first %d of the batch's %d tokens after one warm-up "
+                      "pass (fp64 forward incl. routing, mask and combine), %.1f s; pass "
+                      "%.3f-%.3f s; torch CPU threads held at 1" % (
+                          len(times), n, w.T, dt, min(times), max(times))}
 
 
 def run_reference(args, w, rate):
-    """The reference arm: the fp64 CPU oracle, each step a bounded sample."""
+    """The reference arm: the fp64 CPU oracle, each step one pass over a
+    bounded sample of the batch.  The untimed set-up (layer, tables, tau)
+    is the GPU arm's own, so both arms see the same workload."""
     import oracle
     dev = torch.device("cuda", 0) if torch.cuda.is_available() else None
     if dev is None:
@@ -738,33 +780,35 @@ def run_reference(args, w, rate):
         u = workloads.make_tokens(w)
         amax = np.ones(w.E, dtype=np.float32)
         tau = 0.0
+        layer = {k: (v.float().numpy() if torch.is_tensor(v) else v) for k, v in layer.items()}
+        u = u.double().numpy()
     else:
         st = setup_prefill(w, rate, dev)
         layer, u, amax = _oracle_inputs(st)
         tau = st["tau"]
-    t0 = time.perf_counter()
-    oracle.moe_forward(layer, u[:4], tau, amax, amax)
-    per_tok = (time.perf_counter() - t0) / 4
     budget = 150.0 / max(1, args.steps + args.warmup)
-    n = int(max(4, min(w.T, budget / max(per_tok, 1e-6))))
-    for _ in range(args.warmup):
-        oracle.moe_forward(layer, u[:n], tau, amax, amax)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle.moe_forward(layer, u[:n], tau, amax, amax)
-    dt = time.perf_counter() - t0
+    n = oracle_pass_size(layer, u, tau, amax, budget)
+    times = oracle_passes(layer, u, tau, amax, n, args.steps, warm=args.warmup)
+    dt = sum(times)
     val = args.steps * n / dt
-    unit, sample = "tokens/s", "%d of %d tokens per step" % (n, w.T)
+    unit = "tokens/s"
+    sample = "%d of %d tokens per step (one oracle pass), %d warm-up passes; pass %.3f-%.3f s; " \
+             "torch CPU threads held at 1" % (n, w.T, args.warmup, min(times), max(times))
     if w.name.startswith("stack"):  # one layer timed; the chain costs layers times as much
         val /= w.layers
         unit = "tokens/s (through all %d chained MoE layers)" % w.layers
         sample += "; one layer timed, the %d-layer rate is its rate / %d" % (w.layers, w.layers)
+    config = {"workload": w.name, "tokens": w.T, "hidden": w.d, "experts": w.E,
+              "expert_ffn": w.m, "top_k": w.k, "skip_rate": rate, "skip_of": w.skip_of,
+              "router_bias": w.bias, "tau": tau,
+              "parallelism": "replicas" if args.gpus > 1 else "single",
+              "launch": "one oracle pass per step on the host cores",
+              "l2": "not applicable: the oracle runs on the host"}
     return {"metric": METRIC, "value": val, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "tokens": w.T, "hidden": w.d, "experts": w.E,
-                       "expert_ffn": w.m, "top_k": w.k, "skip_rate": rate},
+            "data": "synthetic (seeded N(0,0.02) weights, N(0,1) tokens)", "impl": "reference",
+            "config": config,
             "cpu_baseline": {"value": val, "unit": unit, "kind": "oracle",
                              "cores": oracle.threads(), "sample": sample},
             "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0,

@@ -260,16 +260,30 @@ ACE_API ace_status ace_moe_scores(const ace_layer* layer, const void* u, int T,
  *     each call zeroes what must start at zero.  Calls whose GPU work
  *     overlaps (on different streams or host threads) race on the array:
  *     serialise them.
- *   - Shapes whose scratch exceeds the array (router logits T x E fp32,
- *     gated intermediates T x k x m bf16, slot tables), non-bf16 layers and
- *     shapes the decode kernel does not serve return ACE_ERR_UNSUPPORTED
- *     before anything is launched; bad pointers return ACE_ERR_INVALID_ARG.
- *   - Device-detected flags stay in the array (there is no workspace to
- *     read them from); the kernel's waits are bounded as elsewhere.
+ *   - The layer checks and shape rule are ace_moe_forward's (bf16 layers
+ *     need d % 128 == 0 and m % 128 == 0).  Shapes whose scratch exceeds the
+ *     array (router logits T x E fp32, gated intermediates T x k x m bf16,
+ *     slot tables), non-bf16 layers and shapes the decode kernel does not
+ *     serve return ACE_ERR_UNSUPPORTED before anything is launched; bad
+ *     pointers return ACE_ERR_INVALID_ARG.
+ *   - Device-detected flags go to a status word in the array; read them
+ *     with ace_noalloc_read_status.  The kernel's waits are bounded as
+ *     elsewhere.
  *   Results equal ace_moe_forward's for the same inputs.
  * ---------------------------------------------------------------------- */
 ACE_API ace_status ace_moe_decode_noalloc(const ace_layer* layer, const void* u, int T,
                                           const ace_fwd_opts* opts, void* y, void* stream);
+
+/* ------------------------------------------------------------------------
+ * ace_noalloc_read_status -- synchronise `stream` and return the device
+ *   status word of the most recent ace_moe_decode_noalloc call on the
+ *   current device (ACE_FLAG_* bits in *flags, which may be NULL), read
+ *   from the library's scratch array; ACE_ERR_TIMEOUT / ACE_ERR_DEVICE_FAULT
+ *   when the corresponding bit is set, else ACE_OK.  Allocates nothing.
+ *   Like the array itself, the word is shared by every call on the device:
+ *   read it before the next call is enqueued.
+ * ---------------------------------------------------------------------- */
+ACE_API ace_status ace_noalloc_read_status(uint32_t* flags, void* stream);
 
 /* ------------------------------------------------------------------------
  * ace_tables_workspace_size
@@ -340,6 +354,23 @@ ACE_API ace_status ace_read_status(void* ws, size_t ws_bytes, uint32_t* flags,
 
 /* Human-readable name of a status code (static storage). */
 ACE_API const char* ace_status_str(ace_status s);
+
+/* ------------------------------------------------------------------------
+ * ace_set_peer_wait_limit_ns -- time limit of the waits in which one CTA of
+ *   a kernel waits for other CTAs of the same launch: the decode kernel's
+ *   two grid barriers (T <= 8) and, in the prefill's fused expert kernel, a
+ *   down item's wait for the h rows of its tile.  The paper has no
+ *   counterpart: it is a robustness setting of this implementation.
+ *   Default 2 s (ns == 0 restores it).  A wait that runs out sets
+ *   ACE_FLAG_TIMEOUT in the call's status word; the kernel then lets every
+ *   copy it issued land, frees its tensor memory and returns, so the
+ *   context stays usable and the next call runs normally (outputs of the
+ *   timed-out call are undefined).  Process-wide; read when a call enqueues
+ *   its kernels, so a captured CUDA graph keeps the value of its capture.
+ *   Waits inside one CTA (on its own copies and MMAs) keep the fixed 2 s
+ *   bound.  Returns the previous limit.
+ * ---------------------------------------------------------------------- */
+ACE_API uint64_t ace_set_peer_wait_limit_ns(uint64_t ns);
 
 /* Name and description of the CUDA runtime error behind the most recent
  * ACE_ERR_CUDA returned on the calling thread ("no error" if none), static

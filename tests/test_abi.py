@@ -176,3 +176,33 @@ def test_stack_rejects_bad_calls(ace):
     opts[2].fusion = 1                                                 # min without view tables
     assert f(Ls, 3, ok["u"], 4, opts, ok["y"], ok["ws"], ok["nb"], None) == \
         ace.ACE_ERR_INVALID_ARG
+
+
+def test_noalloc_rejects_bad_calls_before_any_device_call(ace):
+    """ace_moe_decode_noalloc applies ace_moe_forward's layer checks and shape
+    rule, and its own token range, on the host."""
+    f = ace.lib().ace_moe_decode_noalloc
+    opts = ace.ace_fwd_opts(tau=0.1, renorm_topk=1, fusion=0, eps_rms=1e-6)
+    L = _fake_layer(ace)
+    u, y = 0x20000, 0x40000
+    assert f(ctypes.byref(L), u, 9, ctypes.byref(opts), y, None) == ace.ACE_ERR_INVALID_ARG
+    assert f(ctypes.byref(L), u, 0, ctypes.byref(opts), y, None) == ace.ACE_ERR_INVALID_ARG
+    assert f(ctypes.byref(L), u, 4, None, y, None) == ace.ACE_ERR_INVALID_ARG
+    assert f(ctypes.byref(L), u, 4, ctypes.byref(opts), u + 64, None) == ace.ACE_ERR_INVALID_ARG
+    assert f(ctypes.byref(L), u + 8, 4, ctypes.byref(opts), y, None) == ace.ACE_ERR_INVALID_ARG
+    for bad in (dict(d=192), dict(m=192), dict(d=100), dict(E=1024)):
+        assert f(ctypes.byref(_fake_layer(ace, **bad)), u, 4, ctypes.byref(opts), y,
+                 None) == ace.ACE_ERR_UNSUPPORTED, bad
+    assert f(ctypes.byref(_fake_layer(ace, dtype=ace.ACE_F32)), u, 4, ctypes.byref(opts), y,
+             None) == ace.ACE_ERR_UNSUPPORTED
+    assert f(ctypes.byref(_fake_layer(ace, k=0)), u, 4, ctypes.byref(opts), y,
+             None) == ace.ACE_ERR_INVALID_ARG
+
+
+def test_peer_wait_limit_setting(ace):
+    """Process-wide limit of the cross-CTA waits: 2 s by default, 0 restores
+    the default, the previous value is returned."""
+    assert ace.ace_set_peer_wait_limit_ns(0) == 2_000_000_000
+    assert ace.ace_set_peer_wait_limit_ns(5000) == 2_000_000_000
+    assert ace.ace_set_peer_wait_limit_ns(0) == 5000
+    assert ace.ace_set_peer_wait_limit_ns(0) == 2_000_000_000

@@ -176,10 +176,30 @@ def test_forward_on_a_side_stream():
 
 
 # ------------------------------------------------------------ full sizes
-def _full(w, n_out=48, seed=0):
+def tile_covering_tokens(gpu, n_out, tile_n=256, seed=0):
+    """Tokens whose outputs cover every expert GEMM tile at both ends: the
+    tokens of the first and last kept slot of each (expert, 256-slot tile),
+    topped up with random tokens to n_out."""
+    off = gpu["expert_offsets"]
+    st = gpu["slot_token"]
+    toks = set()
+    for e in range(len(off) - 1):
+        for a in range(off[e], off[e + 1], tile_n):
+            b = min(off[e + 1], a + tile_n) - 1
+            toks.update((int(st[a]), int(st[b])))
+    T = gpu["keep"].shape[0]
+    rng = np.random.default_rng(seed)
+    rest = np.setdiff1d(np.arange(T), np.fromiter(toks, dtype=np.int64))
+    extra = max(0, n_out - len(toks))
+    toks.update(rng.choice(rest, size=min(extra, rest.size), replace=False).tolist())
+    return np.array(sorted(toks))
+
+
+def _full(w, n_out=None, seed=0):
     """Full-size layer drawn on the GPU (the CPU copy feeds the oracle); RCR
-    table from the oracle, a spread GSP table; every token's routing and
-    mask compared, outputs on a sample of tokens."""
+    table from the oracle, a spread GSP table; every token's routing, mask and
+    slot lists compared; outputs on every token (n_out None) or on n_out
+    tokens that cover every expert GEMM tile."""
     layer = workloads.make_layer(w, seed=seed, device="cuda")
     u = workloads.make_tokens(w, device="cuda")
     layer_cpu = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in layer.items()}
@@ -193,11 +213,10 @@ def _full(w, n_out=48, seed=0):
     n = oracle.n_skip_for(w.T, w.k, w.skip, of=w.skip_of)
     tau = midpoint_tau(ref["c"], n)
     gpu = run_gpu(layer_cpu, u_cpu, np.maximum(A_gsp, A_rcr), tau)
-    rng = np.random.default_rng(0)
-    toks = np.sort(rng.choice(w.T, size=n_out, replace=False))
+    toks = None if n_out is None else tile_covering_tokens(gpu, n_out)
     res = compare(layer_cpu, u_cpu, gpu, A_gsp, A_rcr, tau, out_tokens=toks)
     print(w.name, res)
-    return res, gpu, n
+    return res, gpu, n, toks
 
 
 # The tensor-core router sums exact bf16 x bf16 products of a three-term split
@@ -208,16 +227,21 @@ ROUTER_TC_REL = 5e-7
 
 
 def test_full_prefill_1024():
-    res, gpu, n = _full(workloads.WORKLOADS["prefill_1024"])
+    res, gpu, n, _ = _full(workloads.WORKLOADS["prefill_1024"])
+    assert res["compared_tokens"] + res["excluded_tokens"] == 1024  # every token's output
+    assert res["slots_checked"] == int(gpu["n_kept"][0])
     assert res["mask_mismatch"] == 0
     assert abs(int((gpu["keep"] == 0).sum()) - n) <= res["band"] + res["ties"] * 8
     assert res["logit_err"] <= ROUTER_TC_REL * res["logit_scale"], res
 
 
 def test_full_prefill_8192_e256_skewed():
-    res, gpu, n = _full(workloads.WORKLOADS["prefill_8192_e256"], n_out=32)
+    res, gpu, n, toks = _full(workloads.WORKLOADS["prefill_8192_e256"], n_out=1024)
     counts = np.diff(gpu["expert_offsets"])
     assert counts.max() > 256  # skewed: some experts need several slot tiles
+    assert toks.size >= 1024
+    assert res["compared_tokens"] + res["excluded_tokens"] == toks.size
+    assert res["slots_checked"] == int(gpu["n_kept"][0])
     assert res["logit_err"] <= ROUTER_TC_REL * res["logit_scale"], res
 
 
@@ -275,13 +299,13 @@ def test_decode_back_to_back_launches(T):
     assert torch.equal(ys, y0.unsqueeze(0).expand_as(ys))
 
 
-@pytest.mark.parametrize("T,d", [(2, 288), (6, 288), (3, 96), (7, 2048)])
+@pytest.mark.parametrize("T,d", [(2, 384), (6, 384), (3, 128), (7, 2048)])
 def test_decode_item_forms_and_strides(T, d):
     """Both forms of the decode kernel's gate/up items: row pairs on the CUDA
     cores below 3 tokens, whole stages on the tensor cores from 3.  The hidden
-    sizes cover staged rows that need no padding (2d = 576 is 64 modulo 128)
-    and an MMA block count that leaves the unrolled group of four part empty
-    (d = 96: 3 blocks of 32)."""
+    sizes give one (d = 128), three (384) and sixteen (2048) groups of four
+    32-wide MMA blocks per staged row, and phase-D row counts per CTA of one,
+    three and fourteen."""
     w = W("dec_forms", T=T, d=d, E=32, m=128, k=8, dtype="bf16", bias=True, skip=0.5,
           skip_of="slots")
     layer, u, A_gsp, A_rcr, amax, tau, _ = setup_case(w, tables="spread")

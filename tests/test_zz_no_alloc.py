@@ -46,7 +46,7 @@ def test_noalloc_decode_matches_workspace_forward(T):
         ace.ace_moe_forward(L, u, tau, y_ref, ws)
         y = torch.full_like(u, float("nan"))
         ace.ace_moe_decode_noalloc(L, u, tau, y)
-        torch.cuda.synchronize()
+        assert ace.ace_noalloc_read_status() == (ace.ACE_OK, 0), call  # the array's status word
         assert torch.isfinite(y.float()).all()
         assert _rel(y, y_ref) <= 2e-2, (call, _rel(y, y_ref))
         assert torch.equal(y, y_ref), call  # same kernel, same inputs: identical bits
@@ -79,4 +79,17 @@ def test_noalloc_rejects_what_it_cannot_serve():
     yb = torch.zeros_like(ub)
     assert f(ctypes.byref(Lb), ctypes.c_void_p(ub.data_ptr()), 8, ctypes.byref(opts),
              ctypes.c_void_p(yb.data_ptr()), s) == ace.ACE_ERR_UNSUPPORTED
+    # the shape rule of ace_moe_forward: bf16 layers need d and m multiples of 128
+    odd = workloads.Workload("odd", T=4, d=192, E=16, m=128, k=4, dtype="bf16", bias=False,
+                             skip=0.5, skip_of="slots")
+    lo = workloads.make_layer(odd, seed=4, device="cuda")
+    Lo = ace.make_layer(lo["gamma"], lo["wr"], lo["wg"], lo["wu"], lo["wd"], odd.k)
+    uo = torch.zeros(4, odd.d, dtype=torch.bfloat16, device="cuda")
+    yo = torch.zeros_like(uo)
+    assert f(ctypes.byref(Lo), ctypes.c_void_p(uo.data_ptr()), 4, ctypes.byref(opts),
+             ctypes.c_void_p(yo.data_ptr()), s) == ace.ACE_ERR_UNSUPPORTED
+    wso = ace.alloc_workspace(1 << 20)
+    with pytest.raises(ace.AceError) as ei:
+        ace.ace_moe_forward(Lo, uo, 0.1, yo, wso)
+    assert ei.value.code == ace.ACE_ERR_UNSUPPORTED
     torch.cuda.synchronize()

@@ -82,6 +82,10 @@ _lib.ace_tau_workspace_size.restype = ctypes.c_size_t
 _lib.ace_tau_quantile.argtypes = [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp,
                                   ctypes.c_size_t, _vp]
 _lib.ace_tau_quantile.restype = ctypes.c_int
+_lib.ace_noalloc_read_status.argtypes = [_P(ctypes.c_uint32), _vp]
+_lib.ace_noalloc_read_status.restype = ctypes.c_int
+_lib.ace_set_peer_wait_limit_ns.argtypes = [ctypes.c_uint64]
+_lib.ace_set_peer_wait_limit_ns.restype = ctypes.c_uint64
 _lib.ace_read_status.argtypes = [_vp, ctypes.c_size_t, _P(ctypes.c_uint32), _vp]
 _lib.ace_read_status.restype = ctypes.c_int
 _lib.ace_status_str.argtypes = [ctypes.c_int]
@@ -248,6 +252,20 @@ def ace_read_status(ws, stream=None):
     flags = ctypes.c_uint32(0)
     code = _lib.ace_read_status(_ptr(ws), ws.numel(), ctypes.byref(flags), _stream(stream))
     return code, int(flags.value)
+
+
+def ace_noalloc_read_status(stream=None):
+    """Synchronise the stream; (status code, flag bits) of the last
+    ace_moe_decode_noalloc call on the current device."""
+    flags = ctypes.c_uint32(0)
+    code = _lib.ace_noalloc_read_status(ctypes.byref(flags), _stream(stream))
+    return code, int(flags.value)
+
+
+def ace_set_peer_wait_limit_ns(ns):
+    """Set the limit of cross-CTA waits (0: the 2 s default); returns the
+    previous limit."""
+    return int(_lib.ace_set_peer_wait_limit_ns(int(ns)))
 
 
 class DebugOut:

@@ -2,6 +2,8 @@
 // validation, the workspace layout, and the launch sequence of the forward.
 #include <string.h>
 
+#include <atomic>
+
 #include "ace_common.cuh"
 #include "ace_internal.h"
 #include "compact.cuh"
@@ -117,7 +119,17 @@ ace_status check_layer(const ace_layer* L, bool need_experts) {
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
+// Limit of the waits in which a CTA waits on other CTAs (ace_set_peer_wait_limit_ns).
+std::atomic<uint64_t> g_peer_wait_ns{kWaitLimitNs};
+
 }  // namespace
+
+namespace ace {
+ace_status validate_layer(const ace_layer* L, bool need_experts) {
+  return check_layer(L, need_experts);
+}
+uint64_t peer_wait_ns() { return g_peer_wait_ns.load(std::memory_order_relaxed); }
+}  // namespace ace
 
 namespace ace {
 // The fusion rule is known and the tables it reads are present.
@@ -471,7 +483,11 @@ const char* ace_status_str(ace_status s) {
   return "ACE_UNKNOWN_STATUS";
 }
 
-const char* ace_version(void) { return "0.1.0"; }
+uint64_t ace_set_peer_wait_limit_ns(uint64_t ns) {
+  return g_peer_wait_ns.exchange(ns == 0 ? kWaitLimitNs : ns);
+}
+
+const char* ace_version(void) { return "0.2.0"; }
 
 const char* ace_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
 

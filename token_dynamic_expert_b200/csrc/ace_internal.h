@@ -41,6 +41,13 @@ struct FwdLayout {
 FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms);
 
 int device_sm_count();
+// The argument and shape checks of a layer (need_experts: the expert weights
+// are read as well), shared by every entry point.
+ace_status validate_layer(const ace_layer* L, bool need_experts);
+// Current limit (ns) of the waits in which a CTA waits on other CTAs: the
+// decode kernel's grid barriers and the fused expert kernel's wait for a
+// tile's h rows.  Read when a call enqueues its kernels.
+uint64_t peer_wait_ns();
 // Zeroes n_words 32-bit words on the stream (the status block of a call).
 cudaError_t launch_clear_words(void* p, int n_words, cudaStream_t s);
 ace_status check_fusion(const ace_layer& L, int fusion);

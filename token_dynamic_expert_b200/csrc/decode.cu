@@ -49,10 +49,11 @@ constexpr int kStageRows = 2 * kStagePairs;         // staged rows: 4 gate, then
 constexpr int kMaxSlots = kDecodeMaxT * kMaxK;
 
 // Bytes between the rows of bf16(x) and between the staged weight rows of a
-// phase-C stage: 2d, plus 64 when 2d is a multiple of 128, so that rows n and
-// n + 1 start 64 bytes apart modulo 128 and the 16-byte loads of a quarter
-// warp (two rows, four consecutive 16-byte pieces of each) hit distinct banks.
-__host__ __device__ constexpr int row_stride(int d) { return 2 * d + ((2 * d) % 128 == 0 ? 64 : 0); }
+// phase-C stage: 2d + 64.  The hidden size is a multiple of 128, so 2d is a
+// multiple of 256 and the padding puts rows n and n + 1 64 bytes apart modulo
+// 128: the 16-byte loads of a quarter warp (two rows, four consecutive
+// 16-byte pieces of each) then hit distinct banks.
+__host__ __device__ constexpr int row_stride(int d) { return 2 * d + 64; }
 constexpr int kStageBytes = kStageRows * row_stride(2048);  // bytes per ring slot (d <= 2048)
 
 struct DecodeArgs {
@@ -82,6 +83,7 @@ struct DecodeArgs {
   uint32_t* bar_count;
   uint32_t* status;
   unsigned long long* trace;  // optional [grid][8] phase stamps
+  uint64_t peer_wait_ns;      // limit of a grid-barrier wait
   int nring;                  // stages of the copy ring for this call
   int region;                 // byte offset of the region after the ring
   size_t dyn_bytes;           // dynamic shared memory of the launch
@@ -113,6 +115,10 @@ struct DecShared {
   int item_ctr;                // phase C: the CTA's next item (a stage, or a stage's row pair)
   int n_ls;                    // phase C: the CTA's stage count, once known (else INT_MAX)
   int abort;
+  // bulk copies the producer issued, so that a CTA leaving early lets them land
+  int n_c_issued;              // phase-C stages (ring slot = stage % nring)
+  int n_d_issued;              // phase-D W^down stages (ring slot = expert % nring_d)
+  int h_issued;                // the h copy of phase D
 };
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
@@ -148,7 +154,7 @@ __device__ bool grid_barrier(const DecodeArgs& a, DecShared& sh, uint32_t n) {
     if (seen + 1 < target) {
       const uint64_t t0 = global_ns();
       while (ld_acquire(a.bar_count) < target) {
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > a.peer_wait_ns) {
           raise_flag(a.status, ACE_FLAG_TIMEOUT);
           sh.abort = 1;
           break;
@@ -180,6 +186,21 @@ __device__ bool await_stage(const DecodeArgs& a, DecShared& sh, int slot, int ls
     __nanosleep(64);
   }
   return true;
+}
+
+// Waits (fixed limit) until the last fill of every ring slot that received
+// one has landed: n fills went to slots f % nring, fill f completing the
+// slot's phase f / nring.
+__device__ void drain_ring(uint64_t* full, int nring, int n) {
+  for (int f = n - nring > 0 ? n - nring : 0; f < n; ++f) mbar_drain(&full[f % nring], (f / nring) & 1);
+}
+
+// Called by the producer thread before the CTA leaves: every bulk copy it
+// issued has landed, so none writes shared memory after the CTA is gone.
+__device__ void drain_copies(DecShared& sh, int nring, int nring_d) {
+  drain_ring(sh.full_c, nring, sh.n_c_issued);
+  drain_ring(sh.full_d, nring_d, sh.n_d_issued);
+  if (sh.h_issued) mbar_drain(&sh.h_bar, 0);
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& q, float (&f)[8]) {
@@ -251,6 +272,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     mbar_init(&sh.h_bar, 1);
     sh.item_ctr = 0;
     sh.n_ls = INT_MAX;
+    sh.n_c_issued = sh.n_d_issued = sh.h_issued = 0;
     for (int i = 0; i < kRing; ++i) sh.slot_gen[i] = -1;
     fence_barrier_init();
     // one round trip for every input of phase A
@@ -504,6 +526,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       }
       // the CTA's stage count: warps that drew a stage number at or past it leave
       *(volatile int*)&sh.n_ls = ls;
+      sh.n_c_issued = ls;
       if (ok && n_pre > 0) {
         // once every phase-C stage is consumed, the first W^down stages go in
         for (int st = max(0, ls - nring); st < ls && ok; ++st)
@@ -512,6 +535,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
           mbar_expect_tx(&sh.full_d[ui], dbytes);
           bulk_g2s(ring_d + (size_t)ui * dstage, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m,
                    dbytes, &sh.full_d[ui]);
+          sh.n_d_issued = ui + 1;
         }
       }
     }
@@ -558,17 +582,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         float c[4][4];  // four accumulators (blocks mod 4), so the MMA chains overlap
 #pragma unroll
         for (int j = 0; j < 4; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.f;
-        for (int b0 = 0; b0 < nblk; b0 += 4) {
+        for (int b0 = 0; b0 < nblk; b0 += 4) {  // nblk = d / 32 is a multiple of 4
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int blk = b0 + j;
-            if (blk < nblk) {
-              uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-              if (g < NT) xv = *reinterpret_cast<const uint4*>(xrow + blk * 64);
-              const uint4 wv = *reinterpret_cast<const uint4*>(wrow + blk * 64);
-              mma_bf16_m16n8k16(c[j], xv.x, xv.y, wv.x, wv.y);
-              mma_bf16_m16n8k16(c[j], xv.z, xv.w, wv.z, wv.w);
-            }
+            uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+            if (g < NT) xv = *reinterpret_cast<const uint4*>(xrow + blk * 64);
+            const uint4 wv = *reinterpret_cast<const uint4*>(wrow + blk * 64);
+            mma_bf16_m16n8k16(c[j], xv.x, xv.y, wv.x, wv.y);
+            mma_bf16_m16n8k16(c[j], xv.z, xv.w, wv.z, wv.w);
           }
         }
         __syncwarp();
@@ -639,7 +661,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   // h is read back by bulk copies (the async proxy) after the grid barrier
   asm volatile("fence.proxy.async.global;" ::: "memory");
   stamp(a, 4);
-  if (!grid_barrier(a, sh, 2)) return;
+  if (!grid_barrier(a, sh, 2)) {
+    if (producer && lane == 0) drain_copies(sh, nring, nring_d);
+    return;
+  }
   stamp(a, 5);
 
   // ---------------------------------------------------------- phase D
@@ -652,12 +677,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         asm volatile("fence.proxy.async.global;" ::: "memory");
         mbar_expect_tx(&sh.h_bar, (uint32_t)(S * m * 2));
         bulk_g2s(hs, a.h, (uint32_t)(S * m * 2), &sh.h_bar);
+        sh.h_issued = 1;
         for (int ui = n_pre; ui < U; ++ui) {
           const int slot = ui % nring_d;
           if (!wait_bar(&sh.empty_d[slot], ((ui / nring_d) & 1) ^ 1u, a, sh)) break;
           mbar_expect_tx(&sh.full_d[slot], dbytes);
           bulk_g2s(ring_d + (size_t)slot * dstage, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m,
                    dbytes, &sh.full_d[slot]);
+          sh.n_d_issued = ui + 1;
         }
       }
     } else {
@@ -725,6 +752,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     }
   }
   __syncthreads();  // both groups' sums are in
+  if (producer && lane == 0) drain_copies(sh, nring, nring_d);  // (all consumed unless aborted)
   if (warp < nrows && lane < NT)
     a.y[(size_t)lane * d + i0 + warp] =
         __float2bfloat16_rn(sh.acc_d[0][warp][lane] + sh.acc_d[1][warp][lane]);
@@ -788,7 +816,9 @@ size_t decode_smem_bytes(int T, int d, int m, int k, int E, int num_sms) {
 }
 
 bool decode_fits(int T, int d, int m, int k, int E, int num_sms) {
-  if (T < 1 || T > kDecodeMaxT || d > 2048 || d % 32 != 0 || m % 8 != 0) return false;
+  // the bf16 shape rule of every entry point (d and m multiples of 128) also
+  // keeps the staged rows and the MMA blocks of phase C whole
+  if (T < 1 || T > kDecodeMaxT || d > 2048 || d % 128 != 0 || m % 128 != 0) return false;
   const int n = ring_stages(T, d, m, k, E, num_sms);
   if (n < 2) return false;
   // phase A inside the ring: x (fp32), u (bf16), gamma, the router rows
@@ -845,6 +875,7 @@ cudaError_t launch_decode(const ace_layer& L, int fusion, const void* u, int T, 
   a.bar_count = bar;
   a.status = status;
   a.trace = trace;
+  a.peer_wait_ns = peer_wait_ns();
   a.nring = ring_stages(T, L.d, L.m, L.k, L.E, num_sms);
   a.region = a.nring * kStageBytes;
   const size_t smem = decode_smem_bytes(T, L.d, L.m, L.k, L.E, num_sms);

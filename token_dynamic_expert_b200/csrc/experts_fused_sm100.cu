@@ -16,7 +16,8 @@
 // complete.  The gate/up tail of the launch then overlaps the first down
 // items instead of idling SMs, and there is one launch instead of two.
 // Gate/up items all precede down items in every CTA's order, so no wait can
-// be on an item that has not been dealt.
+// be on an item that has not been dealt, and the launch is cooperative, so
+// every CTA that owes a tile its gate/up items is resident.
 #include <math.h>
 
 #include "ace_common.cuh"
@@ -37,13 +38,6 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;         // two accumulators of 256 columns
 constexpr int kSmemBytes = 1024 + kStageBudget + kXchgBytes + 512;
 
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (global_ns() - t0 > kWaitLimitNs) return false;
-  return true;
-}
-
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
@@ -61,6 +55,7 @@ struct FusedArgs {
   const float* slot_gate;  // [S]
   uint32_t* tile_done;     // [max_tiles] gate/up items written per tile (zeroed)
   uint32_t* status;
+  uint64_t peer_wait_ns;   // limit of a down item's wait for its tile's h rows
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -153,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t t0 = global_ns();
           bool ready = true;
           while (ld_acquire_u32(a.tile_done + ti) < (uint32_t)items0) {
-            if (*abort_flag || global_ns() - t0 > kWaitLimitNs) {
+            if (*abort_flag || global_ns() - t0 > a.peer_wait_ns) {
               if (!*abort_flag) raise_flag(a.status, ACE_FLAG_TIMEOUT);
               *abort_flag = 1;
               ready = false;
@@ -192,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*abort_flag) {  // let every copy this thread started land before exiting
         for (int s = 0; s < NS; ++s)
-          if ((issued >> s) & 1u) mbar_wait_drain(&full[s], (issued_par >> s) & 1u);
+          if ((issued >> s) & 1u) mbar_drain(&full[s], (issued_par >> s) & 1u);
       }
     }
   } else if (warp == 1) {
@@ -236,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // wait for every MMA this thread issued before TMEM is released
       mma_commit(drain);
-      mbar_wait_drain(drain, 0);
+      mbar_drain(drain, 0);
     }
   } else {
     // ----------------------------------------------------------- epilogue
@@ -386,8 +381,20 @@ cudaError_t launch_experts_fused(const ace_layer& L, int cap_slots, const void* 
   a.slot_gate = slot_gate;
   a.tile_done = tile_done;
   a.status = status;
-  k_experts_fused<<<num_sms, kThreads, kSmemBytes, s>>>(mg, mu, mx, md, mh, a);
-  return cudaGetLastError();
+  a.peer_wait_ns = peer_wait_ns();
+  // down items wait on other CTAs' gate/up items: a cooperative launch makes
+  // every CTA of the grid resident at once (one per SM)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeCooperative;
+  attrs[0].val.cooperative = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_experts_fused, mg, mu, mx, md, mh, a);
 }
 
 }  // namespace ace

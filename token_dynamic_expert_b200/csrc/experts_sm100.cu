@@ -55,13 +55,6 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;         // two accumulators of 256 columns
 constexpr int kSmemBytes = 1024 + kStageBudget + kXchgBytes + 512;
 
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (global_ns() - t0 > kWaitLimitNs) return false;
-  return true;
-}
-
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
 
 __device__ __forceinline__ void epilogue_bar() {
@@ -175,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*abort_flag) {  // let every copy this thread started land before exiting
         for (int s = 0; s < NS; ++s)
-          if ((issued >> s) & 1u) mbar_wait_drain(&full[s], (issued_par >> s) & 1u);
+          if ((issued >> s) & 1u) mbar_drain(&full[s], (issued_par >> s) & 1u);
       }
     }
   } else if (warp == 1) {
@@ -216,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // wait for every MMA this thread issued before TMEM is released
       mma_commit(drain);
-      mbar_wait_drain(drain, 0);
+      mbar_drain(drain, 0);
     }
   } else {
     // ----------------------------------------------------------- epilogue

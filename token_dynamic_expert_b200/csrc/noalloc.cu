@@ -85,26 +85,21 @@ using namespace ace;
 
 extern "C" ace_status ace_moe_decode_noalloc(const ace_layer* layer, const void* u, int T,
                                              const ace_fwd_opts* opts, void* y, void* stream) {
-  if (!layer || !opts || !u || !y) return ACE_ERR_INVALID_ARG;
+  // the same layer checks and shape rule as ace_moe_forward
+  const ace_status st = validate_layer(layer, true);
+  if (st != ACE_OK) return st;
+  if (!opts || !u || !y) return ACE_ERR_INVALID_ARG;
   const ace_layer& L = *layer;
   if (L.dtype != ACE_BF16) return ACE_ERR_UNSUPPORTED;
   if (T < 1 || T > kDecodeMaxT) return ACE_ERR_INVALID_ARG;
-  if (L.d <= 0 || L.E <= 0 || L.m <= 0 || L.k <= 0 || L.k > L.E || L.k > kMaxK)
-    return ACE_ERR_INVALID_ARG;
-  if (!L.gamma || !L.w_router || !L.w_gate || !L.w_up || !L.w_down) return ACE_ERR_INVALID_ARG;
   if (check_fusion(L, (int)opts->fusion) != ACE_OK) return ACE_ERR_INVALID_ARG;
-  const uintptr_t mis = reinterpret_cast<uintptr_t>(u) | reinterpret_cast<uintptr_t>(y) |
-                        reinterpret_cast<uintptr_t>(L.gamma) |
-                        reinterpret_cast<uintptr_t>(L.w_router) |
-                        reinterpret_cast<uintptr_t>(L.w_gate) |
-                        reinterpret_cast<uintptr_t>(L.w_up) | reinterpret_cast<uintptr_t>(L.w_down);
-  if (mis % 16 != 0) return ACE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(u) | reinterpret_cast<uintptr_t>(y)) % 16 != 0)
+    return ACE_ERR_INVALID_ARG;
   {
     const uint8_t *ub = (const uint8_t*)u, *yb = (const uint8_t*)y;
     const size_t bytes = (size_t)T * L.d * 2;
     if (ub < yb + bytes && yb < ub + bytes) return ACE_ERR_INVALID_ARG;
   }
-  if (L.E > kMaxE || L.d % 64 != 0 || L.m % 64 != 0) return ACE_ERR_UNSUPPORTED;
   const int num_sms = device_sm_count();
   if (!decode_fits(T, L.d, L.m, L.k, L.E, num_sms)) return ACE_ERR_UNSUPPORTED;
   const StaticLayout ly = static_layout(T, L.E, L.k, L.m);
@@ -129,5 +124,18 @@ extern "C" ace_status ace_moe_decode_noalloc(const ace_layer* layer, const void*
                     reinterpret_cast<uint32_t*>(w) + 16, reinterpret_cast<uint32_t*>(w), nullptr,
                     num_sms, s) != cudaSuccess)
     return ACE_ERR_CUDA;
+  return ACE_OK;
+}
+
+extern "C" ace_status ace_noalloc_read_status(uint32_t* flags, void* stream) {
+  void* base = nullptr;
+  if (scratch_address(&base) != cudaSuccess) return ACE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, base, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return ACE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ACE_ERR_CUDA;
+  if (flags) *flags = v;
+  if (v & ACE_FLAG_TIMEOUT) return ACE_ERR_TIMEOUT;
+  if (v & (ACE_FLAG_BAD_INDEX | ACE_FLAG_OVERFLOW)) return ACE_ERR_DEVICE_FAULT;
   return ACE_OK;
 }
