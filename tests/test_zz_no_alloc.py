@@ -68,10 +68,10 @@ def test_noalloc_rejects_what_it_cannot_serve():
              ctypes.c_void_p(y.data_ptr()), s) == ace.ACE_ERR_INVALID_ARG
     assert f(ctypes.byref(L), ctypes.c_void_p(u.data_ptr()), 4, ctypes.byref(opts),
              ctypes.c_void_p(u.data_ptr()), s) == ace.ACE_ERR_INVALID_ARG  # u, y overlap
-    # A layer whose scratch exceeds the fixed array: 8 tokens x top-16 x FFN 4096 bf16
-    # intermediates are 1 MiB.  Its buffers are real and of its own shape, so nothing
-    # would be read out of bounds even if the call were (wrongly) accepted.
-    big = workloads.Workload("big", T=8, d=256, E=32, m=4096, k=16, dtype="bf16", bias=False,
+    # A layer the decode kernel does not serve (hidden size above 2048).  Its
+    # buffers are real and of its own shape, so nothing would be read out of
+    # bounds even if the call were (wrongly) accepted.
+    big = workloads.Workload("big", T=8, d=4096, E=8, m=128, k=2, dtype="bf16", bias=False,
                              skip=0.5, skip_of="slots")
     lb = workloads.make_layer(big, seed=3, device="cuda")
     Lb = ace.make_layer(lb["gamma"], lb["wr"], lb["wg"], lb["wu"], lb["wd"], big.k)

@@ -109,16 +109,12 @@ struct DecShared {
   int e_base[kMaxE];           // per expert: its first slot
   float acc_d[2][kCompWarps][kDecodeMaxT];  // phase D: per group, row and token
   uint64_t in_bar;             // phase A: u, gamma and the router rows have landed
-  uint64_t h_bar;              // phase D: h of the kept slots has landed
   int slot_stage[kRing];       // phase C: the stage a ring slot holds (-1: no more)
-  int slot_gen[kRing];         // phase C: the CTA's stage number a slot was last claimed for
-  int item_ctr;                // phase C: the CTA's next item (a stage, or a stage's row pair)
-  int n_ls;                    // phase C: the CTA's stage count, once known (else INT_MAX)
   int abort;
   // bulk copies the producer issued, so that a CTA leaving early lets them land
   int n_c_issued;              // phase-C stages (ring slot = stage % nring)
+  int n_c_marked;              // phase-C end marks after them (one more phase per slot)
   int n_d_issued;              // phase-D W^down stages (ring slot = expert % nring_d)
-  int h_issued;                // the h copy of phase D
 };
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
@@ -171,23 +167,6 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const D
   return mbar_wait(bar, parity, a.status, &sh.abort);
 }
 
-// Waits until the producer has claimed ring slot `slot` for the CTA's stage
-// `ls` (true), or has published a stage count at or below ls (false); false
-// as well when the bounded wait runs out (ACE_FLAG_TIMEOUT) or the CTA aborted.
-__device__ bool await_stage(const DecodeArgs& a, DecShared& sh, int slot, int ls) {
-  const uint64_t t0 = global_ns();
-  while (*(volatile int*)&sh.slot_gen[slot] != ls) {
-    if (ls >= *(volatile int*)&sh.n_ls) return false;
-    if (*(volatile int*)&sh.abort || global_ns() - t0 > kWaitLimitNs) {
-      if (!*(volatile int*)&sh.abort) raise_flag(a.status, ACE_FLAG_TIMEOUT);
-      sh.abort = 1;
-      return false;
-    }
-    __nanosleep(64);
-  }
-  return true;
-}
-
 // Waits (fixed limit) until the last fill of every ring slot that received
 // one has landed: n fills went to slots f % nring, fill f completing the
 // slot's phase f / nring.
@@ -198,9 +177,10 @@ __device__ void drain_ring(uint64_t* full, int nring, int n) {
 // Called by the producer thread before the CTA leaves: every bulk copy it
 // issued has landed, so none writes shared memory after the CTA is gone.
 __device__ void drain_copies(DecShared& sh, int nring, int nring_d) {
-  drain_ring(sh.full_c, nring, sh.n_c_issued);
+  // phase C: stages, then end marks (no bytes; they complete on arrival) as
+  // the slots' last fills, so the waited parities are those of the last phases
+  drain_ring(sh.full_c, nring, sh.n_c_issued + sh.n_c_marked);
   drain_ring(sh.full_d, nring_d, sh.n_d_issued);
-  if (sh.h_issued) mbar_drain(&sh.h_bar, 0);
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& q, float (&f)[8]) {
@@ -262,18 +242,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     sh.abort = 0;
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sh.full_c[i], 1);
-      mbar_init(&sh.empty_c[i], NT > 2 ? 1 : kStagePairs);  // the stage's items
+      mbar_init(&sh.empty_c[i], NT > 2 ? 1 : 2);  // the slot's warps
     }
     for (int i = 0; i < kRingD; ++i) {
       mbar_init(&sh.full_d[i], 1);
       mbar_init(&sh.empty_d[i], kCompWarps / 2);
     }
     mbar_init(&sh.in_bar, 1);
-    mbar_init(&sh.h_bar, 1);
-    sh.item_ctr = 0;
-    sh.n_ls = INT_MAX;
-    sh.n_c_issued = sh.n_d_issued = sh.h_issued = 0;
-    for (int i = 0; i < kRing; ++i) sh.slot_gen[i] = -1;
+    sh.n_c_issued = sh.n_d_issued = sh.n_c_marked = 0;
     fence_barrier_init();
     // one round trip for every input of phase A
     mbar_expect_tx(&sh.in_bar, (uint32_t)(NT * d * 2 + d * 4 + n_mine * d * 2));
@@ -461,19 +437,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const int rs = row_stride(d);
   // phase-D geometry (its first stages are filled while phase C ends)
   const int nrows = i1 - i0;  // <= kCompWarps: output row i0 + w belongs to warp w
+  // a phase-D stage: the CTA's W^down rows of one surviving expert, then the
+  // h rows of that expert's kept slots (consecutive in h)
   const uint32_t dbytes = (uint32_t)(nrows * m * 2);
-  const size_t hbytes = ((size_t)S * m * 2 + 1023) & ~(size_t)1023;
-  const uint32_t dstage = (dbytes + 1023u) & ~1023u;
-  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(dsm);
-  uint8_t* ring_d = dsm + hbytes;
+  const uint32_t dstage = (uint32_t)(((size_t)dbytes + (size_t)NT * m * 2 + 1023) & ~(size_t)1023);
+  uint8_t* ring_d = dsm;
   // even: phase D's two consumer groups take alternate experts, so each slot
   // belongs to one group, which waits on the slot's fills in order
-  const int nring_d =
-      dstage ? (int)min((size_t)kRingD, (a.dyn_bytes - 1024 - hbytes) / dstage) & ~1 : 2;
+  const int nring_d = (int)min((size_t)kRingD, (a.dyn_bytes - 1024) / dstage) & ~1;
   // stages that lie inside phase C's ring (free once its last stage is
   // consumed), clear of bf16(x) that phase C still reads
-  const int n_pre = (nrows > 0 && hbytes + dstage <= (size_t)a.region)
-                        ? min(min(nring_d, U), (int)(((size_t)a.region - hbytes) / dstage))
+  const int n_pre = (nrows > 0 && dstage <= (size_t)a.region)
+                        ? min(min(nring_d, U), (int)((size_t)a.region / dstage))
                         : 0;
   if (producer) {
     if (lane == 0) {
@@ -511,7 +486,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
           claim_odd = (int)atomicAdd(stage_ctr, 1u);
         }
         sh.slot_stage[slot] = gst;
-        *(volatile int*)&sh.slot_gen[slot] = ls;
         // rows j0 .. j0 + 3 of W^gate, then of W^up, one padded row each
         const int pa = gst * kStagePairs, ui = pa / m, j0 = pa - ui * m;
         const size_t off = ((size_t)sh.uexp[ui] * m + j0) * d;
@@ -524,15 +498,26 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
                    (uint32_t)(d * 2), &sh.full_c[slot]);
         }
       }
-      // the CTA's stage count: warps that drew a stage number at or past it leave
-      *(volatile int*)&sh.n_ls = ls;
       sh.n_c_issued = ls;
+      // End marks: the next fill of every slot carries stage -1 and no bytes
+      // (a plain arrival completes its phase), so each slot's warps learn that
+      // there is no more.  A slot is marked once its last stage is consumed
+      // (slot ls % nring was waited for above); after the marks every
+      // phase-C stage is consumed.
+      for (int j = 0; j < nring && ok; ++j) {
+        const int lsj = ls + j, slot = lsj % nring;
+        if (j > 0 && !(ok = wait_bar(&sh.empty_c[slot], ((lsj / nring) & 1) ^ 1u, a, sh))) break;
+        sh.slot_stage[slot] = -1;
+        mbar_arrive(&sh.full_c[slot]);
+        sh.n_c_marked = j + 1;
+      }
       if (ok && n_pre > 0) {
-        // once every phase-C stage is consumed, the first W^down stages go in
-        for (int st = max(0, ls - nring); st < ls && ok; ++st)
-          ok = wait_bar(&sh.empty_c[st % nring], (st / nring) & 1, a, sh);
+        // the first W^down stages go into the drained ring
         for (int ui = 0; ui < n_pre && ok; ++ui) {
-          mbar_expect_tx(&sh.full_d[ui], dbytes);
+          // the stage's h rows follow after the second grid barrier, on the
+          // same phase of the barrier
+          const uint32_t hb = (uint32_t)((sh.ufirst[ui + 1] - sh.ufirst[ui]) * m * 2);
+          mbar_expect_tx(&sh.full_d[ui], dbytes + hb);
           bulk_g2s(ring_d + (size_t)ui * dstage, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m,
                    dbytes, &sh.full_d[ui]);
           sh.n_d_issued = ui + 1;
@@ -540,120 +525,123 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       }
     }
   } else {
-    // Items are drawn in order from a CTA counter by whichever warp is free.
-    // A warp may draw an item of a stage up to a ring lap ahead, so it first
-    // waits until the producer has claimed the slot for that stage
-    // (slot_gen) or has published the CTA's stage count (n_ls), then for the
-    // data.  Two forms of item, by token count:
-    //  * NT >= 3: a whole stage.  The warp forms on the tensor cores
-    //    (m16n8k16, bf16 operands, fp32 accumulation) the dots of the call's
-    //    tokens (MMA rows; rows NT .. 15 are zero) with the stage's 8 rows
-    //    (MMA columns: 4 gate, 4 up) over the whole hidden size.  In each
-    //    32-wide block of the hidden size, lane (g, q) holds the elements
-    //    8q .. 8q + 7 of token g's bf16(x) and of staged row g; the block's
-    //    two MMAs take elements 8q + {0..3} and 8q + {4..7} as the k of their
-    //    fragments, the same permutation of the block's 32 k on both
-    //    operands, so each MMA sums exact products of matching elements.
-    //    One warp per stage keeps several stages in work at once, so the
-    //    ring turns over at the rate the weights arrive.
-    //  * NT <= 2: one (gate, up) row pair of a stage, dotted on the CUDA
-    //    cores with each kept token of the pair's expert; the four pairs of
-    //    a stage go to four warps, which finishes a stage sooner when a CTA
-    //    has only a few.
+    // Each ring slot has fixed consumer warps, which take its fills in order
+    // (fill f of slot s is the CTA's stage f * nring + s) until an end mark:
+    // a warp only ever waits for the next phase of its own slot, so no wait
+    // can see an older phase, and waiting warps sleep in the barrier instead
+    // of polling.  Two forms, by token count:
+    //  * NT >= 3: one warp per slot forms, on the tensor cores (m16n8k16,
+    //    bf16 operands, fp32 accumulation), the dots of the call's tokens
+    //    (MMA rows; rows NT .. 15 are zero) with the stage's 8 rows (MMA
+    //    columns: 4 gate, 4 up) over the whole hidden size.  In each 32-wide
+    //    block of the hidden size, lane (g, q) holds the elements 8q .. 8q + 7
+    //    of token g's bf16(x) and of staged row g; the block's two MMAs take
+    //    elements 8q + {0..3} and 8q + {4..7} as the k of their fragments,
+    //    the same permutation of the block's 32 k on both operands, so each
+    //    MMA sums exact products of matching elements.
+    //  * NT <= 2: two warps per slot, each dotting two (gate, up) row pairs
+    //    of the stage on the CUDA cores with each kept token of the pair's
+    //    expert.
     // Either way the warp writes h = SiLU(gate) * up for the tokens that
     // kept the stage's expert.
-    constexpr int kItems = NT > 2 ? 1 : kStagePairs;  // items per stage
+    constexpr int kWPS = NT > 2 ? 1 : 2;  // warps per slot
     const int g = lane >> 2, q = lane & 3;
     const int nblk = d / 32;
     const uint8_t* xrow = reinterpret_cast<const uint8_t*>(xb) + (size_t)g * rs + 16 * q;
-    for (;;) {
-      int it = 0;
-      if (lane == 0) it = atomicAdd(&sh.item_ctr, 1);
-      it = __shfl_sync(0xffffffffu, it, 0);
-      const int ls = it / kItems, r = it - ls * kItems;
-      const int slot = ls % nring;
-      if (!await_stage(a, sh, slot, ls)) break;
-      if (!wait_bar(&sh.full_c[slot], (ls / nring) & 1, a, sh)) break;
-      const int gst = sh.slot_stage[slot];
-      const uint8_t* stage = ring + (size_t)slot * kStageBytes;
-      if constexpr (NT > 2) {
-        (void)r;
-        const uint8_t* wrow = stage + (size_t)g * rs + 16 * q;
-        float c[4][4];  // four accumulators (blocks mod 4), so the MMA chains overlap
+    const int slot = warp / kWPS, half = warp % kWPS;
+    if (slot < nring) {
+      for (int f = 0;; ++f) {
+        // lane 0 waits (bounded); once the phase is complete every lane takes
+        // its acquire with one test (the phase stays complete until this
+        // warp releases the slot)
+        int ok = 1;
+        if (lane == 0) ok = wait_bar(&sh.full_c[slot], f & 1, a, sh);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        mbar_try_wait(&sh.full_c[slot], f & 1);
+        const int gst = sh.slot_stage[slot];
+        if (gst < 0) break;  // end mark
+        const uint8_t* stage = ring + (size_t)slot * kStageBytes;
+        if constexpr (NT > 2) {
+          const uint8_t* wrow = stage + (size_t)g * rs + 16 * q;
+          float c[4][4];  // four accumulators (blocks mod 4), so the MMA chains overlap
 #pragma unroll
-        for (int j = 0; j < 4; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.f;
-        for (int b0 = 0; b0 < nblk; b0 += 4) {  // nblk = d / 32 is a multiple of 4
+          for (int j = 0; j < 4; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.f;
+          for (int b0 = 0; b0 < nblk; b0 += 4) {  // nblk = d / 32 is a multiple of 4
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int blk = b0 + j;
-            uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-            if (g < NT) xv = *reinterpret_cast<const uint4*>(xrow + blk * 64);
-            const uint4 wv = *reinterpret_cast<const uint4*>(wrow + blk * 64);
-            mma_bf16_m16n8k16(c[j], xv.x, xv.y, wv.x, wv.y);
-            mma_bf16_m16n8k16(c[j], xv.z, xv.w, wv.z, wv.w);
+            for (int j = 0; j < 4; ++j) {
+              const int blk = b0 + j;
+              uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+              if (g < NT) xv = *reinterpret_cast<const uint4*>(xrow + blk * 64);
+              const uint4 wv = *reinterpret_cast<const uint4*>(wrow + blk * 64);
+              mma_bf16_m16n8k16(c[j], xv.x, xv.y, wv.x, wv.y);
+              mma_bf16_m16n8k16(c[j], xv.z, xv.w, wv.z, wv.w);
+            }
           }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty_c[slot]);  // the warp's reads of the slot are done
-        // token g with staged rows 2q, 2q + 1: gate rows of pairs 2q, 2q + 1
-        // on lanes q = 0, 1; the matching up rows (4 + 2q, 5 + 2q) two lanes up
-        const float d0 = (c[0][0] + c[1][0]) + (c[2][0] + c[3][0]);
-        const float d1 = (c[0][1] + c[1][1]) + (c[2][1] + c[3][1]);
-        const float u0 = __shfl_down_sync(0xffffffffu, d0, 2);
-        const float u1 = __shfl_down_sync(0xffffffffu, d1, 2);
-        if (q < 2 && g < NT) {
-          const int pa = gst * kStagePairs, ui = pa / m, j0 = pa - ui * m;
-          const uint32_t mk = sh.tok_mask[sh.uexp[ui]];
-          if ((mk >> g) & 1u) {
-            const int si = sh.ufirst[ui] + __popc(mk & ((1u << g) - 1u));
-            __nv_bfloat16* hp = a.h + (size_t)si * m + j0 + 2 * q;
-            hp[0] = __float2bfloat16_rn(silu(d0) * u0);
-            hp[1] = __float2bfloat16_rn(silu(d1) * u1);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.empty_c[slot]);  // the warp's reads of the slot are done
+          // token g with staged rows 2q, 2q + 1: gate rows of pairs 2q, 2q + 1
+          // on lanes q = 0, 1; the matching up rows (4 + 2q, 5 + 2q) two lanes up
+          const float d0 = (c[0][0] + c[1][0]) + (c[2][0] + c[3][0]);
+          const float d1 = (c[0][1] + c[1][1]) + (c[2][1] + c[3][1]);
+          const float u0 = __shfl_down_sync(0xffffffffu, d0, 2);
+          const float u1 = __shfl_down_sync(0xffffffffu, d1, 2);
+          if (q < 2 && g < NT) {
+            const int pa = gst * kStagePairs, ui = pa / m, j0 = pa - ui * m;
+            const uint32_t mk = sh.tok_mask[sh.uexp[ui]];
+            if ((mk >> g) & 1u) {
+              const int si = sh.ufirst[ui] + __popc(mk & ((1u << g) - 1u));
+              __nv_bfloat16* hp = a.h + (size_t)si * m + j0 + 2 * q;
+              hp[0] = __float2bfloat16_rn(silu(d0) * u0);
+              hp[1] = __float2bfloat16_rn(silu(d1) * u1);
+            }
           }
-        }
-      } else {
-        const int p = gst * kStagePairs + r;
-        const int ui = p / m, j = p - ui * m;
-        const int s0 = sh.ufirst[ui], nt = sh.ufirst[ui + 1] - s0;  // <= NT
-        const uint4* wg = reinterpret_cast<const uint4*>(stage + (size_t)r * rs);
-        const uint4* wu = reinterpret_cast<const uint4*>(stage + (size_t)(r + kStagePairs) * rs);
-        const uint4* xq = reinterpret_cast<const uint4*>(xb);
-        int xo[NT];  // each kept token's row of bf16(x), in 16-byte chunks
+        } else {
+          for (int rr = 0; rr < kStagePairs / kWPS; ++rr) {
+            const int r = half * (kStagePairs / kWPS) + rr;
+            const int p = gst * kStagePairs + r;
+            const int ui = p / m, j = p - ui * m;
+            const int s0 = sh.ufirst[ui], nt = sh.ufirst[ui + 1] - s0;  // <= NT
+            const uint4* wg = reinterpret_cast<const uint4*>(stage + (size_t)r * rs);
+            const uint4* wu = reinterpret_cast<const uint4*>(stage + (size_t)(r + kStagePairs) * rs);
+            const uint4* xq = reinterpret_cast<const uint4*>(xb);
+            int xo[NT];  // each kept token's row of bf16(x), in 16-byte chunks
 #pragma unroll
-        for (int t = 0; t < NT; ++t) xo[t] = (t < nt ? sh.slot_t[s0 + t] : 0) * (rs / 16);
-        float ga[NT], ua[NT];
+            for (int t = 0; t < NT; ++t) xo[t] = (t < nt ? sh.slot_t[s0 + t] : 0) * (rs / 16);
+            float ga[NT], ua[NT];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) ga[t] = ua[t] = 0.f;
-        for (int cc = lane; cc < d / 8; cc += 32) {
-          float w1[8], w2[8];
-          bf16x8_to_f32(wg[cc], w1);
-          bf16x8_to_f32(wu[cc], w2);
+            for (int t = 0; t < NT; ++t) ga[t] = ua[t] = 0.f;
+            for (int cc = lane; cc < d / 8; cc += 32) {
+              float w1[8], w2[8];
+              bf16x8_to_f32(wg[cc], w1);
+              bf16x8_to_f32(wu[cc], w2);
 #pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            if (t < nt) {
-              float xv[8];
-              bf16x8_to_f32(xq[xo[t] + cc], xv);
+              for (int t = 0; t < NT; ++t) {
+                if (t < nt) {
+                  float xv[8];
+                  bf16x8_to_f32(xq[xo[t] + cc], xv);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                ga[t] = fmaf(w1[e], xv[e], ga[t]);
-                ua[t] = fmaf(w2[e], xv[e], ua[t]);
+                  for (int e = 0; e < 8; ++e) {
+                    ga[t] = fmaf(w1[e], xv[e], ga[t]);
+                    ua[t] = fmaf(w2[e], xv[e], ua[t]);
+                  }
+                }
+              }
+            }
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+              if (t < nt) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                  ga[t] += __shfl_xor_sync(0xffffffffu, ga[t], o);
+                  ua[t] += __shfl_xor_sync(0xffffffffu, ua[t], o);
+                }
+                if (lane == t) a.h[(size_t)(s0 + t) * m + j] = __float2bfloat16_rn(silu(ga[t]) * ua[t]);
               }
             }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.empty_c[slot]);
         }
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          if (t < nt) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              ga[t] += __shfl_xor_sync(0xffffffffu, ga[t], o);
-              ua[t] += __shfl_xor_sync(0xffffffffu, ua[t], o);
-            }
-            if (lane == t) a.h[(size_t)(s0 + t) * m + j] = __float2bfloat16_rn(silu(ga[t]) * ua[t]);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty_c[slot]);
       }
     }
   }
@@ -662,28 +650,43 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   asm volatile("fence.proxy.async.global;" ::: "memory");
   stamp(a, 4);
   if (!grid_barrier(a, sh, 2)) {
-    if (producer && lane == 0) drain_copies(sh, nring, nring_d);
+    if (producer && lane == 0) {
+      // the pre-issued stages expect their h rows too: copy them (whatever h
+      // holds) so that their phases complete, then let everything land
+      for (int ui = 0; ui < sh.n_d_issued; ++ui) {
+        const int s0 = sh.ufirst[ui];
+        bulk_g2s(ring_d + (size_t)ui * dstage + dbytes, a.h + (size_t)s0 * m,
+                 (uint32_t)((sh.ufirst[ui + 1] - s0) * m * 2), &sh.full_d[ui]);
+      }
+      drain_copies(sh, nring, nring_d);
+    }
     return;
   }
   stamp(a, 5);
 
   // ---------------------------------------------------------- phase D
-  // shared memory: h of the kept slots (one bulk copy), then a ring of
-  // stages that each hold the CTA's output rows of one surviving expert's
-  // W^down; the first n_pre stages were issued at the end of phase C
+  // a ring of stages that each hold the CTA's output rows of one surviving
+  // expert's W^down and the h rows of its kept slots; the W^down rows of the
+  // first n_pre stages were issued at the end of phase C
   if (nrows > 0) {
     if (producer) {
       if (lane == 0) {
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        mbar_expect_tx(&sh.h_bar, (uint32_t)(S * m * 2));
-        bulk_g2s(hs, a.h, (uint32_t)(S * m * 2), &sh.h_bar);
-        sh.h_issued = 1;
-        for (int ui = n_pre; ui < U; ++ui) {
+        asm volatile("fence.proxy.async.global;" ::: "memory");  // h is read by bulk copies
+        for (int ui = 0; ui < sh.n_d_issued; ++ui) {
+          const int s0 = sh.ufirst[ui];
+          const uint32_t hb = (uint32_t)((sh.ufirst[ui + 1] - s0) * m * 2);
+          bulk_g2s(ring_d + (size_t)ui * dstage + dbytes, a.h + (size_t)s0 * m, hb,
+                   &sh.full_d[ui]);
+        }
+        for (int ui = sh.n_d_issued; ui < U; ++ui) {
           const int slot = ui % nring_d;
           if (!wait_bar(&sh.empty_d[slot], ((ui / nring_d) & 1) ^ 1u, a, sh)) break;
-          mbar_expect_tx(&sh.full_d[slot], dbytes);
-          bulk_g2s(ring_d + (size_t)slot * dstage, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m,
-                   dbytes, &sh.full_d[slot]);
+          const int s0 = sh.ufirst[ui];
+          const uint32_t hb = (uint32_t)((sh.ufirst[ui + 1] - s0) * m * 2);
+          uint8_t* st = ring_d + (size_t)slot * dstage;
+          mbar_expect_tx(&sh.full_d[slot], dbytes + hb);
+          bulk_g2s(st, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m, dbytes, &sh.full_d[slot]);
+          bulk_g2s(st + dbytes, a.h + (size_t)s0 * m, hb, &sh.full_d[slot]);
           sh.n_d_issued = ui + 1;
         }
       }
@@ -698,7 +701,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         sh.acc_d[grp][wl + 8][lane] = 0.f;
       }
       __syncwarp();
-      bool ok = wait_bar(&sh.h_bar, 0, a, sh);
+      bool ok = true;
       for (int ui = grp; ok && ui < U; ui += 2) {
         const int slot = ui % nring_d;
         if (!(ok = wait_bar(&sh.full_d[slot], (ui / nring_d) & 1, a, sh))) break;
@@ -707,6 +710,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         // and the two rows' loads and reductions overlap
         if (wl < nrows) {
           const bool two = wl + 8 < nrows;
+          const __nv_bfloat16* hs =  // the stage's h rows: slot s0 + i at row i
+              reinterpret_cast<const __nv_bfloat16*>(ring_d + (size_t)slot * dstage + dbytes);
           const uint4* w0 =
               reinterpret_cast<const uint4*>(ring_d + (size_t)slot * dstage + (size_t)wl * m * 2);
           const uint4* w1 = w0 + (two ? 8 * m / 8 : 0);
@@ -721,7 +726,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
               for (int q = 0; q < 4; ++q) {
                 if (q >= nt) break;
                 float hv[8];
-                bf16x8_to_f32(reinterpret_cast<const uint4*>(hs + (size_t)(sg + q) * m)[c], hv);
+                bf16x8_to_f32(reinterpret_cast<const uint4*>(hs + (size_t)(sg + q - s0) * m)[c], hv);
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) {
                   d0[q] = fmaf(a8[cc], hv[cc], d0[q]);
@@ -827,10 +832,9 @@ bool decode_fits(int T, int d, int m, int k, int E, int num_sms) {
   if (staged > (size_t)n * kStageBytes) return false;
   const int rows = (d + num_sms - 1) / num_sms;                    // phase-D rows per CTA
   if (rows > kCompWarps) return false;
-  // phase D: h of every kept slot plus at least two stages of W^down rows
-  const size_t hbytes = ((size_t)T * k * m * 2 + 1023) & ~(size_t)1023;
-  const size_t dstage = ((size_t)rows * m * 2 + 1023) & ~(size_t)1023;
-  return decode_smem_bytes(T, d, m, k, E, num_sms) >= 1024 + hbytes + 2 * dstage;
+  // phase D: at least two stages of W^down rows and an expert's h rows
+  const size_t dstage = ((size_t)rows * m * 2 + (size_t)T * m * 2 + 1023) & ~(size_t)1023;
+  return decode_smem_bytes(T, d, m, k, E, num_sms) >= 1024 + 2 * dstage;
 }
 
 cudaError_t launch_decode(const ace_layer& L, int fusion, const void* u, int T, float tau,
