@@ -12,20 +12,20 @@
 //            mask ([ACE] "3. Conservative Fusion", top-1 always kept), the
 //            kept slots sorted by (expert, token), the distinct experts
 //   phase C  gate/up ([ACE] eq. f): the surviving (expert, row) pairs, in
-//            stages of 4 row pairs (a fixed first lap per CTA, then stages
-//            the CTAs take from a grid-wide counter as their rings free up),
-//            stream through a shared-memory
-//            ring by TMA bulk copies issued from a producer warp; free
-//            compute warps take a whole stage (3+ tokens: tensor-core dots
-//            of every token with its 8 rows) or one row pair of it (1-2
-//            tokens: CUDA-core dots) and write h = SiLU(x W^gate) (.) x W^up
-//            for the tokens that kept the expert; once the ring drains, the
-//            first W^down stages of phase D are issued
+//            stages of 4 row pairs dealt round robin to the CTAs, stream
+//            through a shared-memory ring by bulk copies issued from a
+//            producer warp; each ring slot has 2-3 fixed compute warps that
+//            split the hidden size and form, on the tensor cores, the dots of
+//            every token with the stage's 8 rows, then write
+//            h = SiLU(x W^gate) (.) x W^up for the tokens that kept the
+//            expert; once the ring drains, the first W^down stages of phase D
+//            are issued
 //   -- grid barrier --
 //   phase D  down + combine: the CTA's output rows of every surviving
-//            expert's W^down stream through the ring; warp w owns output row
-//            w and sums g * (h W^down) over the token's kept slots, experts
-//            in ascending order
+//            expert's W^down, with the h rows of the expert's kept slots,
+//            stream through the ring; each slot's warps form h W^down on the
+//            tensor cores and add g * (h W^down) into per-warp sums, which
+//            are added in warp order at the end
 // The grid barrier is a generation counter in the workspace with a bounded
 // spin; the launch is cooperative so every CTA is resident.  Every mbarrier
 // wait is bounded as well.  Numerics follow the prefill path: fp32 router on
@@ -55,6 +55,13 @@ constexpr int kMaxSlots = kDecodeMaxT * kMaxK;
 // 16-byte pieces of each) then hit distinct banks.
 __host__ __device__ constexpr int row_stride(int d) { return 2 * d + 64; }
 constexpr int kStageBytes = kStageRows * row_stride(2048);  // bytes per ring slot (d <= 2048)
+// Phase C splits the hidden size of a stage over at most kPartsC warps; the
+// partial dots of parts 1 .. kPartsC - 1 meet part 0 in shared memory, two
+// buffers per slot (by fill parity)
+constexpr int kPartsC = 3;
+constexpr int kPartBytes = kRing * 2 * (kPartsC - 1) * 32 * 8;
+// Phase D splits the expert size of a stage over at most kPartsD warps
+constexpr int kPartsD = 4;
 
 struct DecodeArgs {
   const float* gamma;
@@ -86,6 +93,7 @@ struct DecodeArgs {
   uint64_t peer_wait_ns;      // limit of a grid-barrier wait
   int nring;                  // stages of the copy ring for this call
   int region;                 // byte offset of the region after the ring
+  int part_off;               // byte offset of phase C's partial dots
   size_t dyn_bytes;           // dynamic shared memory of the launch
 };
 
@@ -107,7 +115,6 @@ struct DecShared {
   uint32_t tok_mask[kMaxE];    // per expert: bit t set when token t kept a slot of it
   float fac[kMaxE];            // per expert: the fused table factor F(A^GSP, A^RCR)
   int e_base[kMaxE];           // per expert: its first slot
-  float acc_d[2][kCompWarps][kDecodeMaxT];  // phase D: per group, row and token
   uint64_t in_bar;             // phase A: u, gamma and the router rows have landed
   int slot_stage[kRing];       // phase C: the stage a ring slot holds (-1: no more)
   int abort;
@@ -215,6 +222,43 @@ __device__ __forceinline__ void mma_bf16_m16n8k16(float (&c)[4], uint32_t a0, ui
 
 
 
+// c += A * B for one m16n8k16 tile, bf16 operands, fp32 accumulators, all
+// sixteen rows of A
+__device__ __forceinline__ void mma_bf16_m16n8k16_full(float (&c)[4], uint32_t a0, uint32_t a1,
+                                                       uint32_t a2, uint32_t a3, uint32_t b0,
+                                                       uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Named barrier `id` over `count` threads that also ANDs `v` over them: every
+// participant gets the same answer, so a group of warps can leave a loop
+// together.
+__device__ __forceinline__ bool bar_red_and(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+// Phase-D geometry of a CTA with `rows` output rows (the same on the host,
+// which sizes shared memory, and in the kernel): a stage holds the rows of
+// one expert's W^down and the h rows of its kept slots (at most T)
+__host__ __device__ inline size_t dstage_bytes(int rows, int T, int m) {
+  return ((size_t)rows * m * 2 + (size_t)T * m * 2 + 1023) & ~(size_t)1023;
+}
+// per-warp sums of phase D: [warp][16 rows][T tokens] fp32
+__host__ __device__ constexpr size_t dacc_bytes(int T) { return (size_t)kCompWarps * 16 * T * 4; }
+
 // NT = the call's token count.
 template <int NT>
 __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
@@ -238,15 +282,28 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const int n_router_warps = (E + G - 1) / G;
   // router rows of this CTA: experts blockIdx.x + G * r, r < n_mine
   const int n_mine = (int)blockIdx.x < E ? min(n_router_warps, (E - 1 - (int)blockIdx.x) / G + 1) : 0;
+  // phase C: each ring slot has wps_c consumer warps, which split the hidden
+  // size of the slot's stages
+  const int wps_c = min(kPartsC, kCompWarps / nring);
+  // phase D: the CTA's output rows i0 .. i1 - 1 (warp w of a slot's MMA
+  // covers all of them, <= 16); each ring slot has wps_d consumer warps,
+  // which split the expert size
+  const int rows_per_cta = (d + G - 1) / G;
+  const int i0 = min(d, (int)blockIdx.x * rows_per_cta), i1 = min(d, i0 + rows_per_cta);
+  const int nrows = i1 - i0;
+  const uint32_t dbytes = (uint32_t)(nrows * m * 2);
+  const size_t dstage = dstage_bytes(nrows, NT, m);
+  const int nring_d = (int)min((size_t)kRingD, (a.dyn_bytes - 1024 - dacc_bytes(NT)) / dstage);
+  const int wps_d = min(min(kPartsD, kCompWarps / nring_d), m / 32);
   if (threadIdx.x == 0) {
     sh.abort = 0;
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sh.full_c[i], 1);
-      mbar_init(&sh.empty_c[i], NT > 2 ? 1 : 2);  // the slot's warps
+      mbar_init(&sh.empty_c[i], wps_c);  // the slot's warps
     }
     for (int i = 0; i < kRingD; ++i) {
       mbar_init(&sh.full_d[i], 1);
-      mbar_init(&sh.empty_d[i], kCompWarps / 2);
+      mbar_init(&sh.empty_d[i], wps_d);
     }
     mbar_init(&sh.in_bar, 1);
     sh.n_c_issued = sh.n_d_issued = sh.n_c_marked = 0;
@@ -430,61 +487,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const int S = sh.n_slots, U = sh.n_uexp;
 
   // ---------------------------------------------------------- phase C
-  const int rows_per_cta = (d + G - 1) / G;  // phase-D output rows per CTA (<= 16)
-  const int i0 = min(d, (int)blockIdx.x * rows_per_cta), i1 = min(d, i0 + rows_per_cta);
   const int P = U * m;  // surviving (expert, row) pairs
   const int n_stages = P / kStagePairs;  // m % 8 == 0: a stage never spans two experts
   const int rs = row_stride(d);
-  // phase-D geometry (its first stages are filled while phase C ends)
-  const int nrows = i1 - i0;  // <= kCompWarps: output row i0 + w belongs to warp w
-  // a phase-D stage: the CTA's W^down rows of one surviving expert, then the
-  // h rows of that expert's kept slots (consecutive in h)
-  const uint32_t dbytes = (uint32_t)(nrows * m * 2);
-  const uint32_t dstage = (uint32_t)(((size_t)dbytes + (size_t)NT * m * 2 + 1023) & ~(size_t)1023);
+  // phase D's stages (its first ones are filled while phase C ends): the
+  // CTA's W^down rows of one surviving expert, then the h rows of that
+  // expert's kept slots (consecutive in h); the per-warp sums follow the ring
   uint8_t* ring_d = dsm;
-  // even: phase D's two consumer groups take alternate experts, so each slot
-  // belongs to one group, which waits on the slot's fills in order
-  const int nring_d = (int)min((size_t)kRingD, (a.dyn_bytes - 1024) / dstage) & ~1;
   // stages that lie inside phase C's ring (free once its last stage is
-  // consumed), clear of bf16(x) that phase C still reads
+  // consumed), clear of bf16(x) and the partial dots that phase C still reads
   const int n_pre = (nrows > 0 && dstage <= (size_t)a.region)
                         ? min(min(nring_d, U), (int)((size_t)a.region / dstage))
                         : 0;
   if (producer) {
     if (lane == 0) {
-      // The ring's first lap takes the fixed stages blockIdx.x + G * ls, so
-      // it is issued at once.  Later stages come from a grid-wide counter as
-      // the ring frees up (CTAs that run ahead take more of them), numbered
-      // from G * nring on; each is claimed two stages before it is issued, so
-      // the atomic's round trip overlaps the wait for a free slot.  The two
-      // pending claims alternate (even and odd stages after the first lap)
-      // and a CTA's claims increase in the order it makes them: when the
-      // claim in use is past the last stage, so is the one still pending.
-      uint32_t* stage_ctr = a.bar_count + 1;
-      const int dyn0 = G * nring;
-      int claim_even = 0, claim_odd = 0;
+      // The CTA's stages are blockIdx.x + G * ls, ls = 0, 1, ...: a fixed
+      // round robin (the CTAs' counts differ by one at most), so the issue
+      // loop never waits on anything but a free slot.  (A grid-wide counter
+      // that hands out stages costs an atomic round trip per stage, which
+      // under full DRAM load is longer than a stage's streaming time.)
       int ls = 0;  // this CTA's stages so far
       bool ok = true;
       for (;; ++ls) {
+        const int gst = (int)blockIdx.x + G * ls;
+        if (gst >= n_stages) break;
         const int slot = ls % nring;
         if (!(ok = wait_bar(&sh.empty_c[slot], ((ls / nring) & 1) ^ 1u, a, sh))) break;
-        int gst;
-        if (ls < nring) {
-          gst = (int)blockIdx.x + G * ls;
-          if (gst >= n_stages) break;
-          if (ls == nring - 1) {
-            claim_even = (int)atomicAdd(stage_ctr, 1u);
-            claim_odd = (int)atomicAdd(stage_ctr, 1u);
-          }
-        } else if (((ls - nring) & 1) == 0) {
-          gst = dyn0 + claim_even;
-          if (gst >= n_stages) break;
-          claim_even = (int)atomicAdd(stage_ctr, 1u);
-        } else {
-          gst = dyn0 + claim_odd;
-          if (gst >= n_stages) break;
-          claim_odd = (int)atomicAdd(stage_ctr, 1u);
-        }
         sh.slot_stage[slot] = gst;
         // rows j0 .. j0 + 3 of W^gate, then of W^up, one padded row each
         const int pa = gst * kStagePairs, ui = pa / m, j0 = pa - ui * m;
@@ -501,12 +529,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       sh.n_c_issued = ls;
       // End marks: the next fill of every slot carries stage -1 and no bytes
       // (a plain arrival completes its phase), so each slot's warps learn that
-      // there is no more.  A slot is marked once its last stage is consumed
-      // (slot ls % nring was waited for above); after the marks every
-      // phase-C stage is consumed.
+      // there is no more.  A slot is marked once its last stage is consumed;
+      // after the marks every phase-C stage is consumed.
       for (int j = 0; j < nring && ok; ++j) {
         const int lsj = ls + j, slot = lsj % nring;
-        if (j > 0 && !(ok = wait_bar(&sh.empty_c[slot], ((lsj / nring) & 1) ^ 1u, a, sh))) break;
+        if (!(ok = wait_bar(&sh.empty_c[slot], ((lsj / nring) & 1) ^ 1u, a, sh))) break;
         sh.slot_stage[slot] = -1;
         mbar_arrive(&sh.full_c[slot]);
         sh.n_c_marked = j + 1;
@@ -525,64 +552,85 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       }
     }
   } else {
-    // Each ring slot has fixed consumer warps, which take its fills in order
-    // (fill f of slot s is the CTA's stage f * nring + s) until an end mark:
-    // a warp only ever waits for the next phase of its own slot, so no wait
-    // can see an older phase, and waiting warps sleep in the barrier instead
-    // of polling.  Two forms, by token count:
-    //  * NT >= 3: one warp per slot forms, on the tensor cores (m16n8k16,
-    //    bf16 operands, fp32 accumulation), the dots of the call's tokens
-    //    (MMA rows; rows NT .. 15 are zero) with the stage's 8 rows (MMA
-    //    columns: 4 gate, 4 up) over the whole hidden size.  In each 32-wide
-    //    block of the hidden size, lane (g, q) holds the elements 8q .. 8q + 7
-    //    of token g's bf16(x) and of staged row g; the block's two MMAs take
-    //    elements 8q + {0..3} and 8q + {4..7} as the k of their fragments,
-    //    the same permutation of the block's 32 k on both operands, so each
-    //    MMA sums exact products of matching elements.
-    //  * NT <= 2: two warps per slot, each dotting two (gate, up) row pairs
-    //    of the stage on the CUDA cores with each kept token of the pair's
-    //    expert.
-    // Either way the warp writes h = SiLU(gate) * up for the tokens that
-    // kept the stage's expert.
-    constexpr int kWPS = NT > 2 ? 1 : 2;  // warps per slot
+    // Each ring slot has wps_c fixed consumer warps (parts), which take its
+    // fills in order (fill f of slot s is the CTA's stage f * nring + s) until
+    // an end mark: a warp only ever waits for the next phase of its own slot,
+    // so no wait can see an older phase, and waiting warps sleep in the
+    // barrier instead of polling.  Part p forms, on the tensor cores
+    // (m16n8k16, bf16 operands, fp32 accumulation), the dots of the call's
+    // tokens (MMA rows; rows NT .. 15 are zero) with the stage's 8 rows (MMA
+    // columns: 4 gate, 4 up) over its share of the hidden size, 32-wide
+    // blocks b0 .. b1 - 1.  In each block, lane (g, q) holds the elements
+    // 8q .. 8q + 7 of token g's bf16(x) and of staged row g; the block's two
+    // MMAs take elements 8q + {0..3} and 8q + {4..7} as the k of their
+    // fragments, the same permutation of the block's 32 k on both operands,
+    // so each MMA sums exact products of matching elements.  Parts 1, 2 leave
+    // their dots in shared memory; after a named barrier over the slot's
+    // warps (which also tells every part whether to go on), part 0 adds them
+    // in part order and writes h = SiLU(gate) * up for the tokens that kept
+    // the stage's expert.
+    const int slot = warp / wps_c, part = warp % wps_c;
     const int g = lane >> 2, q = lane & 3;
     const int nblk = d / 32;
+    const int b0 = part * nblk / wps_c, b1 = (part + 1) * nblk / wps_c;
     const uint8_t* xrow = reinterpret_cast<const uint8_t*>(xb) + (size_t)g * rs + 16 * q;
-    const int slot = warp / kWPS, half = warp % kWPS;
+    float2* partial = reinterpret_cast<float2*>(dsm + a.part_off);  // [kRing][2][kPartsC - 1][32]
     if (slot < nring) {
       for (int f = 0;; ++f) {
         // lane 0 waits (bounded); once the phase is complete every lane takes
-        // its acquire with one test (the phase stays complete until this
-        // warp releases the slot)
+        // its acquire with one test (the phase stays complete until all of
+        // the slot's warps release it)
         int ok = 1;
         if (lane == 0) ok = wait_bar(&sh.full_c[slot], f & 1, a, sh);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        mbar_try_wait(&sh.full_c[slot], f & 1);
-        const int gst = sh.slot_stage[slot];
-        if (gst < 0) break;  // end mark
-        const uint8_t* stage = ring + (size_t)slot * kStageBytes;
-        if constexpr (NT > 2) {
-          const uint8_t* wrow = stage + (size_t)g * rs + 16 * q;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        int gst = -1;
+        if (ok) {
+          mbar_try_wait(&sh.full_c[slot], f & 1);
+          gst = sh.slot_stage[slot];
+        }
+        const bool go = ok && gst >= 0;  // (gst < 0: end mark)
+        float d0 = 0.f, d1 = 0.f;
+        if (go) {
+          const uint8_t* wrow = ring + (size_t)slot * kStageBytes + (size_t)g * rs + 16 * q;
           float c[4][4];  // four accumulators (blocks mod 4), so the MMA chains overlap
 #pragma unroll
           for (int j = 0; j < 4; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.f;
-          for (int b0 = 0; b0 < nblk; b0 += 4) {  // nblk = d / 32 is a multiple of 4
+          int blk = b0;
+          for (; blk + 4 <= b1; blk += 4) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const int blk = b0 + j;
               uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-              if (g < NT) xv = *reinterpret_cast<const uint4*>(xrow + blk * 64);
-              const uint4 wv = *reinterpret_cast<const uint4*>(wrow + blk * 64);
+              if (g < NT) xv = *reinterpret_cast<const uint4*>(xrow + (blk + j) * 64);
+              const uint4 wv = *reinterpret_cast<const uint4*>(wrow + (blk + j) * 64);
               mma_bf16_m16n8k16(c[j], xv.x, xv.y, wv.x, wv.y);
               mma_bf16_m16n8k16(c[j], xv.z, xv.w, wv.z, wv.w);
             }
           }
+          for (; blk < b1; ++blk) {
+            uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+            if (g < NT) xv = *reinterpret_cast<const uint4*>(xrow + blk * 64);
+            const uint4 wv = *reinterpret_cast<const uint4*>(wrow + blk * 64);
+            mma_bf16_m16n8k16(c[0], xv.x, xv.y, wv.x, wv.y);
+            mma_bf16_m16n8k16(c[0], xv.z, xv.w, wv.z, wv.w);
+          }
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.empty_c[slot]);  // the warp's reads of the slot are done
-          // token g with staged rows 2q, 2q + 1: gate rows of pairs 2q, 2q + 1
-          // on lanes q = 0, 1; the matching up rows (4 + 2q, 5 + 2q) two lanes up
-          const float d0 = (c[0][0] + c[1][0]) + (c[2][0] + c[3][0]);
-          const float d1 = (c[0][1] + c[1][1]) + (c[2][1] + c[3][1]);
+          // token g with staged rows 2q, 2q + 1
+          d0 = (c[0][0] + c[1][0]) + (c[2][0] + c[3][0]);
+          d1 = (c[0][1] + c[1][1]) + (c[2][1] + c[3][1]);
+          if (part > 0)
+            partial[((slot * 2 + (f & 1)) * (kPartsC - 1) + part - 1) * 32 + lane] =
+                make_float2(d0, d1);
+        }
+        if (!bar_red_and(1 + slot, wps_c * 32, go)) break;
+        if (part == 0) {
+          for (int p2 = 1; p2 < wps_c; ++p2) {
+            const float2 v = partial[((slot * 2 + (f & 1)) * (kPartsC - 1) + p2 - 1) * 32 + lane];
+            d0 += v.x;
+            d1 += v.y;
+          }
+          // gate rows of pairs 2q, 2q + 1 on lanes q = 0, 1; the matching up
+          // rows (4 + 2q, 5 + 2q) two lanes up
           const float u0 = __shfl_down_sync(0xffffffffu, d0, 2);
           const float u1 = __shfl_down_sync(0xffffffffu, d1, 2);
           if (q < 2 && g < NT) {
@@ -595,52 +643,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
               hp[1] = __float2bfloat16_rn(silu(d1) * u1);
             }
           }
-        } else {
-          for (int rr = 0; rr < kStagePairs / kWPS; ++rr) {
-            const int r = half * (kStagePairs / kWPS) + rr;
-            const int p = gst * kStagePairs + r;
-            const int ui = p / m, j = p - ui * m;
-            const int s0 = sh.ufirst[ui], nt = sh.ufirst[ui + 1] - s0;  // <= NT
-            const uint4* wg = reinterpret_cast<const uint4*>(stage + (size_t)r * rs);
-            const uint4* wu = reinterpret_cast<const uint4*>(stage + (size_t)(r + kStagePairs) * rs);
-            const uint4* xq = reinterpret_cast<const uint4*>(xb);
-            int xo[NT];  // each kept token's row of bf16(x), in 16-byte chunks
-#pragma unroll
-            for (int t = 0; t < NT; ++t) xo[t] = (t < nt ? sh.slot_t[s0 + t] : 0) * (rs / 16);
-            float ga[NT], ua[NT];
-#pragma unroll
-            for (int t = 0; t < NT; ++t) ga[t] = ua[t] = 0.f;
-            for (int cc = lane; cc < d / 8; cc += 32) {
-              float w1[8], w2[8];
-              bf16x8_to_f32(wg[cc], w1);
-              bf16x8_to_f32(wu[cc], w2);
-#pragma unroll
-              for (int t = 0; t < NT; ++t) {
-                if (t < nt) {
-                  float xv[8];
-                  bf16x8_to_f32(xq[xo[t] + cc], xv);
-#pragma unroll
-                  for (int e = 0; e < 8; ++e) {
-                    ga[t] = fmaf(w1[e], xv[e], ga[t]);
-                    ua[t] = fmaf(w2[e], xv[e], ua[t]);
-                  }
-                }
-              }
-            }
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-              if (t < nt) {
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                  ga[t] += __shfl_xor_sync(0xffffffffu, ga[t], o);
-                  ua[t] += __shfl_xor_sync(0xffffffffu, ua[t], o);
-                }
-                if (lane == t) a.h[(size_t)(s0 + t) * m + j] = __float2bfloat16_rn(silu(ga[t]) * ua[t]);
-              }
-            }
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.empty_c[slot]);
         }
       }
     }
@@ -691,76 +693,80 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         }
       }
     } else {
-      // two groups of 8 warps take alternate experts (the phase-D ring is
-      // even, so a slot always belongs to one group); warp wl of a group owns
-      // the CTA's output rows wl and wl + 8 and sums, per token, g * (h W^down)
-      // over its group's experts in ascending order
-      const int grp = warp >> 3, wl = warp & 7;
-      if (lane < NT) {
-        sh.acc_d[grp][wl][lane] = 0.f;
-        sh.acc_d[grp][wl + 8][lane] = 0.f;
-      }
-      __syncwarp();
-      bool ok = true;
-      for (int ui = grp; ok && ui < U; ui += 2) {
-        const int slot = ui % nring_d;
-        if (!(ok = wait_bar(&sh.full_d[slot], (ui / nring_d) & 1, a, sh))) break;
-        const int s0 = sh.ufirst[ui], s1 = sh.ufirst[ui + 1];
-        // both rows of the warp in one pass: the h chunks are loaded once
-        // and the two rows' loads and reductions overlap
-        if (wl < nrows) {
-          const bool two = wl + 8 < nrows;
-          const __nv_bfloat16* hs =  // the stage's h rows: slot s0 + i at row i
-              reinterpret_cast<const __nv_bfloat16*>(ring_d + (size_t)slot * dstage + dbytes);
-          const uint4* w0 =
-              reinterpret_cast<const uint4*>(ring_d + (size_t)slot * dstage + (size_t)wl * m * 2);
-          const uint4* w1 = w0 + (two ? 8 * m / 8 : 0);
-          for (int sg = s0; sg < s1; sg += 4) {  // the expert's kept tokens, 4 at a time
-            const int nt = min(4, s1 - sg);
-            float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int c = lane; c < m / 8; c += 32) {
-              float a8[8], b8[8];
-              bf16x8_to_f32(w0[c], a8);
-              bf16x8_to_f32(w1[c], b8);
+      // Each ring slot has wps_d fixed consumer warps (parts), which take its
+      // fills (experts slot, slot + nring_d, ...) in order; part p covers the
+      // 32-wide blocks kb0 .. kb1 - 1 of the expert size.  One MMA tile per
+      // block pair of k: A = the stage's W^down rows (MMA rows: the CTA's
+      // output rows, rows nrows .. 15 zero), B = the stage's h rows (MMA
+      // columns: the expert's kept slots, columns nt .. 7 zero), with the
+      // same permutation of each block's 32 k on both operands as in phase C.
+      // The warp then adds g * (h W^down) of each kept slot into its own sums
+      // [16 rows][NT tokens] in shared memory (its lanes own distinct cells:
+      // a token keeps an expert once), experts in ascending order.
+      const int slot = warp / wps_d, part = warp % wps_d;
+      const int g = lane >> 2, q = lane & 3;
+      const int nbm = m / 32;
+      const int kb0 = part * nbm / wps_d, kb1 = (part + 1) * nbm / wps_d;
+      float* acc = reinterpret_cast<float*>(ring_d + (size_t)nring_d * dstage) + warp * 16 * NT;
+      const bool ra = g < nrows, rb = g + 8 < nrows;
+      if (slot < nring_d) {
+        for (int i = lane; i < 16 * NT; i += 32) acc[i] = 0.f;
+        __syncwarp();
+        for (int ui = slot; ui < U; ui += nring_d) {
+          const int f = ui / nring_d;
+          int ok = 1;
+          if (lane == 0) ok = wait_bar(&sh.full_d[slot], f & 1, a, sh);
+          if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+          mbar_try_wait(&sh.full_d[slot], f & 1);
+          const int s0 = sh.ufirst[ui], nt = sh.ufirst[ui + 1] - s0;  // <= NT
+          const uint8_t* st = ring_d + (size_t)slot * dstage;
+          const uint8_t* ar0 = st + (size_t)g * m * 2 + 16 * q;  // W^down row i0 + g
+          const uint8_t* ar1 = ar0 + (size_t)8 * m * 2;            // row i0 + g + 8
+          const uint8_t* br = st + dbytes + (size_t)g * m * 2 + 16 * q;  // h of slot s0 + g
+          const bool hb = g < nt;
+          float c[2][4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                if (q >= nt) break;
-                float hv[8];
-                bf16x8_to_f32(reinterpret_cast<const uint4*>(hs + (size_t)(sg + q - s0) * m)[c], hv);
+          for (int j = 0; j < 2; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.f;
+          for (int blk = kb0; blk < kb1; blk += 2) {
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                  d0[q] = fmaf(a8[cc], hv[cc], d0[q]);
-                  d1[q] = fmaf(b8[cc], hv[cc], d1[q]);
-                }
-              }
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (q >= nt) break;
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) {
-                d0[q] += __shfl_xor_sync(0xffffffffu, d0[q], o);
-                d1[q] += __shfl_xor_sync(0xffffffffu, d1[q], o);
-              }
-              if (lane == 0) {
-                const int t = sh.slot_t[sg + q];
-                const float gq = sh.slot_g[sg + q];
-                sh.acc_d[grp][wl][t] = fmaf(gq, d0[q], sh.acc_d[grp][wl][t]);
-                if (two) sh.acc_d[grp][wl + 8][t] = fmaf(gq, d1[q], sh.acc_d[grp][wl + 8][t]);
+            for (int j = 0; j < 2; ++j) {
+              if (blk + j < kb1) {
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                const uint4 av = ra ? *reinterpret_cast<const uint4*>(ar0 + (blk + j) * 64) : z;
+                const uint4 av8 = rb ? *reinterpret_cast<const uint4*>(ar1 + (blk + j) * 64) : z;
+                const uint4 hv = hb ? *reinterpret_cast<const uint4*>(br + (blk + j) * 64) : z;
+                mma_bf16_m16n8k16_full(c[j], av.x, av8.x, av.y, av8.y, hv.x, hv.y);
+                mma_bf16_m16n8k16_full(c[j], av.z, av8.z, av.w, av8.w, hv.z, hv.w);
               }
             }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.empty_d[slot]);  // the warp's reads of the slot are done
+          // lane (g, q): rows g, g + 8 with the slots s0 + 2q, s0 + 2q + 1
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int col = 2 * q + e2;
+            if (col < nt) {
+              const int t = sh.slot_t[s0 + col];
+              const float gq = sh.slot_g[s0 + col];
+              if (ra) acc[g * NT + t] = fmaf(gq, c[0][e2] + c[1][e2], acc[g * NT + t]);
+              if (rb) acc[(g + 8) * NT + t] = fmaf(gq, c[0][2 + e2] + c[1][2 + e2], acc[(g + 8) * NT + t]);
+            }
+          }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty_d[slot]);
       }
     }
   }
-  __syncthreads();  // both groups' sums are in
+  __syncthreads();  // every warp's sums are in
   if (producer && lane == 0) drain_copies(sh, nring, nring_d);  // (all consumed unless aborted)
-  if (warp < nrows && lane < NT)
-    a.y[(size_t)lane * d + i0 + warp] =
-        __float2bfloat16_rn(sh.acc_d[0][warp][lane] + sh.acc_d[1][warp][lane]);
+  if (nrows > 0 && (int)threadIdx.x < nrows * NT) {
+    // output row i0 + r of token t: the consumer warps' sums in warp order
+    const int r = threadIdx.x / NT, t = threadIdx.x - r * NT;
+    const float* acc0 = reinterpret_cast<const float*>(ring_d + (size_t)nring_d * dstage);
+    float v = 0.f;
+    for (int w = 0; w < nring_d * wps_d; ++w) v += acc0[(w * 16 + r) * NT + t];
+    a.y[(size_t)t * d + i0 + r] = __float2bfloat16_rn(v);
+  }
   stamp(a, 6);
 
   // debug / compaction outputs (CTA 0, off the critical path)
@@ -796,20 +802,18 @@ cudaError_t launch_nt(cudaLaunchConfig_t& cfg, const DecodeArgs& a, size_t smem)
 
 }  // namespace
 
-// Dynamic shared memory: [ring of nring 32 KB stages | bf16(x) [T][d]].  The
-// unrounded fp32 x and the staged inputs of phase A live inside the ring.
-static size_t region_bytes(int T, int d, int m, int k, int E, int num_sms) {
-  (void)m, (void)k, (void)E, (void)num_sms;
-  return (size_t)T * row_stride(d);  // bf16(x), padded rows
+// Dynamic shared memory in phase C: [ring of nring 33 KB stages | bf16(x)
+// [T][d], padded rows | partial dots].  The unrounded fp32 x and the staged
+// inputs of phase A live inside the ring.  Phase D reuses all of it: [its
+// ring | per-warp sums].
+static size_t region_bytes(int T, int d) {
+  return (size_t)T * row_stride(d) + kPartBytes;  // bf16(x), partial dots
 }
 
-static int ring_stages(int T, int d, int m, int k, int E, int num_sms) {
-  const size_t avail = (size_t)kSmemBudget - sizeof(DecShared) - 1024 -
-                       region_bytes(T, d, m, k, E, num_sms);
+static int ring_stages(int T, int d) {
+  const size_t avail = (size_t)kSmemBudget - sizeof(DecShared) - 1024 - region_bytes(T, d);
   const int n = (int)(avail / kStageBytes);
-  // any depth: a warp waits on a slot's full barrier only once the producer
-  // has claimed the slot for the warp's stage (the slot's earlier fill is
-  // then complete and consumed), so no wait can see an older phase
+  // any depth: each slot's warps wait on its fills in order
   return n > kRing ? kRing : n;
 }
 
@@ -824,7 +828,7 @@ bool decode_fits(int T, int d, int m, int k, int E, int num_sms) {
   // the bf16 shape rule of every entry point (d and m multiples of 128) also
   // keeps the staged rows and the MMA blocks of phase C whole
   if (T < 1 || T > kDecodeMaxT || d > 2048 || d % 128 != 0 || m % 128 != 0) return false;
-  const int n = ring_stages(T, d, m, k, E, num_sms);
+  const int n = ring_stages(T, d);
   if (n < 2) return false;
   // phase A inside the ring: x (fp32), u (bf16), gamma, the router rows
   const size_t staged = (size_t)T * d * 6 + (size_t)d * 4 +
@@ -832,9 +836,10 @@ bool decode_fits(int T, int d, int m, int k, int E, int num_sms) {
   if (staged > (size_t)n * kStageBytes) return false;
   const int rows = (d + num_sms - 1) / num_sms;                    // phase-D rows per CTA
   if (rows > kCompWarps) return false;
-  // phase D: at least two stages of W^down rows and an expert's h rows
-  const size_t dstage = ((size_t)rows * m * 2 + (size_t)T * m * 2 + 1023) & ~(size_t)1023;
-  return decode_smem_bytes(T, d, m, k, E, num_sms) >= 1024 + 2 * dstage;
+  // phase D: at least two stages of W^down rows and an expert's h rows, and
+  // the per-warp sums
+  return decode_smem_bytes(T, d, m, k, E, num_sms) >=
+         1024 + dacc_bytes(T) + 2 * dstage_bytes(rows, T, m);
 }
 
 cudaError_t launch_decode(const ace_layer& L, int fusion, const void* u, int T, float tau,
@@ -880,8 +885,9 @@ cudaError_t launch_decode(const ace_layer& L, int fusion, const void* u, int T, 
   a.status = status;
   a.trace = trace;
   a.peer_wait_ns = peer_wait_ns();
-  a.nring = ring_stages(T, L.d, L.m, L.k, L.E, num_sms);
+  a.nring = ring_stages(T, L.d);
   a.region = a.nring * kStageBytes;
+  a.part_off = a.region + T * row_stride(L.d);
   const size_t smem = decode_smem_bytes(T, L.d, L.m, L.k, L.E, num_sms);
   a.dyn_bytes = smem;
   cudaLaunchConfig_t cfg = {};
