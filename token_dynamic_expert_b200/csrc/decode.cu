@@ -54,7 +54,18 @@ constexpr int kMaxSlots = kDecodeMaxT * kMaxK;
 // 128: the 16-byte loads of a quarter warp (two rows, four consecutive
 // 16-byte pieces of each) then hit distinct banks.
 __host__ __device__ constexpr int row_stride(int d) { return 2 * d + 64; }
-constexpr int kStageBytes = kStageRows * row_stride(2048);  // bytes per ring slot (d <= 2048)
+// A phase-C stage (rows j0 .. j0 + 3 of W^gate and W^up) is four groups of
+// two consecutive rows, one bulk copy each: gate j0, j0 + 1 | gate j0 + 2,
+// j0 + 3 | up j0, j0 + 1 | up j0 + 2, j0 + 3, the groups 4d + 64 bytes apart.
+// MMA column n (0 .. 7) is group 2 (n >> 2) + (n & 1), row (n >> 1) & 1 of
+// it, i.e. gate pairs 0, 2, 1, 3 then up pairs 0, 2, 1, 3: the columns that a
+// quarter warp reads together (n even, n + 1) are one group apart, 64 bytes
+// modulo 128, so their 16-byte loads hit distinct banks.
+__host__ __device__ constexpr int group_stride(int d) { return 4 * d + 64; }
+__host__ __device__ constexpr int col_offset(int n, int d) {
+  return ((n >> 2) * 2 + (n & 1)) * group_stride(d) + ((n >> 1) & 1) * 2 * d;
+}
+constexpr int kStageBytes = 4 * group_stride(2048);  // bytes per ring slot (d <= 2048)
 // Phase C splits the hidden size of a stage over at most kPartsC warps; the
 // partial dots of parts 1 .. kPartsC - 1 meet part 0 in shared memory, two
 // buffers per slot (by fill parity)
@@ -361,31 +372,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   }
   __syncthreads();
   stamp(a, 1);
-  // router: warp w < n_mine (counting down from the last compute warp) dots
-  // its staged row with every token's x
-  const int rwarp = kCompWarps - 1 - warp;
-  if (warp < kCompWarps && rwarp < n_mine) {
-    const int my_e = (int)blockIdx.x + G * rwarp;
-    const uint4* wrow = reinterpret_cast<const uint4*>(wrs + (size_t)rwarp * d);
-    float acc[NT];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+  // router: the (row, token) dots of this CTA's staged rows, one per compute
+  // warp (counting down from the last one)
+  for (int it = kCompWarps - 1 - warp; warp < kCompWarps && it < n_mine * NT; it += kCompWarps) {
+    const int r = it / NT, t = it - r * NT;
+    const int my_e = (int)blockIdx.x + G * r;
+    const uint4* wrow = reinterpret_cast<const uint4*>(wrs + (size_t)r * d);
+    float acc = 0.f;
     for (int v = lane; v < d / 8; v += 32) {
-      float w[8];
+      float w[8], xv[8];
       bf16x8_to_f32(wrow[v], w);
+      lds8(xf + t * d + v * 8, xv);
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        float xv[8];
-        lds8(xf + t * d + v * 8, xv);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[t] = fmaf(xv[c], w[c], acc[t]);
-      }
+      for (int c = 0; c < 8; ++c) acc = fmaf(xv[c], w[c], acc);
     }
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      const float sm = warp_sum(acc[t]);
-      if (lane == 0) a.logits[(size_t)t * E + my_e] = sm + (a.bias ? a.bias[my_e] : 0.f);
-    }
+    const float sm = warp_sum(acc);
+    if (lane == 0) a.logits[(size_t)t * E + my_e] = sm + (a.bias ? a.bias[my_e] : 0.f);
   }
   if (!grid_barrier(a, sh, 1)) return;
   stamp(a, 2);
@@ -514,17 +516,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         const int slot = ls % nring;
         if (!(ok = wait_bar(&sh.empty_c[slot], ((ls / nring) & 1) ^ 1u, a, sh))) break;
         sh.slot_stage[slot] = gst;
-        // rows j0 .. j0 + 3 of W^gate, then of W^up, one padded row each
+        // rows j0 .. j0 + 3 of W^gate, then of W^up, two rows per copy
         const int pa = gst * kStagePairs, ui = pa / m, j0 = pa - ui * m;
         const size_t off = ((size_t)sh.uexp[ui] * m + j0) * d;
         mbar_expect_tx(&sh.full_c[slot], (uint32_t)(kStageRows * d * 2));
         uint8_t* sg = ring + (size_t)slot * kStageBytes;
-        for (int n = 0; n < kStagePairs; ++n) {
-          bulk_g2s(sg + (size_t)n * rs, a.wg + off + (size_t)n * d, (uint32_t)(d * 2),
-                   &sh.full_c[slot]);
-          bulk_g2s(sg + (size_t)(n + kStagePairs) * rs, a.wu + off + (size_t)n * d,
-                   (uint32_t)(d * 2), &sh.full_c[slot]);
-        }
+        const int gsz = group_stride(d);
+        bulk_g2s(sg, a.wg + off, (uint32_t)(d * 4), &sh.full_c[slot]);
+        bulk_g2s(sg + gsz, a.wg + off + 2 * (size_t)d, (uint32_t)(d * 4), &sh.full_c[slot]);
+        bulk_g2s(sg + 2 * gsz, a.wu + off, (uint32_t)(d * 4), &sh.full_c[slot]);
+        bulk_g2s(sg + 3 * gsz, a.wu + off + 2 * (size_t)d, (uint32_t)(d * 4), &sh.full_c[slot]);
       }
       sh.n_c_issued = ls;
       // End marks: the next fill of every slot carries stage -1 and no bytes
@@ -561,7 +562,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     // tokens (MMA rows; rows NT .. 15 are zero) with the stage's 8 rows (MMA
     // columns: 4 gate, 4 up) over its share of the hidden size, 32-wide
     // blocks b0 .. b1 - 1.  In each block, lane (g, q) holds the elements
-    // 8q .. 8q + 7 of token g's bf16(x) and of staged row g; the block's two
+    // 8q .. 8q + 7 of token g's bf16(x) and of the row of column g; the block's two
     // MMAs take elements 8q + {0..3} and 8q + {4..7} as the k of their
     // fragments, the same permutation of the block's 32 k on both operands,
     // so each MMA sums exact products of matching elements.  Parts 1, 2 leave
@@ -591,7 +592,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         const bool go = ok && gst >= 0;  // (gst < 0: end mark)
         float d0 = 0.f, d1 = 0.f;
         if (go) {
-          const uint8_t* wrow = ring + (size_t)slot * kStageBytes + (size_t)g * rs + 16 * q;
+          const uint8_t* wrow = ring + (size_t)slot * kStageBytes + col_offset(g, d) + 16 * q;
           float c[4][4];  // four accumulators (blocks mod 4), so the MMA chains overlap
 #pragma unroll
           for (int j = 0; j < 4; ++j) c[j][0] = c[j][1] = c[j][2] = c[j][3] = 0.f;
@@ -629,8 +630,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
             d0 += v.x;
             d1 += v.y;
           }
-          // gate rows of pairs 2q, 2q + 1 on lanes q = 0, 1; the matching up
-          // rows (4 + 2q, 5 + 2q) two lanes up
+          // lanes q = 0, 1 hold the gate dots of pairs q (column 2q) and
+          // q + 2 (column 2q + 1); the matching up dots are two lanes up
           const float u0 = __shfl_down_sync(0xffffffffu, d0, 2);
           const float u1 = __shfl_down_sync(0xffffffffu, d1, 2);
           if (q < 2 && g < NT) {
@@ -638,9 +639,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
             const uint32_t mk = sh.tok_mask[sh.uexp[ui]];
             if ((mk >> g) & 1u) {
               const int si = sh.ufirst[ui] + __popc(mk & ((1u << g) - 1u));
-              __nv_bfloat16* hp = a.h + (size_t)si * m + j0 + 2 * q;
+              __nv_bfloat16* hp = a.h + (size_t)si * m + j0 + q;
               hp[0] = __float2bfloat16_rn(silu(d0) * u0);
-              hp[1] = __float2bfloat16_rn(silu(d1) * u1);
+              hp[2] = __float2bfloat16_rn(silu(d1) * u1);
             }
           }
         }
