@@ -14,7 +14,10 @@
  *     (checkpoint preservation, [ACE] "Practical Implications").
  *   - The library allocates no device memory: scratch space is the caller's
  *     workspace `ws` of at least the size the matching *_workspace_size
- *     query returns, 256-byte aligned.
+ *     query returns, 256-byte aligned.  A workspace needs no initialisation
+ *     and may hold anything between calls: every call brings the words it
+ *     shares between CTAs to a known state itself (the decode kernel without
+ *     a clearing launch, see ace_moe_forward).
  *   - Weight, gamma, activation and output pointers are 16-byte aligned
  *     (the kernels move them in 16-byte vectors and bulk copies); tables
  *     are 4-byte aligned.  A misaligned pointer is ACE_ERR_INVALID_ARG.
@@ -194,6 +197,11 @@ ACE_API size_t ace_workspace_size(const ace_layer* layer, int max_tokens);
  *   dbg may be NULL.
  *   bf16 layers run the expert GEMMs on tcgen05 tensor cores and need
  *   d % 128 == 0 and m % 128 == 0; fp32 layers use CUDA cores.
+ *   Calls of 1-8 tokens on bf16 layers (d <= 2048) take the decode route:
+ *   one cooperative kernel whose grid barriers count in 64 bytes of the
+ *   workspace's status block; its last CTA writes the status word and
+ *   leaves those words zeroed and marked for the next call, so the route
+ *   launches nothing before the kernel.
  * ---------------------------------------------------------------------- */
 ACE_API ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T,
                            const ace_fwd_opts* opts, void* y, void* ws,

@@ -299,18 +299,23 @@ ace_status forward_impl(const ace_layer* layer, const void* u, int T, const ace_
   const FwdLayout ly = fwd_layout(L, T, num_sms);
   if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // status word (offset 0), the decode kernel's grid-barrier words (byte 64)
-  // and the routing CTAs' completion count (byte 128)
-  if (keep_status)
-    ACE_CK(launch_clear_words(at<uint8_t>(ws, ly.status) + 64, 48, s));
-  else
-    ACE_CK(launch_clear_words(at<void>(ws, ly.status), 64, s));
+  const bool decode = T > 0 && L.dtype == ACE_BF16 && T <= kDecodeMaxT &&
+                      decode_fits(T, L.d, L.m, L.k, L.E, num_sms);
+  // status word (offset 0), the decode kernel's cross-CTA words (byte 64)
+  // and the routing CTAs' completion count (byte 128).  The decode kernel
+  // needs no clearing: its words carry their launch's epoch, and it writes
+  // the status word itself as it finishes.
+  if (!decode) {
+    if (keep_status)
+      ACE_CK(launch_clear_words(at<uint8_t>(ws, ly.status) + 64, 48, s));
+    else
+      ACE_CK(launch_clear_words(at<void>(ws, ly.status), 64, s));
+  }
   if (T == 0) return ACE_OK;
   cudaEvent_t ev_b = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_begin) : nullptr;
   cudaEvent_t ev_m = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_mid) : nullptr;
   cudaEvent_t ev_e = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_end) : nullptr;
 
-  const bool decode = L.dtype == ACE_BF16 && T <= kDecodeMaxT && decode_fits(T, L.d, L.m, L.k, L.E, num_sms);
   if (decode) {
     // decode: one cooperative kernel streams the surviving experts' weights
     if (ev_b) ACE_CK(cudaEventRecord(ev_b, s));
@@ -321,7 +326,8 @@ ace_status forward_impl(const ace_layer* layer, const void* u, int T, const ace_
                          at<int32_t>(ws, ly.offsets), at<int32_t>(ws, ly.slot_token),
                          at<int32_t>(ws, ly.slot_rank), at<int32_t>(ws, ly.slot_of),
                          at<int32_t>(ws, ly.n_kept), at<uint32_t>(ws, ly.status) + 16,
-                         at<uint32_t>(ws, ly.status), dbg ? dbg->trace : nullptr, num_sms, s));
+                         at<uint32_t>(ws, ly.status), keep_status, dbg ? dbg->trace : nullptr,
+                         num_sms, s));
     if (ev_e) ACE_CK(cudaEventRecord(ev_e, s));
   } else {
     st = run_prefill(L, u, T, *opts, y, ly, ws, num_sms, dbg, ev_b, ev_m, ev_e, s);

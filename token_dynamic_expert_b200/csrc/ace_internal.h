@@ -98,7 +98,7 @@ cudaError_t launch_decode(const ace_layer& L, int fusion, const void* u, int T, 
                           float eps_rms, void* y, float* logits, void* h, int32_t* idx,
                           float* gate, float* score, uint8_t* keep, int32_t* offsets,
                           int32_t* slot_token, int32_t* slot_rank, int32_t* slot_of,
-                          int32_t* n_kept, uint32_t* bar, uint32_t* status,
+                          int32_t* n_kept, uint32_t* sync, uint32_t* status, bool keep_status,
                           unsigned long long* trace, int num_sms, cudaStream_t s);
 size_t tables_workspace_size(const ace_layer& L);
 ace_status build_tables_impl(const ace_layer* layers, int n_layers, const ace_table_opts& o,

@@ -98,8 +98,9 @@ struct DecodeArgs {
   int32_t* slot_rank;     // [T*k]
   int32_t* slot_of;       // [T][k]
   int32_t* n_kept;        // [1]
-  uint32_t* bar_count;
-  uint32_t* status;
+  uint32_t* sync;             // [16] the launch epoch and its cross-CTA counters
+  uint32_t* status;           // the call's status word (written at the end)
+  int keep_status;            // add the flags to the status word, else replace it
   unsigned long long* trace;  // optional [grid][8] phase stamps
   uint64_t peer_wait_ns;      // limit of a grid-barrier wait
   int nring;                  // stages of the copy ring for this call
@@ -129,6 +130,9 @@ struct DecShared {
   uint64_t in_bar;             // phase A: u, gamma and the router rows have landed
   int slot_stage[kRing];       // phase C: the stage a ring slot holds (-1: no more)
   int abort;
+  uint32_t flags;              // ACE_FLAG_* bits this CTA raised
+  uint32_t epoch;              // the launch's epoch (word 0 of the sync words)
+  int fast;                    // the sync words are marked clean for this epoch
   // bulk copies the producer issued, so that a CTA leaving early lets them land
   int n_c_issued;              // phase-C stages (ring slot = stage % nring)
   int n_c_marked;              // phase-C end marks after them (one more phase per slot)
@@ -151,25 +155,176 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// the same, with an L2 eviction-priority policy for the copied lines
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Expert weights are read once per call: their lines go first when L2 needs
+// room, so they do not push out what the call reads again (h, the logits,
+// the tables, the kernel's code)
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ void stamp(const DecodeArgs& a, int i) {
   if (a.trace && threadIdx.x == 0) a.trace[blockIdx.x * 8 + i] = global_ns();
 }
 
-// Grid-wide barrier number `n` (1, 2, ...) over co-resident CTAs: a
-// monotonic arrival counter (zeroed before the launch); the barrier opens when
-// it reaches n * gridDim.x.  False when the bounded wait ran out
-// (ACE_FLAG_TIMEOUT raised) or an earlier wait failed.
+// Cross-CTA words of a launch (sync: 16 words in the caller's workspace).
+//   word 0      the launch epoch e
+//   word 1      e ^ kCleanMark when words 2-4 are clean (zero)
+//   words 2-4   arrivals, departures and raised flags (fast path)
+//   words 6-11  the same as 64-bit words tagged with e ^ kTagMark in the
+//               high half (slow path)
+// The last CTA to depart writes the launch's flags into the status word,
+// zeroes words 2-4, and marks them clean for epoch e + 1.  So the words need
+// no clearing before a launch (nor a kernel to clear them: inside a CUDA
+// graph that node costs about a microsecond per layer), and a launch that gave
+// up part way through still leaves them clean.  A workspace whose words were
+// never written (or were cleared, or hold anything else) lacks the mark; every
+// CTA reads the mark before any CTA writes a word, so they all take the slow
+// path, where the first CTA to touch a word whose tag is not this launch's
+// re-tags it with a zero count.  A uniform fill (all zero or all ones bytes)
+// can match neither mark; other garbage matches one with odds 2^-32.
+constexpr uint32_t kCleanMark = 0x5bd1e995u;
+constexpr uint32_t kTagMark = 0x9e3779b9u;
+
+__device__ __forceinline__ uint32_t ld_acquire32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t add_acq_rel32(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ uint32_t add_release32(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ uint64_t ld_acquire64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t ld_relaxed64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t cas_acq_rel64(uint64_t* p, uint64_t cmp, uint64_t val) {
+  uint64_t old;
+  asm volatile("atom.acq_rel.gpu.global.cas.b64 %0, [%1], %2, %3;"
+               : "=l"(old) : "l"(p), "l"(cmp), "l"(val) : "memory");
+  return old;
+}
+__device__ __forceinline__ uint64_t add_acq_rel64(uint64_t* p, uint64_t v) {
+  uint64_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ bool tagged(uint64_t v, uint32_t e) {
+  return (uint32_t)(v >> 32) == (e ^ kTagMark);
+}
+__device__ __forceinline__ uint64_t tag_of(uint32_t e) { return (uint64_t)(e ^ kTagMark) << 32; }
+
+// Slow path: adds one to the count of epoch e in word w; returns the count
+// before.
+__device__ uint32_t epoch_add(uint64_t* w, uint32_t e) {
+  uint64_t v = ld_relaxed64(w);
+  for (;;) {
+    // once tagged e, a word keeps the tag for the rest of the launch
+    if (tagged(v, e)) return (uint32_t)add_acq_rel64(w, 1ull);
+    const uint64_t seen = cas_acq_rel64(w, v, tag_of(e) | 1ull);
+    if (seen == v) return 0u;
+    v = seen;
+  }
+}
+
+// Slow path: ORs `bits` into the flags of epoch e in word w.
+__device__ void epoch_or(uint64_t* w, uint32_t e, uint32_t bits) {
+  uint64_t v = ld_relaxed64(w);
+  for (;;) {
+    const uint64_t want = tag_of(e) | ((tagged(v, e) ? (uint32_t)v : 0u) | bits);
+    if (want == v) return;
+    const uint64_t seen = cas_acq_rel64(w, v, want);
+    if (seen == v) return;
+    v = seen;
+  }
+}
+
+// Called once by thread 0 of every CTA as it leaves (normally or after a
+// failed wait), when the CTA's flags are final and it touches no more
+// cross-CTA word.
+__device__ void depart(const DecodeArgs& a, DecShared& sh) {
+  uint32_t* w = a.sync;
+  uint64_t* w64 = reinterpret_cast<uint64_t*>(a.sync);
+  const uint32_t e = sh.epoch;
+  bool last;
+  if (sh.fast) {
+    if (sh.flags) atomicOr(w + 4, sh.flags);
+    last = add_acq_rel32(w + 3, 1u) == gridDim.x - 1;
+  } else {
+    if (sh.flags) epoch_or(w64 + 5, e, sh.flags);
+    last = epoch_add(w64 + 4, e) == gridDim.x - 1;
+  }
+  if (last) {
+    // the last CTA out: every other CTA has published its flags and left its
+    // barriers
+    uint32_t flags;
+    if (sh.fast) {
+      flags = ld_acquire32(w + 4);
+    } else {
+      const uint64_t p = ld_acquire64(w64 + 5);
+      flags = tagged(p, e) ? (uint32_t)p : 0u;
+    }
+    if (a.keep_status) {
+      if (flags) atomicOr(a.status, flags);
+    } else {
+      *reinterpret_cast<volatile uint32_t*>(a.status) = flags;
+    }
+    // (the next launch starts after this one ends, which orders these)
+    w[2] = 0u;
+    w[3] = 0u;
+    w[4] = 0u;
+    w[1] = (e + 1u) ^ kCleanMark;
+    w[0] = e + 1u;
+  }
+}
+
+// Grid-wide barrier number `n` (1, 2, ...) over co-resident CTAs: it opens
+// when the launch's arrival count reaches n * gridDim.x.  False when the
+// bounded wait ran out (ACE_FLAG_TIMEOUT raised) or an earlier wait failed.
 __device__ bool grid_barrier(const DecodeArgs& a, DecShared& sh, uint32_t n) {
   __syncthreads();
   if (threadIdx.x == 0 && !sh.abort) {
-    const uint32_t target = n * gridDim.x;
-    uint32_t seen;
-    asm volatile("atom.add.release.gpu.global.u32 %0, [%1], 1;" : "=r"(seen) : "l"(a.bar_count) : "memory");
-    if (seen + 1 < target) {
+    const uint32_t e = sh.epoch, target = n * gridDim.x;
+    uint32_t* w = a.sync + 2;
+    uint64_t* w64 = reinterpret_cast<uint64_t*>(a.sync) + 3;
+    const uint32_t before = sh.fast ? add_release32(w, 1u) : epoch_add(w64, e);
+    if (before + 1 < target) {
       const uint64_t t0 = global_ns();
-      while (ld_acquire(a.bar_count) < target) {
+      for (;;) {
+        bool open;
+        if (sh.fast) {
+          open = ld_acquire32(w) >= target;
+        } else {
+          const uint64_t v = ld_acquire64(w64);
+          open = tagged(v, e) && (uint32_t)v >= target;
+        }
+        if (open) break;
         if (global_ns() - t0 > a.peer_wait_ns) {
-          raise_flag(a.status, ACE_FLAG_TIMEOUT);
+          raise_flag(&sh.flags, ACE_FLAG_TIMEOUT);
           sh.abort = 1;
           break;
         }
@@ -182,7 +337,7 @@ __device__ bool grid_barrier(const DecodeArgs& a, DecShared& sh, uint32_t n) {
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const DecodeArgs& a,
                                          DecShared& sh) {
-  return mbar_wait(bar, parity, a.status, &sh.abort);
+  return mbar_wait(bar, parity, &sh.flags, &sh.abort);
 }
 
 // Waits (fixed limit) until the last fill of every ring slot that received
@@ -308,6 +463,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   const int wps_d = min(min(kPartsD, kCompWarps / nring_d), m / 32);
   if (threadIdx.x == 0) {
     sh.abort = 0;
+    sh.flags = 0u;
+    volatile const uint32_t* vs = a.sync;
+    sh.epoch = vs[0];
+    sh.fast = vs[1] == (sh.epoch ^ kCleanMark);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sh.full_c[i], 1);
       mbar_init(&sh.empty_c[i], wps_c);  // the slot's warps
@@ -337,7 +496,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   // phase B then looks them up in shared memory
   for (int e = kDecThreads - 1 - (int)threadIdx.x; e < E; e += kDecThreads)
     sh.fac[e] = fused_factor(a.ft, e);
-  if (!wait_bar(&sh.in_bar, 0, a, sh)) return;
+  const bool in_ok = wait_bar(&sh.in_bar, 0, a, sh);
+  if (__syncthreads_or(!in_ok)) {
+    if (threadIdx.x == 0) depart(a, sh);
+    return;
+  }
   if (warp < NT) {  // token warps: x = u / rms(u) * gamma
     const int t = warp;
     const uint4* ur = reinterpret_cast<const uint4*>(us + (size_t)t * d);
@@ -389,7 +552,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     const float sm = warp_sum(acc);
     if (lane == 0) a.logits[(size_t)t * E + my_e] = sm + (a.bias ? a.bias[my_e] : 0.f);
   }
-  if (!grid_barrier(a, sh, 1)) return;
+  if (!grid_barrier(a, sh, 1)) {
+    if (threadIdx.x == 0) depart(a, sh);
+    return;
+  }
   stamp(a, 2);
 
   // ---------------------------------------------------------- phase B
@@ -404,7 +570,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     }
     int sel_e = 0;
     float sel_v = -INFINITY;
-    topk_select(v, nq, E, k, lane, sel_e, sel_v, a.status);
+    topk_select(v, nq, E, k, lane, sel_e, sel_v, &sh.flags);
     const float v0 = __shfl_sync(0xffffffffu, sel_v, 0);
     const float ex = lane < k ? expf(sel_v - v0) : 0.f;
     float denom;
@@ -522,10 +688,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
         mbar_expect_tx(&sh.full_c[slot], (uint32_t)(kStageRows * d * 2));
         uint8_t* sg = ring + (size_t)slot * kStageBytes;
         const int gsz = group_stride(d);
-        bulk_g2s(sg, a.wg + off, (uint32_t)(d * 4), &sh.full_c[slot]);
-        bulk_g2s(sg + gsz, a.wg + off + 2 * (size_t)d, (uint32_t)(d * 4), &sh.full_c[slot]);
-        bulk_g2s(sg + 2 * gsz, a.wu + off, (uint32_t)(d * 4), &sh.full_c[slot]);
-        bulk_g2s(sg + 3 * gsz, a.wu + off + 2 * (size_t)d, (uint32_t)(d * 4), &sh.full_c[slot]);
+        const uint64_t pol = evict_first_policy();
+        bulk_g2s_hint(sg, a.wg + off, (uint32_t)(d * 4), &sh.full_c[slot], pol);
+        bulk_g2s_hint(sg + gsz, a.wg + off + 2 * (size_t)d, (uint32_t)(d * 4), &sh.full_c[slot], pol);
+        bulk_g2s_hint(sg + 2 * gsz, a.wu + off, (uint32_t)(d * 4), &sh.full_c[slot], pol);
+        bulk_g2s_hint(sg + 3 * gsz, a.wu + off + 2 * (size_t)d, (uint32_t)(d * 4), &sh.full_c[slot],
+                      pol);
       }
       sh.n_c_issued = ls;
       // End marks: the next fill of every slot carries stage -1 and no bytes
@@ -546,8 +714,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
           // same phase of the barrier
           const uint32_t hb = (uint32_t)((sh.ufirst[ui + 1] - sh.ufirst[ui]) * m * 2);
           mbar_expect_tx(&sh.full_d[ui], dbytes + hb);
-          bulk_g2s(ring_d + (size_t)ui * dstage, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m,
-                   dbytes, &sh.full_d[ui]);
+          bulk_g2s_hint(ring_d + (size_t)ui * dstage, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m,
+                        dbytes, &sh.full_d[ui], evict_first_policy());
           sh.n_d_issued = ui + 1;
         }
       }
@@ -663,6 +831,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       }
       drain_copies(sh, nring, nring_d);
     }
+    if (threadIdx.x == 0) depart(a, sh);
     return;
   }
   stamp(a, 5);
@@ -688,7 +857,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
           const uint32_t hb = (uint32_t)((sh.ufirst[ui + 1] - s0) * m * 2);
           uint8_t* st = ring_d + (size_t)slot * dstage;
           mbar_expect_tx(&sh.full_d[slot], dbytes + hb);
-          bulk_g2s(st, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m, dbytes, &sh.full_d[slot]);
+          bulk_g2s_hint(st, a.wd + ((size_t)sh.uexp[ui] * d + i0) * m, dbytes, &sh.full_d[slot],
+                        evict_first_policy());
           bulk_g2s(st + dbytes, a.h + (size_t)s0 * m, hb, &sh.full_d[slot]);
           sh.n_d_issued = ui + 1;
         }
@@ -787,6 +957,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     for (int e = threadIdx.x; e <= E; e += blockDim.x) a.offsets[e] = e < E ? sh.e_base[e] : S;
     if (threadIdx.x == 0) *a.n_kept = S;
   }
+  if (threadIdx.x == 0) depart(a, sh);
 }
 
 template <int NT>
@@ -848,7 +1019,7 @@ cudaError_t launch_decode(const ace_layer& L, int fusion, const void* u, int T, 
                           float eps_rms, void* y, float* logits, void* h, int32_t* idx,
                           float* gate, float* score, uint8_t* keep, int32_t* offsets,
                           int32_t* slot_token, int32_t* slot_rank, int32_t* slot_of,
-                          int32_t* n_kept, uint32_t* bar, uint32_t* status,
+                          int32_t* n_kept, uint32_t* sync, uint32_t* status, bool keep_status,
                           unsigned long long* trace, int num_sms, cudaStream_t s) {
   DecodeArgs a;
   a.gamma = L.gamma;
@@ -882,8 +1053,9 @@ cudaError_t launch_decode(const ace_layer& L, int fusion, const void* u, int T, 
   a.slot_rank = slot_rank;
   a.slot_of = slot_of;
   a.n_kept = n_kept;
-  a.bar_count = bar;
+  a.sync = sync;
   a.status = status;
+  a.keep_status = keep_status ? 1 : 0;
   a.trace = trace;
   a.peer_wait_ns = peer_wait_ns();
   a.nring = ring_stages(T, L.d);

@@ -109,7 +109,8 @@ extern "C" ace_status ace_moe_decode_noalloc(const ace_layer* layer, const void*
   if (scratch_address(&base) != cudaSuccess) return ACE_ERR_CUDA;
   uint8_t* w = static_cast<uint8_t*>(base);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the status word and the grid-barrier counter must start at zero
+  // the status word and the decode kernel's cross-CTA words (byte 64) start
+  // from zero
   if (launch_clear_words(w, 64, s) != cudaSuccess) return ACE_ERR_CUDA;
   auto at = [&](size_t off) { return w + off; };
   if (launch_decode(L, (int)opts->fusion, u, T, opts->tau, opts->renorm_topk, opts->eps_rms, y,
@@ -121,8 +122,8 @@ extern "C" ace_status ace_moe_decode_noalloc(const ace_layer* layer, const void*
                     reinterpret_cast<int32_t*>(at(ly.slot_rank)),
                     reinterpret_cast<int32_t*>(at(ly.slot_of)),
                     reinterpret_cast<int32_t*>(at(ly.n_kept)),
-                    reinterpret_cast<uint32_t*>(w) + 16, reinterpret_cast<uint32_t*>(w), nullptr,
-                    num_sms, s) != cudaSuccess)
+                    reinterpret_cast<uint32_t*>(w) + 16, reinterpret_cast<uint32_t*>(w), false,
+                    nullptr, num_sms, s) != cudaSuccess)
     return ACE_ERR_CUDA;
   return ACE_OK;
 }
