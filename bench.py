@@ -36,8 +36,8 @@ import workloads  # noqa: E402
 METRIC = "MoE-layer tokens/s (prefill, decode) at skip rate; % of tensor/HBM roofline"
 
 # DRAM traffic (read + write bytes) per launch of the dominant kernel from one ncu
-# capture (profiles/k_experts_prefill_1024.md); reported only while the kernel's
-# source is the revision the counters were taken on.
+# capture of that kernel on that workload; reported only while the kernel's source
+# is the revision the counters were taken on.
 PROFILED_TRAFFIC = {
     ("prefill_1024", "gateup"): ("token_dynamic_expert_b200/csrc/experts_sm100.cu", "06d17ea9eed8",
                                  825441792),
@@ -57,8 +57,8 @@ def profiled_traffic(workload, kernel):
 # status clear, rmsnorm, router GEMM, top-k/mask (+ offset scan), scatter+gather, the expert
 # GEMMs (one fused launch for small slot tiles, else gate/up and down), combine
 KERNELS_PER_FORWARD = {True: 7, False: 8}
-# per decode layer: status clear, the decode kernel
-KERNELS_PER_DECODE_LAYER = 2
+# per decode layer: the decode kernel alone (its grid-barrier words reset themselves)
+KERNELS_PER_DECODE_LAYER = 1
 
 
 # ----------------------------------------------------------------- helpers
