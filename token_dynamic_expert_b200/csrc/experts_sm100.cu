@@ -45,9 +45,9 @@ namespace {
 
 constexpr int kBM = 128;                    // MMA M (weight rows per A tile)
 constexpr int kBK = 64;                     // K per stage: one 128-B swizzle row of bf16
-constexpr int kBoxN = 32;                   // slot rows per B TMA box
+constexpr int kBoxN = 64;                   // slot rows per B TMA box (fewer, larger loads)
 constexpr int kAStage = kBM * kBK * 2;      // 16 KB
-constexpr int kBoxBytes = kBoxN * kBK * 2;  // 4 KB
+constexpr int kBoxBytes = kBoxN * kBK * 2;  // 8 KB
 constexpr int kMaxStages = 8;
 constexpr int kStageBudget = 200 * 1024;
 constexpr int kXchgBytes = 2 * 2 * 64 * 8 * 4;  // 2 buffers x (gate, up) x 64 rows x 8 floats
