@@ -248,6 +248,65 @@ ACE_API ace_status ace_moe_scores(const ace_layer* layer, const void* u, int T,
                           void* stream);
 
 /* ------------------------------------------------------------------------
+ * ace_moe_route -- the routing half of the forward with its decisions, the
+ *   first step of expert-parallel dispatch ([ACE] "Conclusion", future
+ *   directions: distributed expert dispatch): a rank routes its own tokens,
+ *   then sends each kept slot to the rank that owns the slot's expert.
+ *   Same kernels as ace_moe_forward, so the same bits.
+ *   x (device) [T][d] layer->dtype, 16-byte aligned: the experts' input
+ *   rows (bf16(x) for bf16 layers, x for fp32 layers); idx (device) [T][k]
+ *   int32 experts, column 0 = top-1; gate (device) [T][k] fp32 gates;
+ *   keep (device) [T][k] uint8, 1 = kept (top-1 always).  Workspace: at
+ *   least ace_workspace_size(layer, T) bytes.  The expert weights are not
+ *   read and may be NULL.
+ * ---------------------------------------------------------------------- */
+ACE_API ace_status ace_moe_route(const ace_layer* layer, const void* u, int T,
+                                 const ace_fwd_opts* opts, void* x, int32_t* idx,
+                                 float* gate, uint8_t* keep, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* ------------------------------------------------------------------------
+ * ace_experts_workspace_size -- bytes of workspace ace_moe_experts needs for
+ *   up to max_slots slots of `layer`; 0 for an invalid expert layer.
+ *
+ * ace_moe_experts -- the SwiGLU experts of `layer` on S kept slots grouped by
+ *   expert, the owner's step of expert-parallel dispatch:
+ *     yslot[s] = slot_gate[s] * f_e(xp[s])  for offsets[e] <= s < offsets[e+1]
+ *   with f_e as in ace_moe_forward ([ACE] "Theoretical Foundation", the
+ *   SwiGLU expert).  `layer` holds only the experts the caller owns (E of
+ *   them, d, m, dtype and the three expert matrices); the router, gamma and
+ *   k are not read.  xp (device) [S][d] layer->dtype, 16-byte aligned;
+ *   offsets (device) [E+1] int32, rising from 0 to S (otherwise
+ *   ACE_FLAG_BAD_INDEX is raised and nothing is computed); slot_gate
+ *   (device) [S] fp32; yslot (device) [S][d] fp32, 16-byte aligned.
+ *   Same kernels and numerics as the forward's expert GEMMs (h rounded to
+ *   the storage type, fp32 accumulation).  Device flags: ace_read_status
+ *   on ws.
+ * ---------------------------------------------------------------------- */
+ACE_API size_t ace_experts_workspace_size(const ace_layer* layer, int max_slots);
+ACE_API ace_status ace_moe_experts(const ace_layer* layer, const void* xp, int S,
+                                   const int32_t* offsets, const float* slot_gate,
+                                   float* yslot, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * ace_moe_combine -- the forward's combine on slot outputs the caller
+ *   gathered (in expert-parallel dispatch: the outputs of a rank's kept
+ *   slots, back from their experts' owners):
+ *     y_t = sum over i = 0 .. k-1 with slot_of[t][i] >= 0, in that order, of
+ *           yslot[slot_of[t][i]]
+ *   in fp32, rounded once to dtype ([ACE] "Theoretical Foundation": the
+ *   gate-weighted sum of the kept experts; the gates are already in yslot,
+ *   skipped slots drop out without re-normalising).
+ *   slot_of (device) [T][k] int32, -1 for a skipped slot; yslot (device)
+ *   [n_rows][d] fp32, 16-byte aligned; y (device) [T][d] dtype, 16-byte
+ *   aligned; d % 4 == 0.  An index >= n_rows raises ACE_FLAG_BAD_INDEX and
+ *   drops out.  ws: at least 256 bytes (its status word; ace_read_status).
+ * ---------------------------------------------------------------------- */
+ACE_API ace_status ace_moe_combine(int T, int k, int d, ace_dtype dtype, const int32_t* slot_of,
+                                   const float* yslot, int n_rows, void* y, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * ace_moe_decode_noalloc -- the decode forward (1 <= T <= 8 tokens, bf16
  *   layers) for callers that cannot allocate device memory.  The paper has
  *   no counterpart: this is a deployment variant of ace_moe_forward.

@@ -64,6 +64,17 @@ _lib.ace_moe_forward.restype = ctypes.c_int
 _lib.ace_moe_scores.argtypes = [_P(ace_layer), _vp, ctypes.c_int, _P(ace_fwd_opts), _vp, _vp, _vp,
                                 ctypes.c_size_t, _vp]
 _lib.ace_moe_scores.restype = ctypes.c_int
+_lib.ace_moe_route.argtypes = [_P(ace_layer), _vp, ctypes.c_int, _P(ace_fwd_opts), _vp, _vp, _vp,
+                               _vp, _vp, ctypes.c_size_t, _vp]
+_lib.ace_moe_route.restype = ctypes.c_int
+_lib.ace_experts_workspace_size.argtypes = [_P(ace_layer), ctypes.c_int]
+_lib.ace_experts_workspace_size.restype = ctypes.c_size_t
+_lib.ace_moe_experts.argtypes = [_P(ace_layer), _vp, ctypes.c_int, _vp, _vp, _vp, _vp,
+                                 ctypes.c_size_t, _vp]
+_lib.ace_moe_experts.restype = ctypes.c_int
+_lib.ace_moe_combine.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp,
+                                 ctypes.c_int, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.ace_moe_combine.restype = ctypes.c_int
 _lib.ace_moe_decode_noalloc.argtypes = [_P(ace_layer), _vp, ctypes.c_int, _P(ace_fwd_opts), _vp,
                                         _vp]
 _lib.ace_moe_decode_noalloc.restype = ctypes.c_int
@@ -185,6 +196,56 @@ def ace_moe_scores(layer, u, score, ws, topk_idx=None, renorm=True, eps_rms=1e-6
                                _ptr(score), _ptr(topk_idx), _ptr(ws), ws.numel(), _stream(stream))
     _check(code, "ace_moe_scores")
     return score
+
+
+def ace_moe_route(layer, u, tau, x, idx, gate, keep, ws, renorm=True, eps_rms=1e-6, stream=None,
+                  fusion="max"):
+    """Routing with its decisions (see include/ace.h): x [T][d] the experts'
+    input rows, idx / gate [T][k], keep [T][k] uint8."""
+    opts = ace_fwd_opts(tau=float(tau), renorm_topk=int(bool(renorm)), fusion=_fusion(fusion),
+                        eps_rms=float(eps_rms))
+    code = _lib.ace_moe_route(ctypes.byref(layer), _ptr(u), int(u.shape[0]), ctypes.byref(opts),
+                              _ptr(x), _ptr(idx), _ptr(gate), _ptr(keep), _ptr(ws), ws.numel(),
+                              _stream(stream))
+    _check(code, "ace_moe_route")
+    return x, idx, gate, keep
+
+
+def make_expert_layer(w_gate, w_up, w_down):
+    """An ``ace_layer`` holding only experts (for ace_moe_experts): E, m, d
+    from the weight shapes [E][m][d] and [E][d][m]."""
+    for t in (w_gate, w_up, w_down):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    E, m, d = w_gate.shape
+    return ace_layer(d=d, E=E, m=m, k=1, dtype=_dtype_code(w_gate), gamma=None, w_router=None,
+                     router_bias=None, w_gate=_ptr(w_gate), w_up=_ptr(w_up), w_down=_ptr(w_down),
+                     amax=None, a_gsp=None, a_rcr=None)
+
+
+def ace_experts_workspace_size(layer, max_slots):
+    return int(_lib.ace_experts_workspace_size(ctypes.byref(layer), int(max_slots)))
+
+
+def ace_moe_experts(layer, xp, offsets, slot_gate, yslot, ws, stream=None):
+    """yslot[s] = slot_gate[s] * f_e(xp[s]) for the slots of expert e,
+    offsets[e] <= s < offsets[e + 1] (see include/ace.h)."""
+    code = _lib.ace_moe_experts(ctypes.byref(layer), _ptr(xp), int(xp.shape[0]), _ptr(offsets),
+                                _ptr(slot_gate), _ptr(yslot), _ptr(ws), ws.numel(),
+                                _stream(stream))
+    _check(code, "ace_moe_experts")
+    return yslot
+
+
+def ace_moe_combine(slot_of, yslot, y, ws, stream=None):
+    """y[t] = sum over i of yslot[slot_of[t, i]] for slot_of >= 0, in i order
+    (see include/ace.h); slot_of [T][k] int32, yslot [n][d] fp32."""
+    T, k = slot_of.shape
+    code = _lib.ace_moe_combine(int(T), int(k), int(y.shape[1]), _dtype_code(y), _ptr(slot_of),
+                                _ptr(yslot), int(yslot.shape[0]), _ptr(y), _ptr(ws), ws.numel(),
+                                _stream(stream))
+    _check(code, "ace_moe_combine")
+    return y
 
 
 def ace_moe_decode_noalloc(layer, u, tau, y, renorm=True, eps_rms=1e-6, stream=None,

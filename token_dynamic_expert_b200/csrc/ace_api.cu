@@ -262,7 +262,7 @@ ace_status run_prefill(const ace_layer& L, const void* u, int T, const ace_fwd_o
   }
   if (ev_e) ACE_CK(cudaEventRecord(ev_e, s));
   ACE_CK(launch_combine(L.dtype, T, L.k, L.d, at<int32_t>(ws, ly.slot_of), at<float>(ws, ly.yslot),
-                        y, s));
+                        T * L.k, y, at<uint32_t>(ws, ly.status), s));
   return ACE_OK;
 }
 
@@ -448,6 +448,35 @@ ace_status ace_moe_scores(const ace_layer* layer, const void* u, int T, const ac
   ACE_CK(cudaMemcpyAsync(score, at<void>(ws, ly.score), tk * 4, cudaMemcpyDeviceToDevice, s));
   if (topk_idx)
     ACE_CK(cudaMemcpyAsync(topk_idx, at<void>(ws, ly.idx), tk * 4, cudaMemcpyDeviceToDevice, s));
+  return ACE_OK;
+}
+
+ace_status ace_moe_route(const ace_layer* layer, const void* u, int T, const ace_fwd_opts* opts,
+                         void* x, int32_t* idx, float* gate, uint8_t* keep, void* ws,
+                         size_t ws_bytes, void* stream) {
+  ace_status st = check_common(layer, u, T, opts, ws, false);
+  if (st != ACE_OK) return st;
+  if (T > 0 && (!x || !idx || !gate || !keep || !aligned(x, 16) || !aligned(idx, 4) ||
+                !aligned(gate, 4)))
+    return ACE_ERR_INVALID_ARG;
+  const ace_layer& L = *layer;
+  const int num_sms = device_sm_count();
+  const FwdLayout ly = fwd_layout(L, T, num_sms);
+  if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ACE_CK(launch_clear_words(at<void>(ws, ly.status), 64, s));
+  if (T == 0) return ACE_OK;
+  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, false, s);
+  if (st != ACE_OK) return st;
+  const size_t tk = (size_t)T * L.k, row = (size_t)L.d * esize(L.dtype);
+  if (L.dtype == ACE_BF16)  // bf16(x) is the first of the router operand's three terms
+    ACE_CK(cudaMemcpy2DAsync(x, row, at<void>(ws, ly.xs3), 3 * row, row, (size_t)T,
+                             cudaMemcpyDeviceToDevice, s));
+  else
+    ACE_CK(cudaMemcpyAsync(x, at<void>(ws, ly.x), (size_t)T * row, cudaMemcpyDeviceToDevice, s));
+  ACE_CK(cudaMemcpyAsync(idx, at<void>(ws, ly.idx), tk * 4, cudaMemcpyDeviceToDevice, s));
+  ACE_CK(cudaMemcpyAsync(gate, at<void>(ws, ly.gate), tk * 4, cudaMemcpyDeviceToDevice, s));
+  ACE_CK(cudaMemcpyAsync(keep, at<void>(ws, ly.keep), tk, cudaMemcpyDeviceToDevice, s));
   return ACE_OK;
 }
 

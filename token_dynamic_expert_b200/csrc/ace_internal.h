@@ -108,6 +108,7 @@ size_t tau_workspace_size();
 cudaError_t launch_tau_quantile(const float* score, int n_tok, int k, long long n_skip,
                                 float* tau, void* ws, int num_sms, cudaStream_t s);
 cudaError_t launch_combine(ace_dtype dt, int T, int k, int d, const int32_t* slot_of,
-                           const float* yslot, void* y, cudaStream_t s);
+                           const float* yslot, int n_rows, void* y, uint32_t* status,
+                           cudaStream_t s);
 
 }  // namespace ace
