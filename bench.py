@@ -39,10 +39,8 @@ METRIC = "MoE-layer tokens/s (prefill, decode) at skip rate; % of tensor/HBM roo
 # capture of that kernel on that workload; reported only while the kernel's source
 # is the revision the counters were taken on.
 PROFILED_TRAFFIC = {
-    ("prefill_1024", "gateup"): ("token_dynamic_expert_b200/csrc/experts_sm100.cu", "06d17ea9eed8",
-                                 825441792),
     ("prefill_1024", "fused"): ("token_dynamic_expert_b200/csrc/experts_fused_sm100.cu",
-                                "f2148741ed71", 1228692480),
+                                "179ca8325236", 1229559016),
 }
 
 
