@@ -5,7 +5,7 @@
 // kept a slot of e (a token routes to an expert at most once), its
 // population count, and (its last CTA, compact.cuh) the base position of
 // each (chunk, expert) run.  Here, one CTA per group of 4 tokens:
-//   position of slot (t, i) of expert e = base[c][e] + popcount(bitmap[c][e]
+//   position of slot (t, i) of expert e = base[e][c] + popcount(bitmap[c][e]
 //   below t); the slot tables are written and x_t is copied into row
 //   `position` of the gathered matrix Xp.
 // No result depends on the order atomics resolve in.
@@ -42,7 +42,8 @@ __global__ void __launch_bounds__(256) k_scatter_gather(
           raise_flag(status, ACE_FLAG_BAD_INDEX);
         } else {
           const uint32_t bits = bitmap[(size_t)c * E + e];
-          pos = base[(size_t)c * E + e] + __popc(bits & ((1u << tl) - 1u));
+          pos = base[(size_t)e * ((Tn + kChunk - 1) / kChunk) + c] +
+                __popc(bits & ((1u << tl) - 1u));
           if (pos >= cap) {
             raise_flag(status, ACE_FLAG_OVERFLOW);
             pos = -1;

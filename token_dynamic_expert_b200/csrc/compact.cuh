@@ -74,7 +74,7 @@ __device__ __forceinline__ void scan_experts(const int32_t* hist, int nchunk, in
   // pass 1: per-expert counts
   for (int eb = warp; eb < E; eb += kEpw * nw) {
     int acc[kEpw] = {0, 0, 0, 0};
-#pragma unroll 2
+#pragma unroll 8
     for (int c = lane; c < nchunk; c += 32)
 #pragma unroll
       for (int j = 0; j < kEpw; ++j) {
@@ -113,20 +113,36 @@ __device__ __forceinline__ void scan_experts(const int32_t* hist, int nchunk, in
   if (o.tile_done)
     for (int i = t; i < o.max_tiles; i += blockDim.x) o.tile_done[i] = 0u;
   __syncthreads();
-  // pass 2: base[c][e] = offset of e + kept slots of e in chunks before c
+  // pass 2: base[e][c] = offset of e + kept slots of e in chunks before c
+  // (expert-major, so a warp's stores over consecutive chunks coalesce).  The
+  // loads of kGroups 32-chunk groups go out together before their scans: one
+  // CTA runs this, so its time is round trips to L2, not bandwidth.
+  constexpr int kGroups = 8;
   for (int eb = warp; eb < E; eb += kEpw * nw) {
     int carry[kEpw];
 #pragma unroll
     for (int j = 0; j < kEpw; ++j) carry[j] = eb + j * nw < E ? s_off[eb + j * nw] : 0;
-    for (int c0 = 0; c0 < nchunk; c0 += 32) {
-      const int c = c0 + lane;
+    for (int c0 = 0; c0 < nchunk; c0 += 32 * kGroups) {
+      int v[kEpw][kGroups];
 #pragma unroll
       for (int j = 0; j < kEpw; ++j) {
         const int e = eb + j * nw;
-        const int v = (e < E && c < nchunk) ? __ldcg(hist + (size_t)e * nchunk + c) : 0;
-        const int incl = warp_incl_scan(v, lane);
-        if (e < E && c < nchunk) o.base[(size_t)c * E + e] = carry[j] + incl - v;
-        carry[j] += __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g) {
+          const int c = c0 + g * 32 + lane;
+          v[j][g] = (e < E && c < nchunk) ? __ldcg(hist + (size_t)e * nchunk + c) : 0;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kEpw; ++j) {
+        const int e = eb + j * nw;
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g) {
+          const int c = c0 + g * 32 + lane;
+          const int incl = warp_incl_scan(v[j][g], lane);
+          if (e < E && c < nchunk) o.base[(size_t)e * nchunk + c] = carry[j] + incl - v[j][g];
+          carry[j] += __shfl_sync(0xffffffffu, incl, 31);
+        }
       }
     }
   }
