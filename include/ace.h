@@ -64,7 +64,9 @@ typedef enum {
   ACE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed         */
   ACE_ERR_UNSUPPORTED = 4,  /* valid but not implemented (shape, dtype)     */
   ACE_ERR_DEVICE_FAULT = 5, /* a kernel flagged an out-of-range index       */
-  ACE_ERR_TIMEOUT = 6       /* a kernel's bounded wait ran out              */
+  ACE_ERR_TIMEOUT = 6,      /* a kernel's bounded wait ran out              */
+  ACE_ERR_IO = 7            /* a tables file could not be written or read,
+                               or is not an intact tables file              */
 } ace_status;
 
 /* device status bits (ace_read_status) */
@@ -379,6 +381,32 @@ ACE_API ace_status ace_build_tables(const ace_layer* layers, int n_layers,
                             const ace_table_opts* opts, float* a_gsp,
                             float* a_rcr, float* amax, float* sigma, void* ws,
                             size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Tables files: ace_build_tables's outputs kept on disk, so a table build
+ *   (which depends only on the frozen weights, [ACE] "Practical
+ *   Implications") is done once and reloaded.  Host pointers, fp32:
+ *   a_gsp, a_rcr, amax [n_layers][E]; sigma [n_layers][E][3] or NULL.
+ *   Format: a 32-byte header (magic "ACETBL\0\x01", version 1, n_layers,
+ *   E, flags bit 0 = sigma present, FNV-1a 64 hash of the payload), then
+ *   the arrays in that order, little-endian.
+ *
+ * ace_tables_save -- writes the file under path + ".tmp" and renames it
+ *   into place (a crash never leaves a torn file).  ACE_ERR_IO when the
+ *   file cannot be written.
+ * ace_tables_info -- the file's n_layers, E and whether it holds sigma (any
+ *   output pointer may be NULL).  ACE_ERR_IO for a missing, truncated,
+ *   corrupted (hash mismatch) or foreign file.
+ * ace_tables_load -- reads a file of exactly n_layers x E into the arrays;
+ *   ACE_ERR_INVALID_ARG when the shape differs or sigma is asked for and
+ *   absent, ACE_ERR_IO as for ace_tables_info.  Nothing is written to the
+ *   arrays unless the whole file checks out.
+ * ---------------------------------------------------------------------- */
+ACE_API ace_status ace_tables_save(const char* path, int n_layers, int E, const float* a_gsp,
+                                   const float* a_rcr, const float* amax, const float* sigma);
+ACE_API ace_status ace_tables_info(const char* path, int* n_layers, int* E, int* has_sigma);
+ACE_API ace_status ace_tables_load(const char* path, int n_layers, int E, float* a_gsp,
+                                   float* a_rcr, float* amax, float* sigma);
 
 /* ------------------------------------------------------------------------
  * ace_tau_workspace_size -- bytes of workspace ace_tau_quantile needs

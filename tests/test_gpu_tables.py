@@ -129,3 +129,34 @@ def test_full_size_layer_tables():
     sig = oracle.sigma_factors(cpu["gamma"], cpu["wg"][sample], cpu["wu"][sample],
                                cpu["wd"][sample], iters=200)
     assert _rel(got["sigma"][0][sample], sig) < RTOL
+
+
+def test_tables_file_round_trip_drives_the_same_forward(tmp_path):
+    """Tables built on the GPU, written to a tables file and read back, give
+    the same bits and the same forward output as the tables in memory."""
+    from token_dynamic_expert_b200 import ace
+    w = W("t_io", T=64, d=256, E=16, m=256, k=4, dtype="bf16", bias=False, skip=0.5,
+          skip_of="slots")
+    lc = workloads.make_layer(w, seed=11)
+    g = {kk: (v.to("cuda").contiguous() if torch.is_tensor(v) else v) for kk, v in lc.items()}
+    s = ace.make_layer(g["gamma"], g["wr"], g["wg"], g["wu"], g["wd"], w.k)
+    t = {n: torch.empty(1, w.E, device="cuda") for n in ("a_gsp", "a_rcr", "amax")}
+    sig = torch.empty(1, w.E, 3, device="cuda")
+    tws = ace.alloc_workspace(ace.ace_tables_workspace_size(s))
+    ace.ace_build_tables([s], t["a_gsp"], t["a_rcr"], t["amax"], tws, sigma=sig)
+    assert ace.ace_read_status(tws) == (ace.ACE_OK, 0)
+    p = str(tmp_path / "layer.acetbl")
+    ace.ace_tables_save(p, t["a_gsp"], t["a_rcr"], t["amax"], sig)
+    a_gsp, a_rcr, amax, sig2 = ace.ace_tables_load(p, device="cuda", with_sigma=True)
+    assert torch.equal(amax, t["amax"]) and torch.equal(sig2, sig)
+    assert torch.equal(a_gsp, t["a_gsp"]) and torch.equal(a_rcr, t["a_rcr"])
+    u = workloads.make_tokens(w, token_seed=12, device="cuda")
+    ys = []
+    for am in (t["amax"][0].contiguous(), amax[0].contiguous()):
+        L = ace.make_layer(g["gamma"], g["wr"], g["wg"], g["wu"], g["wd"], w.k, amax=am)
+        ws = ace.alloc_workspace(ace.ace_workspace_size(L, w.T))
+        y = torch.empty_like(u)
+        ace.ace_moe_forward(L, u, 0.1, y, ws)
+        assert ace.ace_read_status(ws) == (ace.ACE_OK, 0)
+        ys.append(y)
+    assert torch.equal(ys[0], ys[1])

@@ -20,7 +20,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 # ------------------------------------------------------------------ C types
 ACE_OK, ACE_ERR_INVALID_ARG, ACE_ERR_WORKSPACE, ACE_ERR_CUDA, ACE_ERR_UNSUPPORTED, \
-    ACE_ERR_DEVICE_FAULT, ACE_ERR_TIMEOUT = range(7)
+    ACE_ERR_DEVICE_FAULT, ACE_ERR_TIMEOUT, ACE_ERR_IO = range(8)
 ACE_BF16, ACE_F32 = 0, 1
 ACE_GSP_FRO, ACE_GSP_SPECTRAL = 0, 1
 ACE_FUSE_MAX, ACE_FUSE_MIN, ACE_FUSE_MEAN, ACE_FUSE_GSP, ACE_FUSE_RCR = 0, 1, 2, 3, 4
@@ -75,6 +75,13 @@ _lib.ace_moe_experts.restype = ctypes.c_int
 _lib.ace_moe_combine.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp,
                                  ctypes.c_int, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.ace_moe_combine.restype = ctypes.c_int
+_lib.ace_tables_save.argtypes = [ctypes.c_char_p, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp]
+_lib.ace_tables_save.restype = ctypes.c_int
+_lib.ace_tables_info.argtypes = [ctypes.c_char_p, _P(ctypes.c_int), _P(ctypes.c_int),
+                                 _P(ctypes.c_int)]
+_lib.ace_tables_info.restype = ctypes.c_int
+_lib.ace_tables_load.argtypes = [ctypes.c_char_p, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp]
+_lib.ace_tables_load.restype = ctypes.c_int
 _lib.ace_moe_decode_noalloc.argtypes = [_P(ace_layer), _vp, ctypes.c_int, _P(ace_fwd_opts), _vp,
                                         _vp]
 _lib.ace_moe_decode_noalloc.restype = ctypes.c_int
@@ -246,6 +253,40 @@ def ace_moe_combine(slot_of, yslot, y, ws, stream=None):
                                 _stream(stream))
     _check(code, "ace_moe_combine")
     return y
+
+
+def _host_f32(t):
+    return t.detach().to("cpu", torch.float32).contiguous()
+
+
+def ace_tables_save(path, a_gsp, a_rcr, amax, sigma=None):
+    """Write ace_build_tables's outputs ([L][E] each, sigma [L][E][3] or None;
+    any device) to a tables file (see include/ace.h)."""
+    g, r, mx = (_host_f32(t).reshape(-1, a_gsp.shape[-1]) for t in (a_gsp, a_rcr, amax))
+    L, E = g.shape
+    sg = None if sigma is None else _host_f32(sigma)
+    code = _lib.ace_tables_save(os.fsencode(path), L, E, _ptr(g), _ptr(r), _ptr(mx), _ptr(sg))
+    _check(code, "ace_tables_save")
+
+
+def ace_tables_info(path):
+    """(n_layers, E, has_sigma) of a tables file."""
+    L, E, hs = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    code = _lib.ace_tables_info(os.fsencode(path), ctypes.byref(L), ctypes.byref(E),
+                                ctypes.byref(hs))
+    _check(code, "ace_tables_info")
+    return L.value, E.value, bool(hs.value)
+
+
+def ace_tables_load(path, device="cpu", with_sigma=False):
+    """(a_gsp, a_rcr, amax[, sigma]) from a tables file, fp32 on `device`."""
+    L, E, hs = ace_tables_info(path)
+    g, r, mx = (torch.empty(L, E, dtype=torch.float32) for _ in range(3))
+    sg = torch.empty(L, E, 3, dtype=torch.float32) if with_sigma else None
+    code = _lib.ace_tables_load(os.fsencode(path), L, E, _ptr(g), _ptr(r), _ptr(mx), _ptr(sg))
+    _check(code, "ace_tables_load")
+    out = tuple(t.to(device) for t in (g, r, mx))
+    return out + ((sg.to(device),) if with_sigma else ())
 
 
 def ace_moe_decode_noalloc(layer, u, tau, y, renorm=True, eps_rms=1e-6, stream=None,

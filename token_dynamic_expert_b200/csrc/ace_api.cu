@@ -514,6 +514,7 @@ const char* ace_status_str(ace_status s) {
     case ACE_ERR_UNSUPPORTED: return "ACE_ERR_UNSUPPORTED";
     case ACE_ERR_DEVICE_FAULT: return "ACE_ERR_DEVICE_FAULT";
     case ACE_ERR_TIMEOUT: return "ACE_ERR_TIMEOUT";
+    case ACE_ERR_IO: return "ACE_ERR_IO";
   }
   return "ACE_UNKNOWN_STATUS";
 }
