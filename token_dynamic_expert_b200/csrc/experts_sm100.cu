@@ -20,6 +20,9 @@
 // MODE 1, dealt round-robin to one persistent CTA per SM; the small items
 // keep the last wave short.
 //
+// The gate/up launch runs on CTA pairs (tcgen05.mma.cta_group::2, see
+// k_experts_pair below); the down launch on single CTAs.
+//
 // Warp roles (6 warps):
 //   warp 0      TMA producer: weight rows (128 x 64 bf16 per stage) and the
 //               tile's slot rows (32-row boxes, only as many as it needs),
@@ -281,6 +284,310 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------- two-SM (CTA pair) form
+// The same grouped GEMMs with tcgen05.mma.cta_group::2: a cluster of two
+// CTAs on two SMs works on one item with M = 256.  CTA r of the pair holds
+// 128 of the A rows (MODE 0: 64 gate + 64 up rows of its 64 intermediate
+// columns; MODE 1: 128 rows of W^down) and half of the tile's slot rows
+// (B rows r * N/2 .. (r + 1) * N/2 - 1), and accumulates its 128 rows x N
+// slots in its own TMEM.  Each slot-row byte a CTA loads now feeds a
+// 256-row MMA, so a stage holds 2/3 of the bytes of the one-SM form for the
+// same MMA work on each SM, and the accumulators stay double-buffered.
+//   * Both CTAs' TMA loads of a stage complete on the leader's (rank 0)
+//     full barrier; the leader's producer arms it for the bytes of both.
+//   * The leader's MMA thread issues the 256-row MMAs and commits, to both
+//     CTAs at once (multicast), the release of a stage and the readiness of
+//     an accumulator.
+//   * Each CTA's epilogue reads its own TMEM and arrives on the leader's
+//     accumulator-empty barrier.
+// Every wait is bounded.  The CTAs of a pair always meet at the closing
+// cluster barrier (no early exit), after which they free their TMEM
+// together.  No TMA multicast.
+constexpr uint32_t kPeerMask = 0xFEFFFFFFu;  // the leader's copy of a barrier address
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* m, int x,
+                                                 int y, uint32_t leader_bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(leader_bar), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` in both CTAs of the pair once every tcgen05 operation this
+// thread issued has completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  const uint16_t mask = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void arrive_on_leader(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   smem_u32(bar) & kPeerMask)
+               : "memory");
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_experts_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                   const __grid_constant__ CUtensorMap tmB, const int4* __restrict__ tiles,
+                   const int32_t* __restrict__ n_tiles_ptr, int max_tiles, int rows_per_expert,
+                   int K, int items_per_tile, int out_rows, void* __restrict__ out, int out_ld,
+                   const float* __restrict__ slot_gate, uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  float* xchg = reinterpret_cast<float*>(smem + kStageBudget);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStageBudget + kXchgBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kMaxStages;
+  uint64_t* tfull = bars + 2 * kMaxStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* s_maxn = reinterpret_cast<int*>(tmem_holder + 2);
+
+  const int warp = (int)warp_id(), lane = (int)lane_id();
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  int n_tiles = *n_tiles_ptr;
+  if (n_tiles > max_tiles || n_tiles < 0) {
+    if (threadIdx.x == 0) raise_flag(status, ACE_FLAG_BAD_INDEX);
+    n_tiles = n_tiles < 0 ? 0 : max_tiles;
+  }
+  const int total = n_tiles * items_per_tile;
+  const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+  const int ksteps = K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kMaxStages; ++s) {
+      mbar_init(&full[s], 1);   // the leader's producer arms it; both CTAs' bytes land on it
+      mbar_init(&empty[s], 1);  // one multicast commit per release
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * 128);  // both CTAs' epilogue threads (the leader's copy counts)
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *s_maxn = 1;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA0);
+    if (MODE == 0) tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {  // the same warp in both CTAs
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  {
+    int mx = 1;
+    for (int i = threadIdx.x; i < n_tiles; i += blockDim.x) mx = max(mx, tiles[i].z);
+    atomicMax(s_maxn, mx);
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers exist before either signals the other
+  tc_fence_after();
+  // stage: this CTA's 128 A rows, then its half of the slot rows (the same
+  // offsets in both CTAs: the MMA reads both halves at them)
+  const int maxhalf = ((min(*s_maxn, kTileN) + 15) & ~15) / 2;
+  const int maxbox = (maxhalf + kBoxN - 1) / kBoxN;
+  const int stage_bytes = kAStage + maxbox * kBoxBytes;
+  int NS = kStageBudget / stage_bytes;
+  NS = NS > kMaxStages ? kMaxStages : NS;
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int w = pair; w < total && !*abort_flag; w += npairs) {
+        const int ti = w / items_per_tile, it = w - ti * items_per_tile;
+        const int4 tl = tiles[ti];
+        const int half = ((tl.z + 15) & ~15) / 2;
+        const int nbox = (half + kBoxN - 1) / kBoxN;
+        const int brow = tl.y + (int)rank * half;
+        for (int kb = 0; kb < ksteps; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, status, abort_flag)) break;
+          uint8_t* sa = smem + stage * stage_bytes;
+          uint8_t* sb = sa + kAStage;
+          if (leader) mbar_expect_tx(&full[stage], 2u * (uint32_t)(kAStage + nbox * kBoxBytes));
+          const uint32_t lbar = smem_u32(&full[stage]) & kPeerMask;
+          if (MODE == 0) {  // 64 gate rows over 64 up rows of this CTA's 64 columns
+            const int r = tl.x * rows_per_expert + it * 128 + (int)rank * 64;
+            tma_load_2d_pair(sa, &tmA0, kb * kBK, r, lbar, pol_w);
+            tma_load_2d_pair(sa + kAStage / 2, &tmA1, kb * kBK, r, lbar, pol_w);
+          } else {
+            tma_load_2d_pair(sa, &tmA0, kb * kBK,
+                             tl.x * rows_per_expert + it * 256 + (int)rank * kBM, lbar, pol_w);
+          }
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d_pair(sb + b * kBoxBytes, &tmB, kb * kBK, brow + b * kBoxN, lbar, pol_x);
+          if (++stage == NS) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer (leader)
+    if (leader && lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int w = pair; w < total && ok; w += npairs) {
+        const int4 tl = tiles[w / items_per_tile];
+        const int npad = (tl.z + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_f32(2 * kBM, npad);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem + (uint32_t)acc * 256u;
+        for (int kb = 0; kb < ksteps; ++kb) {
+          if (!mbar_wait(&full[stage], phase, status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * stage_bytes);
+          const uint32_t b0 = a0 + kAStage;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_bf16_pair(d0, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32),
+                          idesc, (kb | kk) != 0);
+          mma_commit_pair(&empty[stage]);
+          if (++stage == NS) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // every MMA this thread issued has completed before TMEM is released
+      asm volatile(
+          "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+              smem_u32(drain))
+          : "memory");
+      mbar_drain(drain, 0);
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int xb = 0;
+    for (int w = pair; w < total; w += npairs) {
+      const int ti = w / items_per_tile, it = w - ti * items_per_tile;
+      const int4 tl = tiles[ti];
+      const int row0 = tl.y, n = tl.z;
+      if (!mbar_wait(&tfull[acc], acc_phase, status, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * 256u;
+      if (MODE == 0) {
+        const bool is_gate = q < 2;
+        const int r = (q & 1) * 32 + lane;
+        const int col = it * 128 + (int)rank * 64 + r;
+        __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(out);
+        for (int c0 = 0; c0 < n; c0 += 16) {
+          float v[16];
+          tmem_ld16(tbase + (uint32_t)c0, v);
+          tmem_ld_wait();
+          float* xg = xchg + xb * 1024;
+          float* xu = xg + 512;
+          float4* mine = reinterpret_cast<float4*>((is_gate ? xg : xu) + r * 8);
+          const int off = is_gate ? 8 : 0;
+          mine[0] = make_float4(v[off + 0], v[off + 1], v[off + 2], v[off + 3]);
+          mine[1] = make_float4(v[off + 4], v[off + 5], v[off + 6], v[off + 7]);
+          epilogue_bar();
+          const float4* other = reinterpret_cast<const float4*>((is_gate ? xu : xg) + r * 8);
+          const float4 o0 = other[0], o1 = other[1];
+          const float ov[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+          const int base = is_gate ? c0 : c0 + 8;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float g = is_gate ? v[c] : ov[c];
+            const float u = is_gate ? ov[c] : v[8 + c];
+            if (base + c < n)
+              H[(size_t)(row0 + base + c) * out_ld + col] = __float2bfloat16_rn(silu(g) * u);
+          }
+          xb ^= 1;
+        }
+      } else {
+        const int col = it * 256 + (int)rank * kBM + q * 32 + lane;
+        float* Y = reinterpret_cast<float*>(out);
+        for (int c0 = 0; c0 < n; c0 += 16) {
+          float v[16];
+          tmem_ld16(tbase + (uint32_t)c0, v);
+          tmem_ld_wait();
+          if (col < out_rows) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              if (c0 + c < n) {
+                const int slot = row0 + c0 + c;
+                Y[(size_t)slot * out_ld + col] = slot_gate[slot] * v[c];
+              }
+          }
+        }
+      }
+      tc_fence_before();
+      arrive_on_leader(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+  __syncthreads();
+  if (*abort_flag) {
+    // a wait ran out somewhere: copies this CTA started may still be landing
+    // (their completion counts on the leader's barriers), so give them time
+    if (threadIdx.x == 0) {
+      const uint64_t t0 = global_ns();
+      while (global_ns() - t0 < 100000ull) {
+      }
+    }
+    __syncthreads();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs are done with TMEM and with each other's barriers
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
 // ----------------------------------------------------------- tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -324,6 +631,36 @@ cudaError_t set_smem_attr() {
   return e;
 }
 
+template <int MODE>
+cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                        const int4* tiles, const int32_t* n_tiles, int max_tiles,
+                        int rows_per_expert, int K, int items_per_tile, int out_rows, void* out,
+                        int out_ld, const float* slot_gate, uint32_t* status, int num_sms,
+                        cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_experts_pair<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(num_sms & ~1));  // whole pairs
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_experts_pair<MODE>, a0, a1, b, tiles, n_tiles, max_tiles,
+                            rows_per_expert, K, items_per_tile, out_rows, out, out_ld, slot_gate,
+                            status);
+}
+
 }  // namespace
 
 cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* xp, void* h,
@@ -337,15 +674,18 @@ cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* 
       !make_map(&md, L.w_down, E * d, m, kBM) || !make_map(&mh, h, (uint64_t)cap_slots, m, kBoxN))
     return cudaErrorInvalidValue;
   cudaError_t e;
-  if ((e = set_smem_attr<0>()) != cudaSuccess) return e;
-  if ((e = set_smem_attr<1>()) != cudaSuccess) return e;
-  const int grid = num_sms;
-  k_experts<0><<<grid, kThreads, kSmemBytes, s>>>(mg, mu, mx, tiles, n_tiles, max_tiles, L.m, L.d,
-                                                 L.m / 64, h, L.m, slot_gate, status);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // gate/up on CTA pairs: items of 128 intermediate columns (m % 128 == 0
+  // for bf16 layers).  Down stays on single CTAs: its epilogue (fp32 slot
+  // rows) is heavier and the pair form measured slower there (0.193 vs
+  // 0.209 ms at 4096 tokens, 0% skip), while gate/up gained a little
+  // (0.301 vs 0.296 ms).
+  if ((e = launch_pair<0>(mg, mu, mx, tiles, n_tiles, max_tiles, L.m, L.d, L.m / 128, L.m, h,
+                          L.m, slot_gate, status, num_sms, s)) != cudaSuccess)
+    return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
-  k_experts<1><<<grid, kThreads, kSmemBytes, s>>>(md, md, mh, tiles, n_tiles, max_tiles, L.d, L.m,
-                                                 L.d / kBM, yslot, L.d, slot_gate, status);
+  if ((e = set_smem_attr<1>()) != cudaSuccess) return e;
+  k_experts<1><<<num_sms, kThreads, kSmemBytes, s>>>(md, md, mh, tiles, n_tiles, max_tiles, L.d,
+                                                     L.m, L.d / kBM, yslot, L.d, slot_gate, status);
   return cudaGetLastError();
 }
 
