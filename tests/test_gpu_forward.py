@@ -79,7 +79,7 @@ def test_bf16_small_layers_oracle_tables(w):
 
 def test_bf16_expert_with_several_slot_tiles():
     """8 experts, top-2, 1100 tokens: ~275 slots per expert, so every expert
-    spans two 256-slot tiles with a ragged second one."""
+    spans two tiles of ~138 slots."""
     w = W("heavy", T=1100, d=256, E=8, m=128, k=2, dtype="bf16", bias=False, skip=0.1,
           skip_of="slots")
     res, gpu = _check(w, tables="spread")
@@ -176,17 +176,19 @@ def test_forward_on_a_side_stream():
 
 
 # ------------------------------------------------------------ full sizes
-def tile_covering_tokens(gpu, n_out, tile_n=256, seed=0):
-    """Tokens whose outputs cover every expert GEMM tile at both ends: the
-    tokens of the first and last kept slot of each (expert, 256-slot tile),
-    topped up with random tokens to n_out."""
+def tile_covering_tokens(gpu, n_out, stride=64, seed=0):
+    """Tokens whose outputs cover every expert GEMM tile: the tokens of the
+    first and last kept slot of each expert and of every 64th slot between,
+    topped up with random tokens to n_out.  An expert of several tiles has
+    tiles of near-equal size, at least 128 slots each, so each of its tiles
+    holds one of these slots."""
     off = gpu["expert_offsets"]
     st = gpu["slot_token"]
     toks = set()
     for e in range(len(off) - 1):
-        for a in range(off[e], off[e + 1], tile_n):
-            b = min(off[e + 1], a + tile_n) - 1
-            toks.update((int(st[a]), int(st[b])))
+        if off[e + 1] > off[e]:
+            toks.update(int(st[a]) for a in range(off[e], off[e + 1], stride))
+            toks.add(int(st[off[e + 1] - 1]))
     T = gpu["keep"].shape[0]
     rng = np.random.default_rng(seed)
     rest = np.setdiff1d(np.arange(T), np.fromiter(toks, dtype=np.int64))

@@ -64,9 +64,6 @@ FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms) {
   o.status = take(256);
   o.part = take(part * 4);
   o.inv_rms = take(T * 4);
-  // bf16 layers: bf16(x) is the hi block of the router operand xs3
-  o.x = take(L.dtype == ACE_BF16 ? 0 : T * d * es);
-  o.xs3 = take(L.dtype == ACE_BF16 ? T * 3 * d * 2 : 0);
   o.idx = take(cap * 4);
   o.gate = take(cap * 4);
   o.score = take(cap * 4);
@@ -167,18 +164,19 @@ P* at(void* ws, size_t off) {
 constexpr size_t kDoneCtrWord = 32;
 
 // The routing half shared by the forward and the score query; with_scan adds
-// the compaction's expert-offset scan (run by the routing's last CTA).
+// the compaction's expert-offset scan (run by the routing's last CTA).  x_out
+// (nullable) receives x rounded to the storage type.
 ace_status run_routing(const ace_layer& L, const void* u, int T, const ace_fwd_opts& o,
                        const FwdLayout& ly, void* ws, int num_sms, float* logits_dbg,
-                       bool with_scan, cudaStream_t s) {
+                       bool with_scan, void* x_out, cudaStream_t s) {
   const int splitk = router_splits_for(L, T, num_sms);
   const bool tc = L.dtype == ACE_BF16;
-  ACE_CK(launch_rmsnorm(L.dtype, u, T, L.d, L.gamma, o.eps_rms, at<float>(ws, ly.inv_rms),
-                        tc ? nullptr : at<void>(ws, ly.x), tc ? at<void>(ws, ly.xs3) : nullptr,
+  ACE_CK(launch_rmsnorm(L.dtype, u, T, L.d, L.gamma, o.eps_rms, at<float>(ws, ly.inv_rms), x_out,
                         s));
   if (tc)
-    ACE_CK(launch_router_tc(at<void>(ws, ly.xs3), L.w_router, T, L.d, L.E, splitk,
-                            at<float>(ws, ly.part), at<uint32_t>(ws, ly.status), num_sms, s));
+    ACE_CK(launch_router_tc(u, at<float>(ws, ly.inv_rms), L.gamma, L.w_router, T, L.d, L.E,
+                            splitk, at<float>(ws, ly.part), at<uint32_t>(ws, ly.status), num_sms,
+                            s));
   else
     ACE_CK(launch_router_logits(L.dtype, u, at<float>(ws, ly.inv_rms), L.gamma, L.w_router, T,
                                 L.d, L.E, splitk, at<float>(ws, ly.part), s));
@@ -229,15 +227,14 @@ ace_status run_prefill(const ace_layer& L, const void* u, int T, const ace_fwd_o
                        const FwdLayout& ly, void* ws, int num_sms, ace_debug_out* dbg,
                        cudaEvent_t ev_b, cudaEvent_t ev_m, cudaEvent_t ev_e, cudaStream_t s) {
   ace_status st =
-      run_routing(L, u, T, o, ly, ws, num_sms, dbg ? dbg->logits : nullptr, true, s);
+      run_routing(L, u, T, o, ly, ws, num_sms, dbg ? dbg->logits : nullptr, true, nullptr, s);
   if (st != ACE_OK) return st;
-  const bool bf = L.dtype == ACE_BF16;
   ACE_CK(launch_scatter_gather(
       L.dtype, T, L.k, L.E, L.d, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
-      at<uint8_t>(ws, ly.keep), at<uint32_t>(ws, ly.bitmap), at<int32_t>(ws, ly.base),
-      bf ? at<void>(ws, ly.xs3) : at<void>(ws, ly.x), (size_t)L.d * (bf ? 3 : 1),
-      at<int32_t>(ws, ly.slot_token), at<int32_t>(ws, ly.slot_rank), at<float>(ws, ly.slot_gate),
-      at<int32_t>(ws, ly.slot_of), at<void>(ws, ly.xp), at<uint32_t>(ws, ly.status), s));
+      at<uint8_t>(ws, ly.keep), at<uint32_t>(ws, ly.bitmap), at<int32_t>(ws, ly.base), u,
+      at<float>(ws, ly.inv_rms), L.gamma, at<int32_t>(ws, ly.slot_token),
+      at<int32_t>(ws, ly.slot_rank), at<float>(ws, ly.slot_gate), at<int32_t>(ws, ly.slot_of),
+      at<void>(ws, ly.xp), at<uint32_t>(ws, ly.status), s));
   if (ev_b) ACE_CK(cudaEventRecord(ev_b, s));
   if (L.dtype == ACE_BF16 && fused_experts(L, T)) {
     // one launch for both expert GEMMs; "mid" is recorded after it as well
@@ -442,7 +439,7 @@ ace_status ace_moe_scores(const ace_layer* layer, const void* u, int T, const ac
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ACE_CK(launch_clear_words(at<void>(ws, ly.status), 64, s));
   if (T == 0) return ACE_OK;
-  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, false, s);
+  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, false, nullptr, s);
   if (st != ACE_OK) return st;
   const size_t tk = (size_t)T * L.k;
   ACE_CK(cudaMemcpyAsync(score, at<void>(ws, ly.score), tk * 4, cudaMemcpyDeviceToDevice, s));
@@ -466,14 +463,9 @@ ace_status ace_moe_route(const ace_layer* layer, const void* u, int T, const ace
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ACE_CK(launch_clear_words(at<void>(ws, ly.status), 64, s));
   if (T == 0) return ACE_OK;
-  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, false, s);
+  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, false, x, s);
   if (st != ACE_OK) return st;
-  const size_t tk = (size_t)T * L.k, row = (size_t)L.d * esize(L.dtype);
-  if (L.dtype == ACE_BF16)  // bf16(x) is the first of the router operand's three terms
-    ACE_CK(cudaMemcpy2DAsync(x, row, at<void>(ws, ly.xs3), 3 * row, row, (size_t)T,
-                             cudaMemcpyDeviceToDevice, s));
-  else
-    ACE_CK(cudaMemcpyAsync(x, at<void>(ws, ly.x), (size_t)T * row, cudaMemcpyDeviceToDevice, s));
+  const size_t tk = (size_t)T * L.k;
   ACE_CK(cudaMemcpyAsync(idx, at<void>(ws, ly.idx), tk * 4, cudaMemcpyDeviceToDevice, s));
   ACE_CK(cudaMemcpyAsync(gate, at<void>(ws, ly.gate), tk * 4, cudaMemcpyDeviceToDevice, s));
   ACE_CK(cudaMemcpyAsync(keep, at<void>(ws, ly.keep), tk, cudaMemcpyDeviceToDevice, s));

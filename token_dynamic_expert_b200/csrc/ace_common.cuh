@@ -243,6 +243,13 @@ __device__ __forceinline__ float fused_factor(const FuseTables& f, int e) {
   }
 }
 
+// The normalised, scaled input element x = (u * (1/rms)) * gamma in fp32,
+// each product rounded (no contraction into an FMA): every kernel that forms
+// x from u uses this, so they all hold the same bits.
+__device__ __forceinline__ float xhat(float u, float inv_rms, float gamma) {
+  return __fmul_rn(__fmul_rn(u, inv_rms), gamma);
+}
+
 // ---------------------------------------------------------------- top-k
 // order-preserving map of a float to an unsigned key (larger float, larger key)
 __device__ __forceinline__ uint32_t fkey(float f) {
@@ -290,6 +297,67 @@ __device__ __forceinline__ void topk_select(const float (&v)[NV], int nq, int E,
     if ((sel_e >> 5) == q) mine = x;
   }
   sel_v = mine;
+}
+
+// inverse of fkey: the float whose key is k
+__device__ __forceinline__ float fkey_inv(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// The same selection as topk_select (same ranks, same tie rule: the lower
+// expert index wins) for a compile-time count NV of logits per lane, in fewer
+// instructions.  Each lane packs its candidates as (key << 32 | ~expert), so
+// that one unsigned compare orders them by logit and then by lower index, and
+// sorts them once, largest first, with Batcher's odd-even merge network
+// (19 compare-exchanges for NV = 8).  Each of the k rounds then looks only at
+// the lanes' list heads: the largest key by redux.max, the smallest expert
+// index among the heads that carry it by redux.max of ~expert, and the owner
+// lane pops its head.  Experts e >= E carry the packed value 0, below every
+// real candidate.  The selected logit comes back exactly from its key.
+template <int NV>
+__device__ __forceinline__ void topk_sorted(const float (&v)[NV], int E, int k, int lane,
+                                            int& sel_e, float& sel_v, uint32_t* status) {
+  uint64_t c[NV];
+#pragma unroll
+  for (int q = 0; q < NV; ++q) {
+    const int e = lane + 32 * q;
+    c[q] = e < E ? ((uint64_t)fkey(v[q]) << 32) | (uint64_t)(~(uint32_t)e) : 0ull;
+  }
+#pragma unroll
+  for (int p = 1; p < NV; p <<= 1)
+#pragma unroll
+    for (int kk = p; kk >= 1; kk >>= 1)
+#pragma unroll
+      for (int j = kk % p; j + kk < NV; j += 2 * kk)
+#pragma unroll
+        for (int i = 0; i < kk; ++i) {
+          const int a = i + j, b = i + j + kk;
+          if (b < NV && a / (2 * p) == b / (2 * p)) {
+            const uint64_t x = c[a], y = c[b];
+            const bool sw = y > x;
+            c[a] = sw ? y : x;
+            c[b] = sw ? x : y;
+          }
+        }
+  for (int i = 0; i < k; ++i) {
+    const uint32_t hk = (uint32_t)(c[0] >> 32);
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, hk);
+    const uint32_t ne = __reduce_max_sync(0xffffffffu, hk == mk ? (uint32_t)c[0] : 0u);
+    int e_sel = (int)~ne;
+    const bool valid = e_sel >= 0 && e_sel < E;
+    if (!valid) {
+      raise_flag(status, ACE_FLAG_BAD_INDEX);
+      e_sel = 0;
+    }
+    const bool pop = valid && (e_sel & 31) == lane;
+#pragma unroll
+    for (int q = 0; q + 1 < NV; ++q) c[q] = pop ? c[q + 1] : c[q];
+    if (pop) c[NV - 1] = 0ull;
+    if (lane == i) {
+      sel_e = e_sel;
+      sel_v = fkey_inv(mk);
+    }
+  }
 }
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }

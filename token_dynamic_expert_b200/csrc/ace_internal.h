@@ -33,7 +33,7 @@ int router_splits_for(const ace_layer& L, int T, int num_sms);
 // Byte offsets of the forward's scratch arrays inside the caller's
 // workspace.  Everything is sized for max_tokens and no skipping.
 struct FwdLayout {
-  size_t status, part, inv_rms, x, xs3, tile_done, idx, gate, score, keep, bitmap, hist, base, counts,
+  size_t status, part, inv_rms, tile_done, idx, gate, score, keep, bitmap, hist, base, counts,
       offsets, n_kept, tiles, n_tiles, slot_token, slot_rank, slot_gate, slot_of, xp, h,
       yslot, total;
   int max_tokens, part_floats, max_tiles;
@@ -54,12 +54,13 @@ ace_status check_fusion(const ace_layer& L, int fusion);
 
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
-                           float eps, float* inv_rms, void* x, void* xs3, cudaStream_t s);
-// Tensor-core router (bf16 layers): part[split][t][e] from the three-term
-// bf16 split xs3 [T][3d] of the fp32 router input and w_router [E][d].
+                           float eps, float* inv_rms, void* x, cudaStream_t s);
+// Tensor-core router (bf16 layers): part[split][t][e] from u [T][d] (bf16),
+// 1/rms, gamma and w_router [E][d].
 int router_tc_splits(int T, int d, int E, int num_sms);
-cudaError_t launch_router_tc(const void* xs3, const void* wr, int T, int d, int E, int splits,
-                             float* part, uint32_t* status, int num_sms, cudaStream_t s);
+cudaError_t launch_router_tc(const void* u, const float* inv_rms, const float* gamma,
+                             const void* wr, int T, int d, int E, int splits, float* part,
+                             uint32_t* status, int num_sms, cudaStream_t s);
 cudaError_t launch_router_logits(ace_dtype dt, const void* u, const float* inv_rms,
                                  const float* gamma, const void* wr, int T, int d, int E,
                                  int splitk, float* part, cudaStream_t s);
@@ -75,9 +76,10 @@ cudaError_t launch_topk_mask(const float* part, int splitk, int T, int E, int k,
 // elements apart.
 cudaError_t launch_scatter_gather(ace_dtype dt, int T, int k, int E, int d, const int32_t* idx,
                                   const float* gate, const uint8_t* keep, const uint32_t* bitmap,
-                                  const int32_t* base, const void* x, size_t x_stride,
-                                  int32_t* slot_token, int32_t* slot_rank, float* slot_gate,
-                                  int32_t* slot_of, void* xp, uint32_t* status, cudaStream_t s);
+                                  const int32_t* base, const void* u, const float* inv_rms,
+                                  const float* gamma, int32_t* slot_token, int32_t* slot_rank,
+                                  float* slot_gate, int32_t* slot_of, void* xp, uint32_t* status,
+                                  cudaStream_t s);
 cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* xp, void* h,
                                  float* yslot, const int4* tiles, const int32_t* n_tiles,
                                  int max_tiles, const float* slot_gate, uint32_t* status,

@@ -5,9 +5,10 @@
 // kept a slot of e (a token routes to an expert at most once), its
 // population count, and (its last CTA, compact.cuh) the base position of
 // each (chunk, expert) run.  Here, one CTA per group of 4 tokens:
-//   position of slot (t, i) of expert e = base[e][c] + popcount(bitmap[c][e]
-//   below t); the slot tables are written and x_t is copied into row
-//   `position` of the gathered matrix Xp.
+//   position of slot (t, i) of expert e = base[c][e] + popcount(bitmap[c][e]
+//   below t); the slot tables are written and x_t = xhat(u_t, 1/rms_t, gamma),
+//   rounded to the storage type, is formed once per token and written into
+//   row `position` of the gathered matrix Xp for each of its kept slots.
 // No result depends on the order atomics resolve in.
 #include "ace_common.cuh"
 #include "ace_internal.h"
@@ -20,15 +21,15 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_scatter_gather(
     int Tn, int k, int E, int d, const int32_t* __restrict__ idx, const float* __restrict__ gate,
     const uint8_t* __restrict__ keep, const uint32_t* __restrict__ bitmap,
-    const int32_t* __restrict__ base, const T* __restrict__ x, size_t x_stride,
-    int32_t* __restrict__ slot_token, int32_t* __restrict__ slot_rank,
-    float* __restrict__ slot_gate, int32_t* __restrict__ slot_of, T* __restrict__ xp, int cap,
-    uint32_t* status) {
-  __shared__ int s_pos[kScatterTok * kMaxK], s_tok[kScatterTok * kMaxK];
-  __shared__ int s_n;
+    const int32_t* __restrict__ base, const T* __restrict__ u, const float* __restrict__ inv_rms,
+    const float* __restrict__ gamma, int32_t* __restrict__ slot_token,
+    int32_t* __restrict__ slot_rank, float* __restrict__ slot_gate, int32_t* __restrict__ slot_of,
+    T* __restrict__ xp, int cap, uint32_t* status) {
+  __shared__ int s_pos[kScatterTok][kMaxK];
+  __shared__ int s_n[kScatterTok];
   const int t0 = blockIdx.x * kScatterTok;
   const int c = t0 / kChunk;
-  if (threadIdx.x == 0) s_n = 0;
+  if (threadIdx.x < kScatterTok) s_n[threadIdx.x] = 0;
   __syncthreads();
   if ((int)threadIdx.x < kScatterTok * k) {
     const int tq = threadIdx.x / k, i = threadIdx.x - tq * k;
@@ -42,7 +43,7 @@ __global__ void __launch_bounds__(256) k_scatter_gather(
           raise_flag(status, ACE_FLAG_BAD_INDEX);
         } else {
           const uint32_t bits = bitmap[(size_t)c * E + e];
-          pos = base[(size_t)e * ((Tn + kChunk - 1) / kChunk) + c] +
+          pos = base[(size_t)c * E + e] +
                 __popc(bits & ((1u << tl) - 1u));
           if (pos >= cap) {
             raise_flag(status, ACE_FLAG_OVERFLOW);
@@ -51,9 +52,8 @@ __global__ void __launch_bounds__(256) k_scatter_gather(
             slot_token[pos] = t;
             slot_rank[pos] = i;
             slot_gate[pos] = gate[o];
-            const int j = atomicAdd(&s_n, 1);  // copy list: order does not matter
-            s_pos[j] = pos;
-            s_tok[j] = t;
+            const int j = atomicAdd(&s_n[tq], 1);  // copy list: order does not matter
+            s_pos[tq][j] = pos;
           }
         }
       }
@@ -61,26 +61,36 @@ __global__ void __launch_bounds__(256) k_scatter_gather(
     }
   }
   __syncthreads();
-  // Xp[pos] = x[t]: 16-byte vectors, four loads in flight per thread
-  const int n = s_n;
-  const int vpr = d * (int)sizeof(T) / 16;
-  const int total = n * vpr;
+  // Xp[pos] = x_t: one 16-byte vector of u per thread and step (four in
+  // flight), turned into x and stored to each kept slot of the token
+  constexpr int V = 16 / (int)sizeof(T);
+  const int vpr = d / V;
+  const int total = kScatterTok * vpr;
   for (int q0 = threadIdx.x; q0 < total; q0 += 4 * blockDim.x) {
     uint4 v[4];
+    float r[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int q = q0 + u * blockDim.x;
-      if (q < total) {
-        const int j = q / vpr, w = q - j * vpr;
-        v[u] = reinterpret_cast<const uint4*>(x + (size_t)s_tok[j] * x_stride)[w];
+    for (int j = 0; j < 4; ++j) {
+      const int q = q0 + j * blockDim.x;
+      const int tq = q / vpr, w = q - tq * vpr, t = t0 + tq;
+      r[j] = 0.f;
+      if (q < total && t < Tn) {
+        v[j] = reinterpret_cast<const uint4*>(u + (size_t)t * d)[w];
+        r[j] = inv_rms[t];
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int q = q0 + u * blockDim.x;
-      if (q < total) {
-        const int j = q / vpr, w = q - j * vpr;
-        reinterpret_cast<uint4*>(xp + (size_t)s_pos[j] * d)[w] = v[u];
+    for (int j = 0; j < 4; ++j) {
+      const int q = q0 + j * blockDim.x;
+      const int tq = q / vpr, w = q - tq * vpr;
+      if (q < total && t0 + tq < Tn) {
+        const T* e = reinterpret_cast<const T*>(&v[j]);
+        uint4 o;
+        T* oe = reinterpret_cast<T*>(&o);
+#pragma unroll
+        for (int cc = 0; cc < V; ++cc) oe[cc] = from_f<T>(xhat(to_f(e[cc]), r[j], gamma[w * V + cc]));
+        const int n = s_n[tq];
+        for (int i = 0; i < n; ++i) reinterpret_cast<uint4*>(xp + (size_t)s_pos[tq][i] * d)[w] = o;
       }
     }
   }
@@ -88,19 +98,21 @@ __global__ void __launch_bounds__(256) k_scatter_gather(
 
 cudaError_t launch_scatter_gather(ace_dtype dt, int T, int k, int E, int d, const int32_t* idx,
                                   const float* gate, const uint8_t* keep, const uint32_t* bitmap,
-                                  const int32_t* base, const void* x, size_t x_stride,
-                                  int32_t* slot_token, int32_t* slot_rank, float* slot_gate,
-                                  int32_t* slot_of, void* xp, uint32_t* status, cudaStream_t s) {
+                                  const int32_t* base, const void* u, const float* inv_rms,
+                                  const float* gamma, int32_t* slot_token, int32_t* slot_rank,
+                                  float* slot_gate, int32_t* slot_of, void* xp, uint32_t* status,
+                                  cudaStream_t s) {
   dim3 grid(cdiv(T, kScatterTok));
   const int cap = T * k;
   if (dt == ACE_BF16)
     k_scatter_gather<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        T, k, E, d, idx, gate, keep, bitmap, base, (const __nv_bfloat16*)x, x_stride, slot_token,
-        slot_rank, slot_gate, slot_of, (__nv_bfloat16*)xp, cap, status);
+        T, k, E, d, idx, gate, keep, bitmap, base, (const __nv_bfloat16*)u, inv_rms, gamma,
+        slot_token, slot_rank, slot_gate, slot_of, (__nv_bfloat16*)xp, cap, status);
   else
     k_scatter_gather<float><<<grid, 256, 0, s>>>(T, k, E, d, idx, gate, keep, bitmap, base,
-                                                 (const float*)x, x_stride, slot_token, slot_rank,
-                                                 slot_gate, slot_of, (float*)xp, cap, status);
+                                                 (const float*)u, inv_rms, gamma, slot_token,
+                                                 slot_rank, slot_gate, slot_of, (float*)xp, cap,
+                                                 status);
   return cudaGetLastError();
 }
 

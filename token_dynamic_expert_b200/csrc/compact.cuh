@@ -51,59 +51,58 @@ struct ScanOut {
 };
 
 // Whole-CTA routine (every thread calls it; blockDim.x a multiple of 32, at
-// least E, at most 1024).  hist is expert-major, [E][nchunk], and read with
-// L2-coherent loads (other CTAs wrote it); base is chunk-major, [nchunk][E].
-// A warp takes four experts at a time: their chunk counts are summed (pass 1)
-// and, once the offsets over experts are known, scanned over the chunks in
-// segments of 32 (pass 2).
-__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += n;
-  }
-  return v;
-}
-
+// least E, at most 1024).  hist and base are chunk-major, [nchunk][E]; hist
+// is read with L2-coherent loads (other CTAs wrote it).
+//
+// The warps split the [nchunk][E] table into 32-expert columns (a lane per
+// expert) times chunk ranges, so that every load and store of a warp covers
+// 32 consecutive experts of one chunk and no step needs a shuffle:
+//   pass 1: each warp sums its range per expert (s_part[range][e]);
+//   then per expert: the count (sum over ranges), the exclusive offsets over
+//   experts (a CTA scan) and the expert's GEMM tiles;
+//   pass 2: each warp walks its range again, writing base[c][e] = offset of
+//   e + kept slots of e in chunks before c.
+// An expert of n kept slots gets ceil(n / tile_n) tiles of near-equal size
+// (they differ by at most one slot), in slot order.
 __device__ __forceinline__ void scan_experts(const int32_t* hist, int nchunk, int E,
                                              const ScanOut& o) {
   __shared__ int s_warp[32];
-  __shared__ int s_cnt[1024], s_off[1024];
+  __shared__ int s_cnt[1024], s_part[1024];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  constexpr int kEpw = 4;  // experts a warp handles at once
-  // pass 1: per-expert counts
-  for (int eb = warp; eb < E; eb += kEpw * nw) {
-    int acc[kEpw] = {0, 0, 0, 0};
+  const int ncol = (E + 31) / 32;              // 32-expert columns
+  const int nrange = nw / ncol;                // chunk ranges (nw >= ncol since E <= 1024)
+  const int per = (nchunk + nrange - 1) / nrange;
+  const int col = warp % ncol, rg = warp / ncol;
+  const int e = col * 32 + lane;
+  const bool active = rg < nrange && e < E;
+  const int c0 = rg * per, c1 = min(nchunk, c0 + per);
+  // pass 1: per-range sums
+  if (active) {
+    int acc = 0;
 #pragma unroll 8
-    for (int c = lane; c < nchunk; c += 32)
-#pragma unroll
-      for (int j = 0; j < kEpw; ++j) {
-        const int e = eb + j * nw;
-        if (e < E) acc[j] += __ldcg(hist + (size_t)e * nchunk + c);
-      }
-#pragma unroll
-    for (int j = 0; j < kEpw; ++j) {
-#pragma unroll
-      for (int sh = 16; sh > 0; sh >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], sh);
-      const int e = eb + j * nw;
-      if (lane == 0 && e < E) s_cnt[e] = acc[j];
-    }
+    for (int c = c0; c < c1; ++c) acc += __ldcg(hist + (size_t)c * E + e);
+    s_part[rg * E + e] = acc;
   }
   __syncthreads();
-  // offsets over experts and the tile list
+  // counts, offsets over experts, the tile list
   const int t = threadIdx.x;
-  const int cnt = t < E ? s_cnt[t] : 0;
+  int cnt = 0;
+  if (t < E)
+    for (int r = 0; r < nrange; ++r) cnt += s_part[r * E + t];
   int total, total_tiles;
   const int off = block_excl_scan(cnt, s_warp, &total);
   const int ntile = t < E ? (cnt + o.tile_n - 1) / o.tile_n : 0;
   const int toff = block_excl_scan(ntile, s_warp, &total_tiles);
   if (t < E) {
-    s_off[t] = off;
+    s_cnt[t] = off;  // from here on: the expert's offset
     o.counts[t] = cnt;
     o.offsets[t] = off;
-    for (int q = 0; q < ntile; ++q)
-      if (toff + q < o.max_tiles)
-        o.tiles[toff + q] = make_int4(t, off + q * o.tile_n, min(o.tile_n, cnt - q * o.tile_n), 0);
+    if (ntile > 0) {
+      const int each = cnt / ntile, rem = cnt - each * ntile;
+      for (int q = 0; q < ntile; ++q)
+        if (toff + q < o.max_tiles)
+          o.tiles[toff + q] = make_int4(t, off + q * each + min(q, rem), each + (q < rem ? 1 : 0), 0);
+    }
   }
   if (t == 0) {
     o.offsets[E] = total;
@@ -113,37 +112,24 @@ __device__ __forceinline__ void scan_experts(const int32_t* hist, int nchunk, in
   if (o.tile_done)
     for (int i = t; i < o.max_tiles; i += blockDim.x) o.tile_done[i] = 0u;
   __syncthreads();
-  // pass 2: base[e][c] = offset of e + kept slots of e in chunks before c
-  // (expert-major, so a warp's stores over consecutive chunks coalesce).  The
-  // loads of kGroups 32-chunk groups go out together before their scans: one
-  // CTA runs this, so its time is round trips to L2, not bandwidth.
-  constexpr int kGroups = 8;
-  for (int eb = warp; eb < E; eb += kEpw * nw) {
-    int carry[kEpw];
+  // pass 2: bases, from the expert's offset and the ranges before this one
+  if (active) {
+    int run = s_cnt[e];
+    for (int r = 0; r < rg; ++r) run += s_part[r * E + e];
+    int c = c0;
+    for (; c + 8 <= c1; c += 8) {
+      int v[8];
 #pragma unroll
-    for (int j = 0; j < kEpw; ++j) carry[j] = eb + j * nw < E ? s_off[eb + j * nw] : 0;
-    for (int c0 = 0; c0 < nchunk; c0 += 32 * kGroups) {
-      int v[kEpw][kGroups];
+      for (int j = 0; j < 8; ++j) v[j] = __ldcg(hist + (size_t)(c + j) * E + e);
 #pragma unroll
-      for (int j = 0; j < kEpw; ++j) {
-        const int e = eb + j * nw;
-#pragma unroll
-        for (int g = 0; g < kGroups; ++g) {
-          const int c = c0 + g * 32 + lane;
-          v[j][g] = (e < E && c < nchunk) ? __ldcg(hist + (size_t)e * nchunk + c) : 0;
-        }
+      for (int j = 0; j < 8; ++j) {
+        o.base[(size_t)(c + j) * E + e] = run;
+        run += v[j];
       }
-#pragma unroll
-      for (int j = 0; j < kEpw; ++j) {
-        const int e = eb + j * nw;
-#pragma unroll
-        for (int g = 0; g < kGroups; ++g) {
-          const int c = c0 + g * 32 + lane;
-          const int incl = warp_incl_scan(v[j][g], lane);
-          if (e < E && c < nchunk) o.base[(size_t)e * nchunk + c] = carry[j] + incl - v[j][g];
-          carry[j] += __shfl_sync(0xffffffffu, incl, 31);
-        }
-      }
+    }
+    for (; c < c1; ++c) {
+      o.base[(size_t)c * E + e] = run;
+      run += __ldcg(hist + (size_t)c * E + e);
     }
   }
 }

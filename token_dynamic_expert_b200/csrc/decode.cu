@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
       float xv[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) xv[c] = f[c] * r * gg[c];
+      for (int c = 0; c < 8; ++c) xv[c] = xhat(f[c], r, gg[c]);
       float4* xo = reinterpret_cast<float4*>(xf + t * d + v * 8);
       xo[0] = make_float4(xv[0], xv[1], xv[2], xv[3]);
       xo[1] = make_float4(xv[4], xv[5], xv[6], xv[7]);

@@ -79,9 +79,12 @@ __global__ void k_tiles_from_offsets(const int32_t* __restrict__ offsets, int E,
   const int ntile = (t < E && !bad) ? (cnt + tile_n - 1) / tile_n : 0;
   int total = 0;
   const int toff = block_excl_scan(ntile, s_warp, &total);
-  for (int q = 0; q < ntile; ++q)
-    if (toff + q < max_tiles)
-      tiles[toff + q] = make_int4(t, off + q * tile_n, min(tile_n, cnt - q * tile_n), 0);
+  if (ntile > 0) {  // near-equal tiles, as the forward's compaction makes them
+    const int each = cnt / ntile, rem = cnt - each * ntile;
+    for (int q = 0; q < ntile; ++q)
+      if (toff + q < max_tiles)
+        tiles[toff + q] = make_int4(t, off + q * each + min(q, rem), each + (q < rem ? 1 : 0), 0);
+  }
   if (t == 0) {
     *n_tiles = min(total, max_tiles);
     if (bad) raise_flag(status, ACE_FLAG_BAD_INDEX);
@@ -123,12 +126,13 @@ ace_status ace_moe_experts(const ace_layer* layer, const void* xp, int S, const 
   int32_t* n_tiles = reinterpret_cast<int32_t*>(w + ly.n_tiles);
   uint32_t* tile_done = reinterpret_cast<uint32_t*>(w + ly.tile_done);
   const int threads = ((L.E + 1 + 31) / 32) * 32;
+  const bool fused = L.dtype == ACE_BF16 && (long long)S < 128LL * L.E;
   k_tiles_from_offsets<<<1, threads > 1024 ? 1024 : threads, 0, s>>>(
       offsets, L.E, S, kTileN, tiles, n_tiles, ly.max_tiles, tile_done, status);
   if (cudaGetLastError() != cudaSuccess) return ACE_ERR_CUDA;
   const int num_sms = device_sm_count();
   cudaError_t e;
-  if (L.dtype == ACE_BF16 && (long long)S < 128LL * L.E) {
+  if (fused) {
     // small tiles: both GEMMs in one launch, as the forward does
     e = launch_experts_fused(L, S, xp, w + ly.h, yslot, tiles, n_tiles, ly.max_tiles, slot_gate,
                              tile_done, status, num_sms, s);

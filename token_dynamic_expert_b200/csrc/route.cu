@@ -1,9 +1,10 @@
 // route.cu -- the online routing half of the ACE MoE forward.
 //
-//   k_rmsnorm        x_t = RMSNorm(u_t) * gamma, the expert input, and 1/rms_t
-//                    (bf16 layers: x as three bf16 terms, the first of which
-//                    is the experts' bf16 input)
-//                    ([ACE] "Theoretical Foundation": x = xbar Gamma_l)
+//   k_rmsnorm        1/rms_t, and (when asked) x_t = RMSNorm(u_t) * gamma
+//                    rounded to the storage type ([ACE] "Theoretical
+//                    Foundation": x = xbar Gamma_l).  The forward's consumers
+//                    (the routers, the row gather) form x from u and 1/rms
+//                    themselves.
 //   k_router_logits  l_{t,e} = x_t . w_e, fp32 CUDA-core GEMM over a K split
 //                    (fp32 layers; bf16 layers use the tensor-core router in
 //                    router_sm100.cu)
@@ -26,17 +27,11 @@ namespace ace {
 
 // ------------------------------------------------------------------ RMSNorm
 // One warp per token, 16-byte loads and stores (d is a multiple of 64).
-// x (nullable) receives x rounded to the storage type.  With xs3 given
-// (bf16 layers), the kernel writes the fp32 router input
-// xhat = u * (1/rms) * gamma as three bf16 terms hi + mid + lo, each the
-// rounding of what the previous terms leave, at xs3[t][0 | d | 2d + i]: the
-// operand of the tensor-core router, whose products with bf16 router rows
-// are then exact in fp32.  The hi term is bf16(x), the experts' input.
+// x (nullable) receives xhat(u, 1/rms, gamma) rounded to the storage type.
 template <typename T>
 __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn, int d,
                                                  const float* __restrict__ gamma, float eps,
-                                                 float* __restrict__ inv_rms, T* __restrict__ x,
-                                                 __nv_bfloat16* __restrict__ xs3) {
+                                                 float* __restrict__ inv_rms, T* __restrict__ x) {
   constexpr int V = 16 / sizeof(T);
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -56,49 +51,27 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn
   ss = warp_sum(ss);
   const float r = 1.0f / sqrtf(ss / (float)d + eps);
   if (lane == 0) inv_rms[t] = r;
+  if (x == nullptr) return;
   uint4* xr = reinterpret_cast<uint4*>(x + (size_t)t * d);
   for (int v = lane; v < nv; v += 32) {
     const uint4 q = ur[v];
     const T* e = reinterpret_cast<const T*>(&q);
     uint4 o;
     T* oe = reinterpret_cast<T*>(&o);
-    float xf[V];
 #pragma unroll
-    for (int c = 0; c < V; ++c) {
-      xf[c] = to_f(e[c]) * r * gamma[v * V + c];
-      oe[c] = from_f<T>(xf[c]);
-    }
-    if (x != nullptr) xr[v] = o;
-    if (xs3 != nullptr && V == 8) {
-      uint4 oh, om, ol;
-      __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(&oh);
-      __nv_bfloat16* mi = reinterpret_cast<__nv_bfloat16*>(&om);
-      __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(&ol);
-#pragma unroll
-      for (int c = 0; c < V; ++c) {
-        h[c] = __float2bfloat16_rn(xf[c]);
-        const float r1 = xf[c] - __bfloat162float(h[c]);
-        mi[c] = __float2bfloat16_rn(r1);
-        lo[c] = __float2bfloat16_rn(r1 - __bfloat162float(mi[c]));
-      }
-      uint4* xs = reinterpret_cast<uint4*>(xs3 + (size_t)t * 3 * d);
-      xs[v] = oh;
-      xs[nv + v] = om;
-      xs[2 * nv + v] = ol;
-    }
+    for (int c = 0; c < V; ++c) oe[c] = from_f<T>(xhat(to_f(e[c]), r, gamma[v * V + c]));
+    xr[v] = o;
   }
 }
 
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
-                           float eps, float* inv_rms, void* x, void* xs3, cudaStream_t s) {
+                           float eps, float* inv_rms, void* x, cudaStream_t s) {
   dim3 grid(cdiv(T, 8));
   if (dt == ACE_BF16)
     k_rmsnorm<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)u, T, d, gamma, eps,
-                                                  inv_rms, (__nv_bfloat16*)x,
-                                                  (__nv_bfloat16*)xs3);
+                                                  inv_rms, (__nv_bfloat16*)x);
   else
-    k_rmsnorm<float><<<grid, 256, 0, s>>>((const float*)u, T, d, gamma, eps, inv_rms, (float*)x,
-                                          nullptr);
+    k_rmsnorm<float><<<grid, 256, 0, s>>>((const float*)u, T, d, gamma, eps, inv_rms, (float*)x);
   return cudaGetLastError();
 }
 
@@ -131,7 +104,7 @@ __global__ void __launch_bounds__(256) k_router_logits(const T* __restrict__ u,
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int kk = k0 + lk + j;
-      As[lk + j][lr] = arow ? to_f(ua[kk]) * rr * gamma[kk] : 0.f;
+      As[lk + j][lr] = arow ? xhat(to_f(ua[kk]), rr, gamma[kk]) : 0.f;
       Bs[lk + j][lr] = brow ? to_f(wb[kk]) : 0.f;
     }
     __syncthreads();
@@ -231,7 +204,7 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
     }
     int my_e = 0;
     float my_v = -INFINITY;
-    topk_select(v, V, E, k, lane, my_e, my_v, status);
+    topk_sorted(v, E, k, lane, my_e, my_v, status);
     const float v0 = __shfl_sync(0xffffffffu, my_v, 0);  // the top-1 logit is the maximum
     const float ex = (lane < k) ? expf(my_v - v0) : 0.f;
     float denom;
@@ -258,7 +231,7 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     bitmap[(size_t)c * E + e] = bm[e];
-    hist[(size_t)e * gridDim.x + c] = __popc(bm[e]);  // expert-major
+    hist[(size_t)c * E + e] = __popc(bm[e]);
   }
   if (done_ctr == nullptr) return;
   // the last CTA to finish runs the expert-offset scan over every chunk's
