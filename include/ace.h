@@ -280,15 +280,15 @@ ACE_API ace_status ace_moe_route(const ace_layer* layer, const void* u, int T,
  *   k are not read.  xp (device) [S][d] layer->dtype, 16-byte aligned;
  *   offsets (device) [E+1] int32, rising from 0 to S (otherwise
  *   ACE_FLAG_BAD_INDEX is raised and nothing is computed); slot_gate
- *   (device) [S] fp32; yslot (device) [S][d] fp32, 16-byte aligned.
- *   Same kernels and numerics as the forward's expert GEMMs (h rounded to
- *   the storage type, fp32 accumulation).  Device flags: ace_read_status
- *   on ws.
+ *   (device) [S] fp32; yslot (device) [S][d] layer->dtype, 16-byte aligned.
+ *   Same kernels and numerics as the forward's expert GEMMs (fp32
+ *   accumulation; h and each yslot row rounded to the storage type).
+ *   Device flags: ace_read_status on ws.
  * ---------------------------------------------------------------------- */
 ACE_API size_t ace_experts_workspace_size(const ace_layer* layer, int max_slots);
 ACE_API ace_status ace_moe_experts(const ace_layer* layer, const void* xp, int S,
                                    const int32_t* offsets, const float* slot_gate,
-                                   float* yslot, void* ws, size_t ws_bytes, void* stream);
+                                   void* yslot, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * ace_moe_combine -- the forward's combine on slot outputs the caller
@@ -300,12 +300,13 @@ ACE_API ace_status ace_moe_experts(const ace_layer* layer, const void* xp, int S
  *   gate-weighted sum of the kept experts; the gates are already in yslot,
  *   skipped slots drop out without re-normalising).
  *   slot_of (device) [T][k] int32, -1 for a skipped slot; yslot (device)
- *   [n_rows][d] fp32, 16-byte aligned; y (device) [T][d] dtype, 16-byte
- *   aligned; d % 4 == 0.  An index >= n_rows raises ACE_FLAG_BAD_INDEX and
- *   drops out.  ws: at least 256 bytes (its status word; ace_read_status).
+ *   [n_rows][d] dtype, 16-byte aligned (ace_moe_experts' output); y (device)
+ *   [T][d] dtype, 16-byte aligned; d a multiple of 8 (bf16) or 4 (fp32).
+ *   An index >= n_rows raises ACE_FLAG_BAD_INDEX and drops out.  ws: at
+ *   least 256 bytes (its status word; ace_read_status).
  * ---------------------------------------------------------------------- */
 ACE_API ace_status ace_moe_combine(int T, int k, int d, ace_dtype dtype, const int32_t* slot_of,
-                                   const float* yslot, int n_rows, void* y, void* ws,
+                                   const void* yslot, int n_rows, void* y, void* ws,
                                    size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------

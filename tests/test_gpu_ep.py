@@ -112,7 +112,7 @@ def test_experts_and_combine_flag_bad_indices():
     ws = ace.alloc_workspace(ace.ace_experts_workspace_size(el, S))
     # offsets that do not end at S
     bad = torch.tensor([0, 3, 5, 5, 9, 9, 10, 11, 11], dtype=torch.int32, device="cuda")
-    ys = torch.zeros(S, w.d, device="cuda")
+    ys = torch.zeros(S, w.d, dtype=torch.bfloat16, device="cuda")
     ace.ace_moe_experts(el, xp, bad, g, ys, ws)
     assert ace.ace_read_status(ws) == (ace.ACE_ERR_DEVICE_FAULT, ace.ACE_FLAG_BAD_INDEX)
     # good offsets: clean, finite
@@ -125,5 +125,5 @@ def test_experts_and_combine_flag_bad_indices():
     y = torch.empty(3, w.d, dtype=torch.bfloat16, device="cuda")
     ace.ace_moe_combine(slot_of, ys, y, ws)
     assert ace.ace_read_status(ws) == (ace.ACE_ERR_DEVICE_FAULT, ace.ACE_FLAG_BAD_INDEX)
-    assert torch.equal(y[2], ys[3].to(torch.bfloat16))
-    assert torch.equal(y[1], ys[2].to(torch.bfloat16))
+    assert torch.equal(y[2], ys[3])
+    assert torch.equal(y[1], ys[2])

@@ -236,7 +236,10 @@ def ace_experts_workspace_size(layer, max_slots):
 
 def ace_moe_experts(layer, xp, offsets, slot_gate, yslot, ws, stream=None):
     """yslot[s] = slot_gate[s] * f_e(xp[s]) for the slots of expert e,
-    offsets[e] <= s < offsets[e + 1] (see include/ace.h)."""
+    offsets[e] <= s < offsets[e + 1] (see include/ace.h); yslot [S][d] in
+    xp's dtype."""
+    if yslot.dtype != xp.dtype:
+        raise ValueError("yslot must have xp's dtype")
     code = _lib.ace_moe_experts(ctypes.byref(layer), _ptr(xp), int(xp.shape[0]), _ptr(offsets),
                                 _ptr(slot_gate), _ptr(yslot), _ptr(ws), ws.numel(),
                                 _stream(stream))
@@ -246,7 +249,9 @@ def ace_moe_experts(layer, xp, offsets, slot_gate, yslot, ws, stream=None):
 
 def ace_moe_combine(slot_of, yslot, y, ws, stream=None):
     """y[t] = sum over i of yslot[slot_of[t, i]] for slot_of >= 0, in i order
-    (see include/ace.h); slot_of [T][k] int32, yslot [n][d] fp32."""
+    (see include/ace.h); slot_of [T][k] int32, yslot [n][d] in y's dtype."""
+    if yslot.dtype != y.dtype:
+        raise ValueError("yslot must have y's dtype")
     T, k = slot_of.shape
     code = _lib.ace_moe_combine(int(T), int(k), int(y.shape[1]), _dtype_code(y), _ptr(slot_of),
                                 _ptr(yslot), int(yslot.shape[0]), _ptr(y), _ptr(ws), ws.numel(),

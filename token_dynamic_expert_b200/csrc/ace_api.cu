@@ -83,7 +83,7 @@ FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms) {
   o.slot_of = take(cap * 4);
   o.xp = take(cap * d * es);
   o.h = take(cap * m * es);
-  o.yslot = take(cap * d * 4);
+  o.yslot = take(cap * d * es);
   o.total = off;
   return o;
 }
@@ -163,16 +163,28 @@ P* at(void* ws, size_t off) {
 // Word of the status block counting finished routing CTAs (zeroed per call).
 constexpr size_t kDoneCtrWord = 32;
 
+// Status words a call zeroes before its kernels run: all 64 of the block, or
+// (a layer stack keeping one status word across layers) words 16-63.
+struct StatusClear {
+  uint32_t* p;
+  int n;
+};
+StatusClear status_clear(const FwdLayout& ly, void* ws, bool keep_status) {
+  uint32_t* w = at<uint32_t>(ws, ly.status);
+  return keep_status ? StatusClear{w + 16, 48} : StatusClear{w, 64};
+}
+
 // The routing half shared by the forward and the score query; with_scan adds
 // the compaction's expert-offset scan (run by the routing's last CTA).  x_out
-// (nullable) receives x rounded to the storage type.
+// (nullable) receives x rounded to the storage type.  The first kernel zeroes
+// the status words `clr` (T > 0 here).
 ace_status run_routing(const ace_layer& L, const void* u, int T, const ace_fwd_opts& o,
                        const FwdLayout& ly, void* ws, int num_sms, float* logits_dbg,
-                       bool with_scan, void* x_out, cudaStream_t s) {
+                       bool with_scan, void* x_out, StatusClear clr, cudaStream_t s) {
   const int splitk = router_splits_for(L, T, num_sms);
   const bool tc = L.dtype == ACE_BF16;
   ACE_CK(launch_rmsnorm(L.dtype, u, T, L.d, L.gamma, o.eps_rms, at<float>(ws, ly.inv_rms), x_out,
-                        s));
+                        clr.p, clr.n, s));
   if (tc)
     ACE_CK(launch_router_tc(u, at<float>(ws, ly.inv_rms), L.gamma, L.w_router, T, L.d, L.E,
                             splitk, at<float>(ws, ly.part), at<uint32_t>(ws, ly.status), num_sms,
@@ -225,9 +237,10 @@ bool fused_experts(const ace_layer& L, int T) { return (long long)T * L.k < 128L
 // combine.
 ace_status run_prefill(const ace_layer& L, const void* u, int T, const ace_fwd_opts& o, void* y,
                        const FwdLayout& ly, void* ws, int num_sms, ace_debug_out* dbg,
-                       cudaEvent_t ev_b, cudaEvent_t ev_m, cudaEvent_t ev_e, cudaStream_t s) {
-  ace_status st =
-      run_routing(L, u, T, o, ly, ws, num_sms, dbg ? dbg->logits : nullptr, true, nullptr, s);
+                       StatusClear clr, cudaEvent_t ev_b, cudaEvent_t ev_m, cudaEvent_t ev_e,
+                       cudaStream_t s) {
+  ace_status st = run_routing(L, u, T, o, ly, ws, num_sms, dbg ? dbg->logits : nullptr, true,
+                              nullptr, clr, s);
   if (st != ACE_OK) return st;
   ACE_CK(launch_scatter_gather(
       L.dtype, T, L.k, L.E, L.d, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
@@ -239,26 +252,26 @@ ace_status run_prefill(const ace_layer& L, const void* u, int T, const ace_fwd_o
   if (L.dtype == ACE_BF16 && fused_experts(L, T)) {
     // one launch for both expert GEMMs; "mid" is recorded after it as well
     ACE_CK(launch_experts_fused(L, T * L.k, at<void>(ws, ly.xp), at<void>(ws, ly.h),
-                                at<float>(ws, ly.yslot), at<int4>(ws, ly.tiles),
+                                at<void>(ws, ly.yslot), at<int4>(ws, ly.tiles),
                                 at<int32_t>(ws, ly.n_tiles), ly.max_tiles,
                                 at<float>(ws, ly.slot_gate), at<uint32_t>(ws, ly.tile_done),
                                 at<uint32_t>(ws, ly.status), num_sms, s));
     if (ev_m) ACE_CK(cudaEventRecord(ev_m, s));
   } else if (L.dtype == ACE_BF16) {
     if (launch_experts_sm100(L, T * L.k, at<void>(ws, ly.xp), at<void>(ws, ly.h),
-                             at<float>(ws, ly.yslot), at<int4>(ws, ly.tiles),
+                             at<void>(ws, ly.yslot), at<int4>(ws, ly.tiles),
                              at<int32_t>(ws, ly.n_tiles), ly.max_tiles,
                              at<float>(ws, ly.slot_gate), at<uint32_t>(ws, ly.status), num_sms,
                              s, ev_m) != cudaSuccess)
       return cuda_fail(cudaGetLastError());
   } else {
-    ACE_CK(launch_experts_simt(L, at<void>(ws, ly.xp), at<void>(ws, ly.h), at<float>(ws, ly.yslot),
+    ACE_CK(launch_experts_simt(L, at<void>(ws, ly.xp), at<void>(ws, ly.h), at<void>(ws, ly.yslot),
                                at<int4>(ws, ly.tiles), at<int32_t>(ws, ly.n_tiles), ly.max_tiles,
                                at<float>(ws, ly.slot_gate), s));
     if (ev_m) ACE_CK(cudaEventRecord(ev_m, s));
   }
   if (ev_e) ACE_CK(cudaEventRecord(ev_e, s));
-  ACE_CK(launch_combine(L.dtype, T, L.k, L.d, at<int32_t>(ws, ly.slot_of), at<float>(ws, ly.yslot),
+  ACE_CK(launch_combine(L.dtype, T, L.k, L.d, at<int32_t>(ws, ly.slot_of), at<void>(ws, ly.yslot),
                         T * L.k, y, at<uint32_t>(ws, ly.status), s));
   return ACE_OK;
 }
@@ -301,13 +314,10 @@ ace_status forward_impl(const ace_layer* layer, const void* u, int T, const ace_
   // status word (offset 0), the decode kernel's cross-CTA words (byte 64)
   // and the routing CTAs' completion count (byte 128).  The decode kernel
   // needs no clearing: its words carry their launch's epoch, and it writes
-  // the status word itself as it finishes.
-  if (!decode) {
-    if (keep_status)
-      ACE_CK(launch_clear_words(at<uint8_t>(ws, ly.status) + 64, 48, s));
-    else
-      ACE_CK(launch_clear_words(at<void>(ws, ly.status), 64, s));
-  }
+  // the status word itself as it finishes.  The prefill's first kernel
+  // zeroes them; with no token there is no kernel, so a clear runs instead.
+  const StatusClear clr = status_clear(ly, ws, keep_status);
+  if (!decode && T == 0) ACE_CK(launch_clear_words(clr.p, clr.n, s));
   if (T == 0) return ACE_OK;
   cudaEvent_t ev_b = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_begin) : nullptr;
   cudaEvent_t ev_m = dbg ? static_cast<cudaEvent_t>(dbg->ev_experts_mid) : nullptr;
@@ -327,7 +337,7 @@ ace_status forward_impl(const ace_layer* layer, const void* u, int T, const ace_
                          num_sms, s));
     if (ev_e) ACE_CK(cudaEventRecord(ev_e, s));
   } else {
-    st = run_prefill(L, u, T, *opts, y, ly, ws, num_sms, dbg, ev_b, ev_m, ev_e, s);
+    st = run_prefill(L, u, T, *opts, y, ly, ws, num_sms, dbg, clr, ev_b, ev_m, ev_e, s);
     if (st != ACE_OK) return st;
   }
   if (dbg) {
@@ -437,9 +447,12 @@ ace_status ace_moe_scores(const ace_layer* layer, const void* u, int T, const ac
   const FwdLayout ly = fwd_layout(L, T, num_sms);
   if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ACE_CK(launch_clear_words(at<void>(ws, ly.status), 64, s));
-  if (T == 0) return ACE_OK;
-  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, false, nullptr, s);
+  const StatusClear clr = status_clear(ly, ws, false);
+  if (T == 0) {
+    ACE_CK(launch_clear_words(clr.p, clr.n, s));
+    return ACE_OK;
+  }
+  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, false, nullptr, clr, s);
   if (st != ACE_OK) return st;
   const size_t tk = (size_t)T * L.k;
   ACE_CK(cudaMemcpyAsync(score, at<void>(ws, ly.score), tk * 4, cudaMemcpyDeviceToDevice, s));
@@ -461,9 +474,12 @@ ace_status ace_moe_route(const ace_layer* layer, const void* u, int T, const ace
   const FwdLayout ly = fwd_layout(L, T, num_sms);
   if (ws_bytes < ly.total) return ACE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  ACE_CK(launch_clear_words(at<void>(ws, ly.status), 64, s));
-  if (T == 0) return ACE_OK;
-  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, false, x, s);
+  const StatusClear clr = status_clear(ly, ws, false);
+  if (T == 0) {
+    ACE_CK(launch_clear_words(clr.p, clr.n, s));
+    return ACE_OK;
+  }
+  st = run_routing(L, u, T, *opts, ly, ws, num_sms, nullptr, false, x, clr, s);
   if (st != ACE_OK) return st;
   const size_t tk = (size_t)T * L.k;
   ACE_CK(cudaMemcpyAsync(idx, at<void>(ws, ly.idx), tk * 4, cudaMemcpyDeviceToDevice, s));

@@ -53,8 +53,10 @@ cudaError_t launch_clear_words(void* p, int n_words, cudaStream_t s);
 ace_status check_fusion(const ace_layer& L, int fusion);
 
 // ---------------------------------------------------------------- launchers
+// 1/rms per token, x (nullable), and zeroes clear[0 .. n_clear) (n_clear <= 256)
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
-                           float eps, float* inv_rms, void* x, cudaStream_t s);
+                           float eps, float* inv_rms, void* x, uint32_t* clear, int n_clear,
+                           cudaStream_t s);
 // Tensor-core router (bf16 layers): part[split][t][e] from u [T][d] (bf16),
 // 1/rms, gamma and w_router [E][d].
 int router_tc_splits(int T, int d, int E, int num_sms);
@@ -80,17 +82,18 @@ cudaError_t launch_scatter_gather(ace_dtype dt, int T, int k, int E, int d, cons
                                   const float* gamma, int32_t* slot_token, int32_t* slot_rank,
                                   float* slot_gate, int32_t* slot_of, void* xp, uint32_t* status,
                                   cudaStream_t s);
+// yslot [S][d] in the layer's storage type
 cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* xp, void* h,
-                                 float* yslot, const int4* tiles, const int32_t* n_tiles,
+                                 void* yslot, const int4* tiles, const int32_t* n_tiles,
                                  int max_tiles, const float* slot_gate, uint32_t* status,
                                  int num_sms, cudaStream_t s, cudaEvent_t ev_mid);
 // Both expert GEMMs in one persistent kernel (bf16 layers): gate/up items
 // first, then down items, each down item waiting for its tile's h rows.
 cudaError_t launch_experts_fused(const ace_layer& L, int cap_slots, const void* xp, void* h,
-                                 float* yslot, const int4* tiles, const int32_t* n_tiles,
+                                 void* yslot, const int4* tiles, const int32_t* n_tiles,
                                  int max_tiles, const float* slot_gate, uint32_t* tile_done,
                                  uint32_t* status, int num_sms, cudaStream_t s);
-cudaError_t launch_experts_simt(const ace_layer& L, const void* xp, void* h, float* yslot,
+cudaError_t launch_experts_simt(const ace_layer& L, const void* xp, void* h, void* yslot,
                                 const int4* tiles, const int32_t* n_tiles, int max_tiles,
                                 const float* slot_gate, cudaStream_t s);
 size_t decode_smem_bytes(int T, int d, int m, int k, int E, int num_sms);
@@ -109,8 +112,9 @@ ace_status build_tables_impl(const ace_layer* layers, int n_layers, const ace_ta
 size_t tau_workspace_size();
 cudaError_t launch_tau_quantile(const float* score, int n_tok, int k, long long n_skip,
                                 float* tau, void* ws, int num_sms, cudaStream_t s);
+// yslot [n_rows][d] and y [T][d] in the storage type dt
 cudaError_t launch_combine(ace_dtype dt, int T, int k, int d, const int32_t* slot_of,
-                           const float* yslot, int n_rows, void* y, uint32_t* status,
+                           const void* yslot, int n_rows, void* y, uint32_t* status,
                            cudaStream_t s);
 
 }  // namespace ace

@@ -105,7 +105,7 @@ size_t ace_experts_workspace_size(const ace_layer* layer, int max_slots) {
 }
 
 ace_status ace_moe_experts(const ace_layer* layer, const void* xp, int S, const int32_t* offsets,
-                           const float* slot_gate, float* yslot, void* ws, size_t ws_bytes,
+                           const float* slot_gate, void* yslot, void* ws, size_t ws_bytes,
                            void* stream) {
   const ace_status st = check_expert_layer(layer);
   if (st != ACE_OK) return st;
@@ -146,10 +146,13 @@ ace_status ace_moe_experts(const ace_layer* layer, const void* xp, int S, const 
 }
 
 ace_status ace_moe_combine(int T, int k, int d, ace_dtype dtype, const int32_t* slot_of,
-                           const float* yslot, int n_rows, void* y, void* ws, size_t ws_bytes,
+                           const void* yslot, int n_rows, void* y, void* ws, size_t ws_bytes,
                            void* stream) {
-  if (T < 0 || k < 1 || k > kMaxK || d <= 0 || d % 4 != 0 || n_rows < 0) return ACE_ERR_INVALID_ARG;
   if (dtype != ACE_BF16 && dtype != ACE_F32) return ACE_ERR_INVALID_ARG;
+  // rows are read and written as 16-byte vectors
+  const int vec = dtype == ACE_BF16 ? 8 : 4;
+  if (T < 0 || k < 1 || k > kMaxK || d <= 0 || d % vec != 0 || n_rows < 0)
+    return ACE_ERR_INVALID_ARG;
   if (T > 0 && (!slot_of || !y || !is_aligned(slot_of, 4) || !is_aligned(y, 16) ||
                 (n_rows > 0 && (!yslot || !is_aligned(yslot, 16)))))
     return ACE_ERR_INVALID_ARG;

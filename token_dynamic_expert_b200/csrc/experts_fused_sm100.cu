@@ -1,7 +1,7 @@
 // experts_fused_sm100.cu -- both grouped SwiGLU expert GEMMs of the prefill
 // ([ACE] "Theoretical Foundation", eq. for f_{l,e}) in one persistent kernel:
 //   gate/up items:  H = SiLU(Xp W^gate_e) (.) (Xp W^up_e)    -> bf16 [S][m]
-//   down items:     Yslot = g * (H W^down_e)                 -> fp32 [S][d]
+//   down items:     Yslot = g * (H W^down_e)                 -> bf16 [S][d]
 //
 // The operands, tiles, warp roles, TMEM accumulators and epilogues are those
 // of the two-launch version (experts_sm100.cu): swap-AB, weight rows on the
@@ -51,7 +51,7 @@ struct FusedArgs {
   const int32_t* n_tiles;
   int max_tiles, m, d;
   __nv_bfloat16* h;        // [S][m]
-  float* yslot;            // [S][d]
+  __nv_bfloat16* yslot;    // [S][d]
   const float* slot_gate;  // [S]
   uint32_t* tile_done;     // [max_tiles] gate/up items written per tile (zeroed)
   uint32_t* status;
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 16; ++c)
             if (c0 + c < n) {
               const int slot = row0 + c0 + c;
-              a.yslot[(size_t)slot * a.d + col] = a.slot_gate[slot] * v[c];
+              a.yslot[(size_t)slot * a.d + col] = __float2bfloat16_rn(a.slot_gate[slot] * v[c]);
             }
         }
       }
@@ -353,7 +353,7 @@ bool fused_map(CUtensorMap* mp, const void* base, uint64_t rows, uint64_t cols,
 }  // namespace
 
 cudaError_t launch_experts_fused(const ace_layer& L, int cap_slots, const void* xp, void* h,
-                                 float* yslot, const int4* tiles, const int32_t* n_tiles,
+                                 void* yslot, const int4* tiles, const int32_t* n_tiles,
                                  int max_tiles, const float* slot_gate, uint32_t* tile_done,
                                  uint32_t* status, int num_sms, cudaStream_t s) {
   CUtensorMap mg, mu, mx, md, mh;
@@ -377,7 +377,7 @@ cudaError_t launch_experts_fused(const ace_layer& L, int cap_slots, const void* 
   a.m = L.m;
   a.d = L.d;
   a.h = static_cast<__nv_bfloat16*>(h);
-  a.yslot = yslot;
+  a.yslot = static_cast<__nv_bfloat16*>(yslot);
   a.slot_gate = slot_gate;
   a.tile_done = tile_done;
   a.status = status;

@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(256) k_simt_gateup(const T* __restrict__ wg,
 template <typename T>
 __global__ void __launch_bounds__(256) k_simt_down(const T* __restrict__ wd, int d, int m,
                                                    const T* __restrict__ h,
-                                                   float* __restrict__ yslot,
+                                                   T* __restrict__ yslot,
                                                    const float* __restrict__ slot_gate,
                                                    const int4* __restrict__ tiles,
                                                    const int32_t* __restrict__ n_tiles) {
@@ -55,11 +55,11 @@ __global__ void __launch_bounds__(256) k_simt_down(const T* __restrict__ wd, int
     const T* hr = h + (size_t)(row0 + r) * m;
     float acc = 0.f;
     for (int j = 0; j < m; ++j) acc = fmaf(to_f(hr[j]), to_f(w[j]), acc);
-    yslot[(size_t)(row0 + r) * d + i] = slot_gate[row0 + r] * acc;
+    yslot[(size_t)(row0 + r) * d + i] = from_f<T>(slot_gate[row0 + r] * acc);
   }
 }
 
-cudaError_t launch_experts_simt(const ace_layer& L, const void* xp, void* h, float* yslot,
+cudaError_t launch_experts_simt(const ace_layer& L, const void* xp, void* h, void* yslot,
                                 const int4* tiles, const int32_t* n_tiles, int max_tiles,
                                 const float* slot_gate, cudaStream_t s) {
   dim3 g1(max_tiles, cdiv(L.m, 64)), g2(max_tiles, cdiv(L.d, 64));
@@ -67,14 +67,15 @@ cudaError_t launch_experts_simt(const ace_layer& L, const void* xp, void* h, flo
     k_simt_gateup<float><<<g1, 256, 0, s>>>((const float*)L.w_gate, (const float*)L.w_up, L.d,
                                             L.m, (const float*)xp, (float*)h, tiles, n_tiles);
     k_simt_down<float><<<g2, 256, 0, s>>>((const float*)L.w_down, L.d, L.m, (const float*)h,
-                                          yslot, slot_gate, tiles, n_tiles);
+                                          (float*)yslot, slot_gate, tiles, n_tiles);
   } else {
     k_simt_gateup<__nv_bfloat16><<<g1, 256, 0, s>>>(
         (const __nv_bfloat16*)L.w_gate, (const __nv_bfloat16*)L.w_up, L.d, L.m,
         (const __nv_bfloat16*)xp, (__nv_bfloat16*)h, tiles, n_tiles);
     k_simt_down<__nv_bfloat16><<<g2, 256, 0, s>>>((const __nv_bfloat16*)L.w_down, L.d, L.m,
-                                                  (const __nv_bfloat16*)h, yslot, slot_gate,
-                                                  tiles, n_tiles);
+                                                  (const __nv_bfloat16*)h,
+                                                  (__nv_bfloat16*)yslot, slot_gate, tiles,
+                                                  n_tiles);
   }
   return cudaGetLastError();
 }

@@ -4,7 +4,7 @@
 // [ACE] "Theoretical Foundation", eq. for f_{l,e}: for the kept slots of
 // expert e (rows row0 .. row0+n-1 of the gathered matrix Xp):
 //   MODE 0:  H = SiLU(Xp W^gate_e) (.) (Xp W^up_e)      -> bf16 [S][m]
-//   MODE 1:  Yslot = g * (H W^down_e)                   -> fp32 [S][d]
+//   MODE 1:  Yslot = g * (H W^down_e)                   -> bf16 [S][d]
 //
 // Operand roles are swapped ("swap-AB"): weight rows sit on the MMA's M side
 // (128, the tensor-core M) and the expert's kept slots on N (16..256, rounded
@@ -23,15 +23,16 @@
 // The gate/up launch runs on CTA pairs (tcgen05.mma.cta_group::2, see
 // k_experts_pair below); the down launch on single CTAs.
 //
-// Warp roles (6 warps):
+// Warp roles:
 //   warp 0      TMA producer: weight rows (128 x 64 bf16 per stage) and the
-//               tile's slot rows (32-row boxes, only as many as it needs),
+//               tile's slot rows (64-row boxes, only as many as it needs),
 //               128-byte swizzle, mbarrier transaction counts.
 //   warp 1      TMEM allocator and MMA issuer (one thread): 4 MMAs of K=16
 //               per stage; tcgen05.commit frees the stage and, after the last
 //               stage of an item, hands the accumulator to the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld 16 columns at a time, SiLU(.)*up or
-//               gate scaling, global stores.
+//   warps 2..   epilogue: tcgen05.ld 16 columns at a time, SiLU(.)*up or
+//               gate scaling, global stores; 4 warps in the gate/up (pair)
+//               kernel, 8 in the down kernel.
 // Two TMEM accumulators of 256 columns alternate between items, so the
 // epilogue of one item overlaps the main loop of the next.  The stage count
 // adapts to the largest slot tile of the launch (more stages when tiles are
@@ -54,7 +55,12 @@ constexpr int kBoxBytes = kBoxN * kBK * 2;  // 8 KB
 constexpr int kMaxStages = 8;
 constexpr int kStageBudget = 200 * 1024;
 constexpr int kXchgBytes = 2 * 2 * 64 * 8 * 4;  // 2 buffers x (gate, up) x 64 rows x 8 floats
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;               // the CTA-pair kernel: 4 epilogue warps
+// The one-CTA kernel (the down GEMM) has 8 epilogue warps, two per TMEM lane
+// quarter taking alternate 16-slot groups: its epilogue (a bf16 store per slot
+// and output column) is the slower side of its pipeline.
+constexpr int kEpiWarps1 = 8;
+constexpr int kThreads1 = 64 + 32 * kEpiWarps1;
 constexpr uint32_t kTmemCols = 512;         // two accumulators of 256 columns
 constexpr int kSmemBytes = 1024 + kStageBudget + kXchgBytes + 512;
 
@@ -65,7 +71,7 @@ __device__ __forceinline__ void epilogue_bar() {
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads1, 1)
     k_experts(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
               const __grid_constant__ CUtensorMap tmB, const int4* __restrict__ tiles,
               const int32_t* __restrict__ n_tiles_ptr, int max_tiles, int rows_per_expert,
@@ -102,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], MODE == 1 ? 32 * kEpiWarps1 : 128);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -214,9 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(drain);
       mbar_drain(drain, 0);
     }
-  } else {
+  } else if (MODE == 1 || warp < 6) {
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may read
+    // MODE 1: the two warps of a quarter take alternate 16-slot groups
+    const int g0 = MODE == 1 ? ((warp - 2) >> 2) * 16 : 0, gstep = MODE == 1 ? 32 : 16;
     int acc = 0;
     uint32_t acc_phase = 0;
     int xb = 0;  // exchange buffer parity (MODE 0)
@@ -258,17 +266,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         const int col = it * kBM + q * 32 + lane;
-        float* Y = reinterpret_cast<float*>(out);
-        for (int c0 = 0; c0 < n; c0 += 16) {
+        __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(out) + col;
+        for (int c0 = g0; c0 < n; c0 += gstep) {
           float v[16];
           tmem_ld16(tbase + (uint32_t)c0, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            if (c0 + c < n) {
-              const int slot = row0 + c0 + c;
-              Y[(size_t)slot * out_ld + col] = slot_gate[slot] * v[c];
-            }
+          for (int c = 0; c < 16; c += 2) {  // two slots per conversion
+            const int slot = row0 + c0 + c;
+            const float ga = c0 + c < n ? slot_gate[slot] : 0.f;
+            const float gb = c0 + c + 1 < n ? slot_gate[slot + 1] : 0.f;
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(ga * v[c], gb * v[c + 1]);
+            if (c0 + c < n) Y[(size_t)slot * out_ld] = pr.x;
+            if (c0 + c + 1 < n) Y[(size_t)(slot + 1) * out_ld] = pr.y;
+          }
         }
       }
       tc_fence_before();
@@ -546,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         const int col = it * 256 + (int)rank * kBM + q * 32 + lane;
-        float* Y = reinterpret_cast<float*>(out);
+        __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(out);
         for (int c0 = 0; c0 < n; c0 += 16) {
           float v[16];
           tmem_ld16(tbase + (uint32_t)c0, v);
@@ -556,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 16; ++c)
               if (c0 + c < n) {
                 const int slot = row0 + c0 + c;
-                Y[(size_t)slot * out_ld + col] = slot_gate[slot] * v[c];
+                Y[(size_t)slot * out_ld + col] = __float2bfloat16_rn(slot_gate[slot] * v[c]);
               }
           }
         }
@@ -664,7 +675,7 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
 }  // namespace
 
 cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* xp, void* h,
-                                 float* yslot, const int4* tiles, const int32_t* n_tiles,
+                                 void* yslot, const int4* tiles, const int32_t* n_tiles,
                                  int max_tiles, const float* slot_gate, uint32_t* status,
                                  int num_sms, cudaStream_t s, cudaEvent_t ev_mid) {
   CUtensorMap mg, mu, mx, md, mh;
@@ -684,7 +695,7 @@ cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* 
     return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
   if ((e = set_smem_attr<1>()) != cudaSuccess) return e;
-  k_experts<1><<<num_sms, kThreads, kSmemBytes, s>>>(md, md, mh, tiles, n_tiles, max_tiles, L.d,
+  k_experts<1><<<num_sms, kThreads1, kSmemBytes, s>>>(md, md, mh, tiles, n_tiles, max_tiles, L.d,
                                                      L.m, L.d / kBM, yslot, L.d, slot_gate, status);
   return cudaGetLastError();
 }

@@ -28,11 +28,15 @@ namespace ace {
 // ------------------------------------------------------------------ RMSNorm
 // One warp per token, 16-byte loads and stores (d is a multiple of 64).
 // x (nullable) receives xhat(u, 1/rms, gamma) rounded to the storage type.
+// As the forward's first kernel it also zeroes the call's status words
+// (clear[0 .. n_clear)), which no kernel of the forward touches before it.
 template <typename T>
 __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn, int d,
                                                  const float* __restrict__ gamma, float eps,
-                                                 float* __restrict__ inv_rms, T* __restrict__ x) {
+                                                 float* __restrict__ inv_rms, T* __restrict__ x,
+                                                 uint32_t* __restrict__ clear, int n_clear) {
   constexpr int V = 16 / sizeof(T);
+  if (blockIdx.x == 0 && (int)threadIdx.x < n_clear) clear[threadIdx.x] = 0u;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= Tn) return;
@@ -65,13 +69,16 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn
 }
 
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
-                           float eps, float* inv_rms, void* x, cudaStream_t s) {
+                           float eps, float* inv_rms, void* x, uint32_t* clear, int n_clear,
+                           cudaStream_t s) {
   dim3 grid(cdiv(T, 8));
+  if (n_clear > 256) return cudaErrorInvalidValue;
   if (dt == ACE_BF16)
     k_rmsnorm<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)u, T, d, gamma, eps,
-                                                  inv_rms, (__nv_bfloat16*)x);
+                                                  inv_rms, (__nv_bfloat16*)x, clear, n_clear);
   else
-    k_rmsnorm<float><<<grid, 256, 0, s>>>((const float*)u, T, d, gamma, eps, inv_rms, (float*)x);
+    k_rmsnorm<float><<<grid, 256, 0, s>>>((const float*)u, T, d, gamma, eps, inv_rms, (float*)x,
+                                          clear, n_clear);
   return cudaGetLastError();
 }
 

@@ -97,7 +97,7 @@ def ace_experts_fn(expert_layer, ws, stream=None):
     from . import ace
 
     def fn(xp, offsets, g):
-        yslot = torch.empty((xp.shape[0], expert_layer.d), dtype=torch.float32, device=xp.device)
+        yslot = torch.empty((xp.shape[0], expert_layer.d), dtype=xp.dtype, device=xp.device)
         if xp.shape[0] > 0:
             ace.ace_moe_experts(expert_layer, xp, offsets, g.float().contiguous(), yslot, ws,
                                 stream=stream)
