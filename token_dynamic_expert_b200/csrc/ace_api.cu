@@ -68,9 +68,11 @@ FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms) {
   o.gate = take(cap * 4);
   o.score = take(cap * 4);
   o.keep = take(cap);
-  o.bitmap = take(nchunk * E * 4);
-  o.hist = take(nchunk * E * 4);
-  o.base = take(nchunk * E * 4);
+  // bitmap and range_cnt adjacent: RMSNorm zeroes them as one block
+  const size_t nrange = (T + kRangeTok - 1) / kRangeTok;
+  o.bitmap = take((nchunk + nrange) * E * 4);
+  o.range_cnt = o.bitmap + nchunk * E * 4;
+  o.rbase = take(nrange * E * 4);
   o.counts = take(E * 4);
   o.offsets = take((E + 1) * 4);
   o.n_kept = take(4);
@@ -183,8 +185,9 @@ ace_status run_routing(const ace_layer& L, const void* u, int T, const ace_fwd_o
                        bool with_scan, void* x_out, StatusClear clr, cudaStream_t s) {
   const int splitk = router_splits_for(L, T, num_sms);
   const bool tc = L.dtype == ACE_BF16;
+  const size_t n_zero = ((size_t)cdiv(T, kChunk) + (size_t)cdiv(T, kRangeTok)) * (size_t)L.E;
   ACE_CK(launch_rmsnorm(L.dtype, u, T, L.d, L.gamma, o.eps_rms, at<float>(ws, ly.inv_rms), x_out,
-                        clr.p, clr.n, s));
+                        clr.p, clr.n, at<uint32_t>(ws, ly.bitmap), n_zero, s));
   if (tc)
     ACE_CK(launch_router_tc(u, at<float>(ws, ly.inv_rms), L.gamma, L.w_router, T, L.d, L.E,
                             splitk, at<float>(ws, ly.part), at<uint32_t>(ws, ly.status), num_sms,
@@ -193,7 +196,7 @@ ace_status run_routing(const ace_layer& L, const void* u, int T, const ace_fwd_o
     ACE_CK(launch_router_logits(L.dtype, u, at<float>(ws, ly.inv_rms), L.gamma, L.w_router, T,
                                 L.d, L.E, splitk, at<float>(ws, ly.part), s));
   ScanOut so{};
-  so.base = at<int32_t>(ws, ly.base);
+  so.rbase = at<int32_t>(ws, ly.rbase);
   so.counts = at<int32_t>(ws, ly.counts);
   so.offsets = at<int32_t>(ws, ly.offsets);
   so.n_kept = at<int32_t>(ws, ly.n_kept);
@@ -206,7 +209,7 @@ ace_status run_routing(const ace_layer& L, const void* u, int T, const ace_fwd_o
   ACE_CK(launch_topk_mask(at<float>(ws, ly.part), splitk, T, L.E, L.k, L.router_bias, ft,
                           o.tau, o.renorm_topk, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
                           at<float>(ws, ly.score), at<uint8_t>(ws, ly.keep),
-                          at<uint32_t>(ws, ly.bitmap), at<int32_t>(ws, ly.hist), logits_dbg,
+                          at<uint32_t>(ws, ly.bitmap), at<int32_t>(ws, ly.range_cnt), logits_dbg,
                           at<uint32_t>(ws, ly.status), at<uint32_t>(ws, ly.status) + kDoneCtrWord,
                           with_scan ? &so : nullptr, s));
   return ACE_OK;
@@ -244,7 +247,7 @@ ace_status run_prefill(const ace_layer& L, const void* u, int T, const ace_fwd_o
   if (st != ACE_OK) return st;
   ACE_CK(launch_scatter_gather(
       L.dtype, T, L.k, L.E, L.d, at<int32_t>(ws, ly.idx), at<float>(ws, ly.gate),
-      at<uint8_t>(ws, ly.keep), at<uint32_t>(ws, ly.bitmap), at<int32_t>(ws, ly.base), u,
+      at<uint8_t>(ws, ly.keep), at<uint32_t>(ws, ly.bitmap), at<int32_t>(ws, ly.rbase), u,
       at<float>(ws, ly.inv_rms), L.gamma, at<int32_t>(ws, ly.slot_token),
       at<int32_t>(ws, ly.slot_rank), at<float>(ws, ly.slot_gate), at<int32_t>(ws, ly.slot_of),
       at<void>(ws, ly.xp), at<uint32_t>(ws, ly.status), s));

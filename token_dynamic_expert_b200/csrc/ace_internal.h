@@ -11,6 +11,7 @@
 namespace ace {
 
 constexpr int kChunk = 32;        // tokens per compaction chunk (one bit each)
+constexpr int kRangeTok = 256;    // tokens per range of the kept-slot counts (8 chunks)
 constexpr int kMaxE = 512;        // experts per layer the routing kernel holds
 constexpr int kMaxK = 16;         // top-k limit
 constexpr int kTileN = 256;       // kept slots per expert tile (GEMM N limit)
@@ -33,7 +34,8 @@ int router_splits_for(const ace_layer& L, int T, int num_sms);
 // Byte offsets of the forward's scratch arrays inside the caller's
 // workspace.  Everything is sized for max_tokens and no skipping.
 struct FwdLayout {
-  size_t status, part, inv_rms, tile_done, idx, gate, score, keep, bitmap, hist, base, counts,
+  size_t status, part, inv_rms, tile_done, idx, gate, score, keep, bitmap, range_cnt, rbase,
+      counts,
       offsets, n_kept, tiles, n_tiles, slot_token, slot_rank, slot_gate, slot_of, xp, h,
       yslot, total;
   int max_tokens, part_floats, max_tiles;
@@ -53,10 +55,11 @@ cudaError_t launch_clear_words(void* p, int n_words, cudaStream_t s);
 ace_status check_fusion(const ace_layer& L, int fusion);
 
 // ---------------------------------------------------------------- launchers
-// 1/rms per token, x (nullable), and zeroes clear[0 .. n_clear) (n_clear <= 256)
+// 1/rms per token, x (nullable); zeroes clear[0 .. n_clear) (n_clear <= 256)
+// and zero[0 .. n_zero)
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
                            float eps, float* inv_rms, void* x, uint32_t* clear, int n_clear,
-                           cudaStream_t s);
+                           uint32_t* zero, size_t n_zero, cudaStream_t s);
 // Tensor-core router (bf16 layers): part[split][t][e] from u [T][d] (bf16),
 // 1/rms, gamma and w_router [E][d].
 int router_tc_splits(int T, int d, int E, int num_sms);
@@ -71,14 +74,14 @@ struct FuseTables;
 cudaError_t launch_topk_mask(const float* part, int splitk, int T, int E, int k,
                              const float* bias, const FuseTables& ft, float tau, int renorm,
                              int32_t* idx, float* gate, float* score, uint8_t* keep,
-                             uint32_t* bitmap, int32_t* hist, float* logits_out,
+                             uint32_t* bitmap, int32_t* range_cnt, float* logits_out,
                              uint32_t* status, uint32_t* done_ctr, const ScanOut* so,
                              cudaStream_t s);
 // Slot tables and the gathered rows Xp[pos] = x[t]; x rows are x_stride
 // elements apart.
 cudaError_t launch_scatter_gather(ace_dtype dt, int T, int k, int E, int d, const int32_t* idx,
                                   const float* gate, const uint8_t* keep, const uint32_t* bitmap,
-                                  const int32_t* base, const void* u, const float* inv_rms,
+                                  const int32_t* rbase, const void* u, const float* inv_rms,
                                   const float* gamma, int32_t* slot_token, int32_t* slot_rank,
                                   float* slot_gate, int32_t* slot_of, void* xp, uint32_t* status,
                                   cudaStream_t s);

@@ -2,13 +2,15 @@
 //
 // Kept slots are ordered by expert, then by token.  The routing kernel left,
 // per chunk c of 32 tokens and expert e, a bitmap of the chunk's tokens that
-// kept a slot of e (a token routes to an expert at most once), its
-// population count, and (its last CTA, compact.cuh) the base position of
-// each (chunk, expert) run.  Here, one CTA per group of 4 tokens:
-//   position of slot (t, i) of expert e = base[c][e] + popcount(bitmap[c][e]
-//   below t); the slot tables are written and x_t = xhat(u_t, 1/rms_t, gamma),
-//   rounded to the storage type, is formed once per token and written into
-//   row `position` of the gathered matrix Xp for each of its kept slots.
+// kept a slot of e (a token routes to an expert at most once), and (its last
+// CTA, compact.cuh) the base position rbase[r][e] of each 256-token range r.
+// Here, one CTA per group of 4 tokens:
+//   position of slot (t, i) of expert e = rbase[r][e]
+//       + popcount(bitmap[c'][e]) over the range's chunks c' before t's chunk c
+//       + popcount(bitmap[c][e] below t);
+// the slot tables are written and x_t = xhat(u_t, 1/rms_t, gamma), rounded to
+// the storage type, is formed once per token and written into row
+// `position` of the gathered matrix Xp for each of its kept slots.
 // No result depends on the order atomics resolve in.
 #include "ace_common.cuh"
 #include "ace_internal.h"
@@ -21,7 +23,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_scatter_gather(
     int Tn, int k, int E, int d, const int32_t* __restrict__ idx, const float* __restrict__ gate,
     const uint8_t* __restrict__ keep, const uint32_t* __restrict__ bitmap,
-    const int32_t* __restrict__ base, const T* __restrict__ u, const float* __restrict__ inv_rms,
+    const int32_t* __restrict__ rbase, const T* __restrict__ u, const float* __restrict__ inv_rms,
     const float* __restrict__ gamma, int32_t* __restrict__ slot_token,
     int32_t* __restrict__ slot_rank, float* __restrict__ slot_gate, int32_t* __restrict__ slot_of,
     T* __restrict__ xp, int cap, uint32_t* status) {
@@ -42,9 +44,12 @@ __global__ void __launch_bounds__(256) k_scatter_gather(
         if (e < 0 || e >= E) {
           raise_flag(status, ACE_FLAG_BAD_INDEX);
         } else {
-          const uint32_t bits = bitmap[(size_t)c * E + e];
-          pos = base[(size_t)c * E + e] +
-                __popc(bits & ((1u << tl) - 1u));
+          const int c0 = (t / kRangeTok) * (kRangeTok / kChunk);
+          pos = rbase[(size_t)(t / kRangeTok) * E + e] +
+                __popc(bitmap[(size_t)c * E + e] & ((1u << tl) - 1u));
+#pragma unroll
+          for (int j = 0; j < kRangeTok / kChunk - 1; ++j)
+            if (c0 + j < c) pos += __popc(bitmap[(size_t)(c0 + j) * E + e]);
           if (pos >= cap) {
             raise_flag(status, ACE_FLAG_OVERFLOW);
             pos = -1;
@@ -98,7 +103,7 @@ __global__ void __launch_bounds__(256) k_scatter_gather(
 
 cudaError_t launch_scatter_gather(ace_dtype dt, int T, int k, int E, int d, const int32_t* idx,
                                   const float* gate, const uint8_t* keep, const uint32_t* bitmap,
-                                  const int32_t* base, const void* u, const float* inv_rms,
+                                  const int32_t* rbase, const void* u, const float* inv_rms,
                                   const float* gamma, int32_t* slot_token, int32_t* slot_rank,
                                   float* slot_gate, int32_t* slot_of, void* xp, uint32_t* status,
                                   cudaStream_t s) {
@@ -106,10 +111,10 @@ cudaError_t launch_scatter_gather(ace_dtype dt, int T, int k, int E, int d, cons
   const int cap = T * k;
   if (dt == ACE_BF16)
     k_scatter_gather<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        T, k, E, d, idx, gate, keep, bitmap, base, (const __nv_bfloat16*)u, inv_rms, gamma,
+        T, k, E, d, idx, gate, keep, bitmap, rbase, (const __nv_bfloat16*)u, inv_rms, gamma,
         slot_token, slot_rank, slot_gate, slot_of, (__nv_bfloat16*)xp, cap, status);
   else
-    k_scatter_gather<float><<<grid, 256, 0, s>>>(T, k, E, d, idx, gate, keep, bitmap, base,
+    k_scatter_gather<float><<<grid, 256, 0, s>>>(T, k, E, d, idx, gate, keep, bitmap, rbase,
                                                  (const float*)u, inv_rms, gamma, slot_token,
                                                  slot_rank, slot_gate, slot_of, (float*)xp, cap,
                                                  status);

@@ -1,10 +1,12 @@
 // compact.cuh -- the expert-offset scan of the compaction, as a block-level
 // device routine run by the last routing CTA to finish.
 //
-// From the per-(expert, 32-token chunk) kept-slot histogram it forms the
+// From the per-(256-token range, expert) kept-slot counts it forms the
 // per-expert counts, the exclusive offsets over experts (kept slots ordered
-// by expert, then token), the per-(chunk, expert) base positions and the list
-// of expert GEMM tiles (expert, first slot, rows <= tile_n) in expert order.
+// by expert, then token), the base position of each (range, expert) run and
+// the list of expert GEMM tiles (expert, first slot, rows <= tile_n) in
+// expert order.  The row gather adds the counts of the chunks before a
+// token's chunk within its range (from the chunk bitmaps).
 #pragma once
 
 #include "ace_common.cuh"
@@ -40,7 +42,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* total) {
 }
 
 struct ScanOut {
-  int32_t* base;     // [nchunk][E]
+  int32_t* rbase;    // [nrange][E]: offset of e + kept slots of e in ranges before r
   int32_t* counts;   // [E]
   int32_t* offsets;  // [E + 1]
   int32_t* n_kept;   // [1]
@@ -50,58 +52,41 @@ struct ScanOut {
   int max_tiles, tile_n;
 };
 
-// Whole-CTA routine (every thread calls it; blockDim.x a multiple of 32, at
-// least E, at most 1024).  hist and base are chunk-major, [nchunk][E]; hist
-// is read with L2-coherent loads (other CTAs wrote it).
-//
-// The warps split the [nchunk][E] table into 32-expert columns (a lane per
-// expert) times chunk ranges, so that every load and store of a warp covers
-// 32 consecutive experts of one chunk and no step needs a shuffle:
-//   pass 1: each warp sums its range per expert (s_part[range][e]);
-//   then per expert: the count (sum over ranges), the exclusive offsets over
-//   experts (a CTA scan) and the expert's GEMM tiles;
-//   pass 2: each warp walks its range again, writing base[c][e] = offset of
-//   e + kept slots of e in chunks before c.
-// An expert of n kept slots gets ceil(n / tile_n) tiles of near-equal size
-// (they differ by at most one slot), in slot order.
-__device__ __forceinline__ void scan_experts(const int32_t* hist, int nchunk, int E,
+// Whole-CTA routine (every thread calls it; blockDim.x a multiple of 32 and
+// at least E / 2).  range_cnt [nrange][E] is read with L2-coherent loads
+// (other CTAs' atomics built it).  Thread i takes experts 2i and 2i + 1, so
+// the exclusive scan over experts runs over per-thread pairs.  An expert of
+// n kept slots gets ceil(n / tile_n) tiles of near-equal size (they differ
+// by one slot at most), in slot order.
+__device__ __forceinline__ void scan_experts(const int32_t* range_cnt, int nrange, int E,
                                              const ScanOut& o) {
   __shared__ int s_warp[32];
-  __shared__ int s_cnt[1024], s_part[1024];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int ncol = (E + 31) / 32;              // 32-expert columns
-  const int nrange = nw / ncol;                // chunk ranges (nw >= ncol since E <= 1024)
-  const int per = (nchunk + nrange - 1) / nrange;
-  const int col = warp % ncol, rg = warp / ncol;
-  const int e = col * 32 + lane;
-  const bool active = rg < nrange && e < E;
-  const int c0 = rg * per, c1 = min(nchunk, c0 + per);
-  // pass 1: per-range sums
-  if (active) {
-    int acc = 0;
-#pragma unroll 8
-    for (int c = c0; c < c1; ++c) acc += __ldcg(hist + (size_t)c * E + e);
-    s_part[rg * E + e] = acc;
-  }
-  __syncthreads();
-  // counts, offsets over experts, the tile list
   const int t = threadIdx.x;
-  int cnt = 0;
-  if (t < E)
-    for (int r = 0; r < nrange; ++r) cnt += s_part[r * E + t];
+  const int e0 = 2 * t;
+  int cnt[2] = {0, 0};
+#pragma unroll 16
+  for (int r = 0; r < nrange; ++r)
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      if (e0 + j < E) cnt[j] += __ldcg(range_cnt + (size_t)r * E + e0 + j);
   int total, total_tiles;
-  const int off = block_excl_scan(cnt, s_warp, &total);
-  const int ntile = t < E ? (cnt + o.tile_n - 1) / o.tile_n : 0;
-  const int toff = block_excl_scan(ntile, s_warp, &total_tiles);
-  if (t < E) {
-    s_cnt[t] = off;  // from here on: the expert's offset
-    o.counts[t] = cnt;
-    o.offsets[t] = off;
-    if (ntile > 0) {
-      const int each = cnt / ntile, rem = cnt - each * ntile;
-      for (int q = 0; q < ntile; ++q)
+  const int off0 = block_excl_scan(cnt[0] + cnt[1], s_warp, &total);
+  int ntile[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) ntile[j] = e0 + j < E ? (cnt[j] + o.tile_n - 1) / o.tile_n : 0;
+  const int toff0 = block_excl_scan(ntile[0] + ntile[1], s_warp, &total_tiles);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int e = e0 + j;
+    if (e >= E) continue;
+    const int off = off0 + (j ? cnt[0] : 0), toff = toff0 + (j ? ntile[0] : 0);
+    o.counts[e] = cnt[j];
+    o.offsets[e] = off;
+    if (ntile[j] > 0) {
+      const int each = cnt[j] / ntile[j], rem = cnt[j] - each * ntile[j];
+      for (int q = 0; q < ntile[j]; ++q)
         if (toff + q < o.max_tiles)
-          o.tiles[toff + q] = make_int4(t, off + q * each + min(q, rem), each + (q < rem ? 1 : 0), 0);
+          o.tiles[toff + q] = make_int4(e, off + q * each + min(q, rem), each + (q < rem ? 1 : 0), 0);
     }
   }
   if (t == 0) {
@@ -111,27 +96,18 @@ __device__ __forceinline__ void scan_experts(const int32_t* hist, int nchunk, in
   }
   if (o.tile_done)
     for (int i = t; i < o.max_tiles; i += blockDim.x) o.tile_done[i] = 0u;
-  __syncthreads();
-  // pass 2: bases, from the expert's offset and the ranges before this one
-  if (active) {
-    int run = s_cnt[e];
-    for (int r = 0; r < rg; ++r) run += s_part[r * E + e];
-    int c = c0;
-    for (; c + 8 <= c1; c += 8) {
-      int v[8];
+  // range bases
+  int run[2] = {off0, off0 + cnt[0]};
+#pragma unroll 8
+  for (int r = 0; r < nrange; ++r)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = __ldcg(hist + (size_t)(c + j) * E + e);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        o.base[(size_t)(c + j) * E + e] = run;
-        run += v[j];
+    for (int j = 0; j < 2; ++j)
+      if (e0 + j < E) {
+        const size_t at = (size_t)r * E + e0 + j;
+        const int c = __ldcg(range_cnt + at);
+        o.rbase[at] = run[j];
+        run[j] += c;
       }
-    }
-    for (; c < c1; ++c) {
-      o.base[(size_t)c * E + e] = run;
-      run += __ldcg(hist + (size_t)c * E + e);
-    }
-  }
 }
 
 }  // namespace ace

@@ -29,14 +29,19 @@ namespace ace {
 // One warp per token, 16-byte loads and stores (d is a multiple of 64).
 // x (nullable) receives xhat(u, 1/rms, gamma) rounded to the storage type.
 // As the forward's first kernel it also zeroes the call's status words
-// (clear[0 .. n_clear)), which no kernel of the forward touches before it.
+// (clear[0 .. n_clear)) and the top-k kernel's bitmaps and range counts
+// (zero[0 .. n_zero)), which no kernel of the forward touches before it.
 template <typename T>
 __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn, int d,
                                                  const float* __restrict__ gamma, float eps,
                                                  float* __restrict__ inv_rms, T* __restrict__ x,
-                                                 uint32_t* __restrict__ clear, int n_clear) {
+                                                 uint32_t* __restrict__ clear, int n_clear,
+                                                 uint32_t* __restrict__ zero, size_t n_zero) {
   constexpr int V = 16 / sizeof(T);
   if (blockIdx.x == 0 && (int)threadIdx.x < n_clear) clear[threadIdx.x] = 0u;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_zero;
+       i += (size_t)gridDim.x * blockDim.x)
+    zero[i] = 0u;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= Tn) return;
@@ -70,15 +75,16 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn
 
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
                            float eps, float* inv_rms, void* x, uint32_t* clear, int n_clear,
-                           cudaStream_t s) {
+                           uint32_t* zero, size_t n_zero, cudaStream_t s) {
   dim3 grid(cdiv(T, 8));
   if (n_clear > 256) return cudaErrorInvalidValue;
   if (dt == ACE_BF16)
     k_rmsnorm<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)u, T, d, gamma, eps,
-                                                  inv_rms, (__nv_bfloat16*)x, clear, n_clear);
+                                                  inv_rms, (__nv_bfloat16*)x, clear, n_clear,
+                                                  zero, n_zero);
   else
     k_rmsnorm<float><<<grid, 256, 0, s>>>((const float*)u, T, d, gamma, eps, inv_rms, (float*)x,
-                                          clear, n_clear);
+                                          clear, n_clear, zero, n_zero);
   return cudaGetLastError();
 }
 
@@ -167,30 +173,44 @@ cudaError_t launch_router_logits(ace_dtype dt, const void* u, const float* inv_r
 }
 
 // -------------------------------------------------------- top-k and the mask
-// One CTA per chunk of 32 tokens, one warp per token.  Lane l holds the
-// logits of experts l, l+32, ...  Selection order is (logit descending,
-// expert index ascending); slot 0 is the top-1 expert.
-template <int V>
-__global__ void __launch_bounds__(1024) k_topk_mask(
+// One warp per token, eight tokens per CTA.  Lane l holds the logits of
+// experts l, l+32, ...  Selection order is (logit descending, expert index
+// ascending); slot 0 is the top-1 expert.  Each kept slot sets its token's bit
+// in the chunk bitmap bitmap[t / 32][e] and counts itself in the range count
+// range_cnt[t / 256][e] (integer atomics: the results do not depend on their
+// order; both arrays are zeroed by RMSNorm).  The last CTA to finish runs the
+// expert-offset scan over the range counts.
+constexpr int kTopkWarps = 8;
+
+// DEEP: every split's loads of a lane in flight at once (64 loads, 128
+// registers, two CTAs an SM) for the many-split launches of short token
+// counts; otherwise four splits at a time in 64 registers (four CTAs an SM),
+// for the few-split launches of long ones.
+template <int V, bool DEEP>
+__global__ void __launch_bounds__(kTopkWarps * 32, DEEP ? 2 : 4) k_topk_mask(
     const float* __restrict__ part, int splitk, int Tn, int E, int k,
     const float* __restrict__ bias, const FuseTables ft, float tau, int renorm,
     int32_t* __restrict__ idx, float* __restrict__ gate, float* __restrict__ score,
-    uint8_t* __restrict__ keep, uint32_t* __restrict__ bitmap, int32_t* __restrict__ hist,
+    uint8_t* __restrict__ keep, uint32_t* __restrict__ bitmap, int32_t* __restrict__ range_cnt,
     float* __restrict__ logits_out, uint32_t* status, uint32_t* done_ctr, ScanOut so) {
-  __shared__ uint32_t bm[kMaxE];
   __shared__ int s_last;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) bm[e] = 0u;
-  __syncthreads();
-  const int c = blockIdx.x;
-  const int tl = warp;
-  const int t = c * kChunk + tl;
+  const int t = blockIdx.x * kTopkWarps + warp;
   if (t < Tn) {
-    // split-K partial sums, all of a split's loads in flight together
+    // the lane's fused factors and bias, loaded beside the partial sums
+    float fv[V], bv[V];
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+      const int e = lane + 32 * q;
+      fv[q] = e < E ? fused_factor(ft, e) : 0.f;
+      bv[q] = (e < E && bias) ? bias[e] : 0.f;
+    }
+    // split-K partial sums in split order
+    constexpr int kUnroll = DEEP ? (V >= 4 ? 64 / V : 16) : (V >= 8 ? 2 : 4);
     float v[V];
 #pragma unroll
     for (int q = 0; q < V; ++q) v[q] = 0.f;
-#pragma unroll 4
+#pragma unroll kUnroll
     for (int sp = 0; sp < splitk; ++sp) {
       const float* pr = part + ((size_t)sp * Tn + t) * E;
 #pragma unroll
@@ -203,7 +223,7 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
     for (int q = 0; q < V; ++q) {
       const int e = lane + 32 * q;
       if (e < E) {
-        if (bias) v[q] += bias[e];
+        if (bias) v[q] += bv[q];
         if (logits_out) logits_out[(size_t)t * E + e] = v[q];
       } else {
         v[q] = -INFINITY;
@@ -212,6 +232,13 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
     int my_e = 0;
     float my_v = -INFINITY;
     topk_sorted(v, E, k, lane, my_e, my_v, status);
+    // the factor of the selected expert, from the lane that holds it
+    float fac = 0.f;
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+      const float x = __shfl_sync(0xffffffffu, fv[q], my_e & 31);
+      if ((my_e >> 5) == q) fac = x;
+    }
     const float v0 = __shfl_sync(0xffffffffu, my_v, 0);  // the top-1 logit is the maximum
     const float ex = (lane < k) ? expf(my_v - v0) : 0.f;
     float denom;
@@ -225,24 +252,22 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
     }
     if (lane < k) {
       const float g = ex / denom;
-      const float sc = g * fused_factor(ft, my_e);
+      const float sc = g * fac;
       const bool kept = (lane == 0) || !(sc < tau);
       const size_t o = (size_t)t * k + lane;
       idx[o] = my_e;
       gate[o] = g;
       score[o] = sc;
       keep[o] = kept ? 1 : 0;
-      if (kept) atomicOr(&bm[my_e], 1u << tl);
+      if (kept) {
+        atomicOr(&bitmap[(size_t)(t / kChunk) * E + my_e], 1u << (t % kChunk));
+        atomicAdd(&range_cnt[(size_t)(t / kRangeTok) * E + my_e], 1);
+      }
     }
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    bitmap[(size_t)c * E + e] = bm[e];
-    hist[(size_t)c * E + e] = __popc(bm[e]);
-  }
   if (done_ctr == nullptr) return;
-  // the last CTA to finish runs the expert-offset scan over every chunk's
-  // histogram (each writer fences its stores before the arrival count)
+  // the last CTA to finish runs the expert-offset scan (each CTA's atomics
+  // are ordered before its arrival count)
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -251,27 +276,40 @@ __global__ void __launch_bounds__(1024) k_topk_mask(
     s_last = prev == gridDim.x - 1;
   }
   __syncthreads();
-  if (s_last) scan_experts(hist, (int)gridDim.x, E, so);
+  if (s_last) scan_experts(range_cnt, (Tn + kRangeTok - 1) / kRangeTok, E, so);
 }
 
 cudaError_t launch_topk_mask(const float* part, int splitk, int T, int E, int k,
                              const float* bias, const FuseTables& ft, float tau, int renorm,
                              int32_t* idx, float* gate, float* score, uint8_t* keep,
-                             uint32_t* bitmap, int32_t* hist, float* logits_out,
+                             uint32_t* bitmap, int32_t* range_cnt, float* logits_out,
                              uint32_t* status, uint32_t* done_ctr, const ScanOut* so,
                              cudaStream_t s) {
-  dim3 grid(cdiv(T, kChunk));
+  dim3 grid(cdiv(T, kTopkWarps));
   const ScanOut sv = so ? *so : ScanOut{};
   if (so == nullptr) done_ctr = nullptr;
-#define ACE_TOPK(V)                                                                         \
-  k_topk_mask<V><<<grid, kChunk * 32, 0, s>>>(part, splitk, T, E, k, bias, ft, tau, renorm,   \
-                                              idx, gate, score, keep, bitmap, hist,           \
-                                              logits_out, status, done_ctr, sv)
-  if (E <= 32) ACE_TOPK(1);
-  else if (E <= 64) ACE_TOPK(2);
-  else if (E <= 128) ACE_TOPK(4);
-  else if (E <= 256) ACE_TOPK(8);
-  else ACE_TOPK(16);
+#define ACE_TOPK(V)                                                                          \
+  if (splitk > 4)                                                                            \
+    k_topk_mask<V, true><<<grid, kTopkWarps * 32, 0, s>>>(                                   \
+        part, splitk, T, E, k, bias, ft, tau, renorm, idx, gate, score, keep, bitmap,        \
+        range_cnt, logits_out, status, done_ctr, sv);                                        \
+  else                                                                                       \
+    k_topk_mask<V, false><<<grid, kTopkWarps * 32, 0, s>>>(                                  \
+        part, splitk, T, E, k, bias, ft, tau, renorm, idx, gate, score, keep, bitmap,        \
+        range_cnt, logits_out, status, done_ctr, sv)
+  if (E <= 32) {
+    ACE_TOPK(1);
+  } else if (E <= 64) {
+    ACE_TOPK(2);
+  } else if (E <= 128) {
+    ACE_TOPK(4);
+  } else if (E <= 256) {
+    ACE_TOPK(8);
+  } else {  // 16 logits a lane: the shallow form would spill
+    k_topk_mask<16, true><<<grid, kTopkWarps * 32, 0, s>>>(
+        part, splitk, T, E, k, bias, ft, tau, renorm, idx, gate, score, keep, bitmap, range_cnt,
+        logits_out, status, done_ctr, sv);
+  }
 #undef ACE_TOPK
   return cudaGetLastError();
 }
