@@ -46,7 +46,7 @@ struct ScanOut {
   int32_t* counts;   // [E]
   int32_t* offsets;  // [E + 1]
   int32_t* n_kept;   // [1]
-  int4* tiles;       // [max_tiles]
+  int4* tiles;       // [max_tiles]: (expert, first slot, slots, index in expert << 16 | tiles of expert)
   int32_t* n_tiles;  // [1]
   uint32_t* tile_done;  // [max_tiles] or NULL: per-tile counters, zeroed here
   int max_tiles, tile_n;
@@ -86,7 +86,8 @@ __device__ __forceinline__ void scan_experts(const int32_t* range_cnt, int nrang
       const int each = cnt[j] / ntile[j], rem = cnt[j] - each * ntile[j];
       for (int q = 0; q < ntile[j]; ++q)
         if (toff + q < o.max_tiles)
-          o.tiles[toff + q] = make_int4(e, off + q * each + min(q, rem), each + (q < rem ? 1 : 0), 0);
+          o.tiles[toff + q] = make_int4(e, off + q * each + min(q, rem), each + (q < rem ? 1 : 0),
+                                        (q << 16) | ntile[j]);
     }
   }
   if (t == 0) {

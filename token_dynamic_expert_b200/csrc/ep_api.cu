@@ -83,7 +83,8 @@ __global__ void k_tiles_from_offsets(const int32_t* __restrict__ offsets, int E,
     const int each = cnt / ntile, rem = cnt - each * ntile;
     for (int q = 0; q < ntile; ++q)
       if (toff + q < max_tiles)
-        tiles[toff + q] = make_int4(t, off + q * each + min(q, rem), each + (q < rem ? 1 : 0), 0);
+        tiles[toff + q] = make_int4(t, off + q * each + min(q, rem), each + (q < rem ? 1 : 0),
+                                    (q << 16) | ntile);
   }
   if (t == 0) {
     *n_tiles = min(total, max_tiles);

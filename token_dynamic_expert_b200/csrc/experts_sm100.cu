@@ -66,6 +66,23 @@ constexpr int kSmemBytes = 1024 + kStageBudget + kXchgBytes + 512;
 
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
 
+// Item w of a launch of (tile, row block) items.  An expert's tiles sit
+// together in the tile list and each tile entry carries (its index within
+// the expert << 16 | the expert's tile count) in .w, so the items can run
+// row block by row block with the expert's tiles side by side: neighbouring
+// items then stream the same weight rows at the same time, and the second
+// tile of an expert reads them from L2 instead of HBM.
+__device__ __forceinline__ void item_of(const int4* __restrict__ tiles, int n_tiles, int ipt,
+                                        int w, int& ti, int& it) {
+  const int t0 = w / ipt;
+  const int4 a = tiles[t0];
+  const int gs = t0 - min(a.w >> 16, t0);             // the expert's first tile
+  const int gn = max(1, min(a.w & 0xffff, n_tiles - gs));
+  const int l = w - gs * ipt;
+  it = min(l / gn, ipt - 1);
+  ti = gs + l % gn;
+}
+
 __device__ __forceinline__ void epilogue_bar() {
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
@@ -148,7 +165,8 @@ __global__ void __launch_bounds__(kThreads1, 1)
       int stage = 0;
       uint32_t phase = 0, issued = 0, issued_par = 0;
       for (int w = blockIdx.x; w < total && !*abort_flag; w += gridDim.x) {
-        const int ti = w / items_per_tile, it = w - ti * items_per_tile;
+        int ti, it;
+        item_of(tiles, n_tiles, items_per_tile, w, ti, it);
         const int4 tl = tiles[ti];
         const int nbox = (tl.z + kBoxN - 1) / kBoxN;
         const uint32_t bytes = kAStage + nbox * kBoxBytes;
@@ -187,7 +205,9 @@ __global__ void __launch_bounds__(kThreads1, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-        const int4 tl = tiles[w / items_per_tile];
+        int ti, it;
+        item_of(tiles, n_tiles, items_per_tile, w, ti, it);
+        const int4 tl = tiles[ti];
         const int npad = (tl.z + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(kBM, npad);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, status, abort_flag)) break;
@@ -229,7 +249,8 @@ __global__ void __launch_bounds__(kThreads1, 1)
     uint32_t acc_phase = 0;
     int xb = 0;  // exchange buffer parity (MODE 0)
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
-      const int ti = w / items_per_tile, it = w - ti * items_per_tile;
+      int ti, it;
+      item_of(tiles, n_tiles, items_per_tile, w, ti, it);
       const int4 tl = tiles[ti];
       const int row0 = tl.y, n = tl.z;
       if (!mbar_wait(&tfull[acc], acc_phase, status, abort_flag)) break;
@@ -442,7 +463,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int w = pair; w < total && !*abort_flag; w += npairs) {
-        const int ti = w / items_per_tile, it = w - ti * items_per_tile;
+        int ti, it;
+        item_of(tiles, n_tiles, items_per_tile, w, ti, it);
         const int4 tl = tiles[ti];
         const int half = ((tl.z + 15) & ~15) / 2;
         const int nbox = (half + kBoxN - 1) / kBoxN;
@@ -477,7 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int w = pair; w < total && ok; w += npairs) {
-        const int4 tl = tiles[w / items_per_tile];
+        int ti, it;
+        item_of(tiles, n_tiles, items_per_tile, w, ti, it);
+        const int4 tl = tiles[ti];
         const int npad = (tl.z + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(2 * kBM, npad);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, status, abort_flag)) break;
@@ -520,7 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     int xb = 0;
     for (int w = pair; w < total; w += npairs) {
-      const int ti = w / items_per_tile, it = w - ti * items_per_tile;
+      int ti, it;
+      item_of(tiles, n_tiles, items_per_tile, w, ti, it);
       const int4 tl = tiles[ti];
       const int row0 = tl.y, n = tl.z;
       if (!mbar_wait(&tfull[acc], acc_phase, status, abort_flag)) break;
