@@ -40,7 +40,7 @@ METRIC = "MoE-layer tokens/s (prefill, decode) at skip rate; % of tensor/HBM roo
 # is the revision the counters were taken on.
 PROFILED_TRAFFIC = {
     ("prefill_1024", "fused"): ("token_dynamic_expert_b200/csrc/experts_fused_sm100.cu",
-                                "179ca8325236", 1229559016),
+                                "10553744e735", 1227740736),
 }
 
 
