@@ -64,6 +64,7 @@ FwdLayout fwd_layout(const ace_layer& L, int max_tokens, int num_sms) {
   o.status = take(256);
   o.part = take(part * 4);
   o.inv_rms = take(T * 4);
+  o.rw3 = take(L.dtype == ACE_BF16 ? 3 * E * d * 2 : 0);  // gamma-folded router rows, 3 terms
   o.idx = take(cap * 4);
   o.gate = take(cap * 4);
   o.score = take(cap * 4);
@@ -187,9 +188,10 @@ ace_status run_routing(const ace_layer& L, const void* u, int T, const ace_fwd_o
   const bool tc = L.dtype == ACE_BF16;
   const size_t n_zero = ((size_t)cdiv(T, kChunk) + (size_t)cdiv(T, kRangeTok)) * (size_t)L.E;
   ACE_CK(launch_rmsnorm(L.dtype, u, T, L.d, L.gamma, o.eps_rms, at<float>(ws, ly.inv_rms), x_out,
-                        clr.p, clr.n, at<uint32_t>(ws, ly.bitmap), n_zero, s));
+                        clr.p, clr.n, at<uint32_t>(ws, ly.bitmap), n_zero, L.w_router, L.E,
+                        tc ? at<void>(ws, ly.rw3) : nullptr, s));
   if (tc)
-    ACE_CK(launch_router_tc(u, at<float>(ws, ly.inv_rms), L.gamma, L.w_router, T, L.d, L.E,
+    ACE_CK(launch_router_tc(u, at<float>(ws, ly.inv_rms), at<void>(ws, ly.rw3), T, L.d, L.E,
                             splitk, at<float>(ws, ly.part), at<uint32_t>(ws, ly.status), num_sms,
                             s));
   else

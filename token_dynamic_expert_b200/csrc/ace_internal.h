@@ -34,7 +34,7 @@ int router_splits_for(const ace_layer& L, int T, int num_sms);
 // Byte offsets of the forward's scratch arrays inside the caller's
 // workspace.  Everything is sized for max_tokens and no skipping.
 struct FwdLayout {
-  size_t status, part, inv_rms, tile_done, idx, gate, score, keep, bitmap, range_cnt, rbase,
+  size_t status, part, inv_rms, rw3, tile_done, idx, gate, score, keep, bitmap, range_cnt, rbase,
       counts,
       offsets, n_kept, tiles, n_tiles, slot_token, slot_rank, slot_gate, slot_of, xp, h,
       yslot, total;
@@ -56,16 +56,18 @@ ace_status check_fusion(const ace_layer& L, int fusion);
 
 // ---------------------------------------------------------------- launchers
 // 1/rms per token, x (nullable); zeroes clear[0 .. n_clear) (n_clear <= 256)
-// and zero[0 .. n_zero)
+// and zero[0 .. n_zero); w3 (nullable, bf16 layers): gamma (.) w_router as
+// three bf16 terms [3][E][d]
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
                            float eps, float* inv_rms, void* x, uint32_t* clear, int n_clear,
-                           uint32_t* zero, size_t n_zero, cudaStream_t s);
+                           uint32_t* zero, size_t n_zero, const void* wr, int E, void* w3,
+                           cudaStream_t s);
 // Tensor-core router (bf16 layers): part[split][t][e] from u [T][d] (bf16),
-// 1/rms, gamma and w_router [E][d].
+// 1/rms and the three-term router operand w3 [3][E][d].
 int router_tc_splits(int T, int d, int E, int num_sms);
-cudaError_t launch_router_tc(const void* u, const float* inv_rms, const float* gamma,
-                             const void* wr, int T, int d, int E, int splits, float* part,
-                             uint32_t* status, int num_sms, cudaStream_t s);
+cudaError_t launch_router_tc(const void* u, const float* inv_rms, const void* w3, int T, int d,
+                             int E, int splits, float* part, uint32_t* status, int num_sms,
+                             cudaStream_t s);
 cudaError_t launch_router_logits(ace_dtype dt, const void* u, const float* inv_rms,
                                  const float* gamma, const void* wr, int T, int d, int E,
                                  int splitk, float* part, cudaStream_t s);

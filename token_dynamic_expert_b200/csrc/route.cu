@@ -30,18 +30,49 @@ namespace ace {
 // x (nullable) receives xhat(u, 1/rms, gamma) rounded to the storage type.
 // As the forward's first kernel it also zeroes the call's status words
 // (clear[0 .. n_clear)) and the top-k kernel's bitmaps and range counts
-// (zero[0 .. n_zero)), which no kernel of the forward touches before it.
+// (zero[0 .. n_zero)), which no kernel of the forward touches before it, and
+// (w3 non-null, bf16 layers) forms the tensor-core router's operand: the
+// router rows with gamma folded in, w'_ek = gamma_k w_ek in fp32, as three
+// bf16 terms hi + mid + lo (each the rounding of what the previous terms
+// leave) at w3[term * E + e][k].
 template <typename T>
 __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn, int d,
                                                  const float* __restrict__ gamma, float eps,
                                                  float* __restrict__ inv_rms, T* __restrict__ x,
                                                  uint32_t* __restrict__ clear, int n_clear,
-                                                 uint32_t* __restrict__ zero, size_t n_zero) {
+                                                 uint32_t* __restrict__ zero, size_t n_zero,
+                                                 const __nv_bfloat16* __restrict__ wr, int E,
+                                                 __nv_bfloat16* __restrict__ w3) {
   constexpr int V = 16 / sizeof(T);
   if (blockIdx.x == 0 && (int)threadIdx.x < n_clear) clear[threadIdx.x] = 0u;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_zero;
        i += (size_t)gridDim.x * blockDim.x)
     zero[i] = 0u;
+  if (w3 != nullptr) {
+    const int vpr = d / 8;
+    const size_t nvec = (size_t)E * vpr;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < nvec;
+         i += (size_t)gridDim.x * blockDim.x) {
+      const int e = (int)(i / vpr), v = (int)(i - (size_t)e * vpr);
+      const uint4 q = reinterpret_cast<const uint4*>(wr + (size_t)e * d)[v];
+      const __nv_bfloat16* wv = reinterpret_cast<const __nv_bfloat16*>(&q);
+      uint4 oh, om, ol;
+      __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(&oh);
+      __nv_bfloat16* mi = reinterpret_cast<__nv_bfloat16*>(&om);
+      __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(&ol);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float wf = __fmul_rn(gamma[v * 8 + c], __bfloat162float(wv[c]));
+        h[c] = __float2bfloat16_rn(wf);
+        const float r1 = __fsub_rn(wf, __bfloat162float(h[c]));
+        mi[c] = __float2bfloat16_rn(r1);
+        lo[c] = __float2bfloat16_rn(__fsub_rn(r1, __bfloat162float(mi[c])));
+      }
+      reinterpret_cast<uint4*>(w3 + (size_t)e * d)[v] = oh;
+      reinterpret_cast<uint4*>(w3 + (size_t)(E + e) * d)[v] = om;
+      reinterpret_cast<uint4*>(w3 + (size_t)(2 * E + e) * d)[v] = ol;
+    }
+  }
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= Tn) return;
@@ -75,16 +106,17 @@ __global__ void __launch_bounds__(256) k_rmsnorm(const T* __restrict__ u, int Tn
 
 cudaError_t launch_rmsnorm(ace_dtype dt, const void* u, int T, int d, const float* gamma,
                            float eps, float* inv_rms, void* x, uint32_t* clear, int n_clear,
-                           uint32_t* zero, size_t n_zero, cudaStream_t s) {
+                           uint32_t* zero, size_t n_zero, const void* wr, int E, void* w3,
+                           cudaStream_t s) {
   dim3 grid(cdiv(T, 8));
   if (n_clear > 256) return cudaErrorInvalidValue;
   if (dt == ACE_BF16)
-    k_rmsnorm<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)u, T, d, gamma, eps,
-                                                  inv_rms, (__nv_bfloat16*)x, clear, n_clear,
-                                                  zero, n_zero);
+    k_rmsnorm<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        (const __nv_bfloat16*)u, T, d, gamma, eps, inv_rms, (__nv_bfloat16*)x, clear, n_clear,
+        zero, n_zero, (const __nv_bfloat16*)wr, E, (__nv_bfloat16*)w3);
   else
     k_rmsnorm<float><<<grid, 256, 0, s>>>((const float*)u, T, d, gamma, eps, inv_rms, (float*)x,
-                                          clear, n_clear, zero, n_zero);
+                                          clear, n_clear, zero, n_zero, nullptr, 0, nullptr);
   return cudaGetLastError();
 }
 

@@ -3,25 +3,25 @@
 //
 // The logits decide the top-k and, through the gates, the skip mask, so they
 // must carry fp32 precision ([ACE] "3. Conservative Fusion": a slot is
-// skipped by comparing g * A against tau).  x (fp32) enters as three bf16
-// terms x = hi + mid + lo (each the round-to-nearest of the remainder, 24
-// significant bits together) and the router rows are bf16, so every product
-// is exact in fp32.  A long tensor-core accumulation would still lose low
-// bits, so the sum is cut into 64-column chunks: per chunk, 12 MMAs
-// (3 terms x 4 K-steps of 16) accumulate into a fresh TMEM buffer, and the
-// epilogue adds the chunk result into fp32 registers.  The error is then that
-// of an fp32 sum over 32 chunk values.
-//
-// The terms are formed in shared memory, not read from HBM: TMA brings the
-// 128 x 64 tile of the layer input u (bf16), and six transform warps turn
-// it in place into x = xhat(u, 1/rms, gamma) and its three terms, then hand
-// the stage to the MMA issuer.  HBM traffic is u itself, once.
+// skipped by comparing g * A against tau).  With x_t = r_t (u_t (.) gamma) and
+// r_t = 1 / rms(u_t) ([ACE] "Theoretical Foundation"), the logit is
+//   l_te = r_t * sum_k u_tk (gamma_k w_ek),
+// so gamma is folded into the router rows: w'_ek = gamma_k w_ek in fp32 enters
+// as three bf16 terms w' = hi + mid + lo (each the round-to-nearest of what
+// the previous terms leave, 24 significant bits together; RMSNorm forms them
+// for the call), and u is bf16, so every product u_tk * term is exact in fp32.
+// A long tensor-core accumulation would still lose low bits, so the sum is cut
+// into 64-column chunks: per chunk, 12 MMAs (3 terms x 4 K-steps of 16)
+// accumulate into a fresh TMEM buffer, and the epilogue adds the chunk result
+// into fp32 registers.  The error is then that of an fp32 sum over the chunk
+// values.  The epilogue multiplies each token's sum by r_t.
 //
 // Tile: 128 tokens (MMA M) x 128 experts (N), K split into `splits` ranges
 // whose fp32 partial sums part[split][t][e] the top-k kernel adds in split
-// order.  Warps: 0 TMA producer, 1 MMA issuer (TMEM allocator), 2..9
-// epilogue (two warps per TMEM lane quarter, 64 columns each), 10..15
-// transform.  Two TMEM buffers of 128 columns alternate between chunks.
+// order.  A stage is the 128 x 64 u tile and the three 128 x 64 term tiles of
+// the tile's router rows, one TMA box each.  Warps: 0 TMA producer, 1 MMA
+// issuer (TMEM allocator), 2..9 epilogue (two warps per TMEM lane quarter, 64
+// columns each).  Two TMEM buffers of 128 columns alternate between chunks.
 // Bounded waits throughout.
 #include "ace_common.cuh"
 #include "ace_internal.h"
@@ -30,28 +30,24 @@ namespace ace {
 namespace {
 
 constexpr int rBM = 128, rBN = 128, rBK = 64, rNS = 3;
-constexpr int rATile = rBM * rBK * 2;           // 16 KB per term
-constexpr int rBTile = rBN * rBK * 2;           // 16 KB
-constexpr int rStage = 3 * rATile + rBTile;     // 64 KB
+constexpr int rATile = rBM * rBK * 2;           // 16 KB: u
+constexpr int rBTile = rBN * rBK * 2;           // 16 KB per term
+constexpr int rStage = rATile + 3 * rBTile;     // 64 KB
 constexpr int rSmem = 1024 + rNS * rStage + 256;
-// 16 warps (4 per SM sub-partition) leave 128 registers a thread: the
-// epilogue keeps its 64 running sums in registers
-constexpr int rThreads = 512;
-constexpr int rTransformWarp0 = 10, rTransformThreads = 192;
+constexpr int rThreads = 320;
 constexpr uint32_t rTmemCols = 256;
 
 __global__ void __launch_bounds__(rThreads, 1)
     k_router_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const float* __restrict__ inv_rms, const float* __restrict__ gamma, int Tn, int d,
-                int E, int splits, float* __restrict__ part, uint32_t* status) {
+                const float* __restrict__ inv_rms, int Tn, int d, int E, int splits,
+                float* __restrict__ part, uint32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + rNS * rStage);
-  uint64_t* raw = bars;           // TMA bytes of u and the router rows landed
-  uint64_t* full = bars + rNS;    // the three terms are formed
-  uint64_t* empty = bars + 2 * rNS;
-  uint64_t* tfull = bars + 3 * rNS;
+  uint64_t* full = bars;
+  uint64_t* empty = bars + rNS;
+  uint64_t* tfull = bars + 2 * rNS;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -65,8 +61,7 @@ __global__ void __launch_bounds__(rThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < rNS; ++s) {
-      mbar_init(&raw[s], 1);
-      mbar_init(&full[s], rTransformThreads);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -101,9 +96,12 @@ __global__ void __launch_bounds__(rThreads, 1)
         for (int c = s * cps; c < (s + 1) * cps; ++c) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, status, abort_flag)) break;
           uint8_t* st = smem + stage * rStage;
-          mbar_expect_tx(&raw[stage], rATile + rBTile);
-          tma_load_2d(st, &tmA, c * rBK, mt * rBM, &raw[stage], pol);
-          tma_load_2d(st + 3 * rATile, &tmB, c * rBK, nt * rBN, &raw[stage], pol);
+          mbar_expect_tx(&full[stage], rStage);
+          tma_load_2d(st, &tmA, c * rBK, mt * rBM, &full[stage], pol);
+#pragma unroll
+          for (int term = 0; term < 3; ++term)  // the term blocks are E rows apart
+            tma_load_2d(st + rATile + term * rBTile, &tmB, c * rBK, term * E + nt * rBN,
+                        &full[stage], pol);
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
           if (++stage == rNS) {
@@ -116,7 +114,7 @@ __global__ void __launch_bounds__(rThreads, 1)
         for (int s = 0; s < rNS; ++s)
           if ((issued >> s) & 1u) {
             const uint64_t t0 = global_ns();
-            while (!mbar_try_wait(&raw[s], (issued_par >> s) & 1u))
+            while (!mbar_try_wait(&full[s], (issued_par >> s) & 1u))
               if (global_ns() - t0 > kWaitLimitNs) break;
           }
       }
@@ -139,7 +137,7 @@ __global__ void __launch_bounds__(rThreads, 1)
           }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + stage * rStage);
-          const uint32_t b0 = a0 + 3 * rATile;
+          const uint32_t b0 = a0 + rATile;
           const uint32_t dcol = tmem + buf * (uint32_t)rBN;
           // smallest term first: the accumulator stays small while the low
           // terms are added
@@ -147,8 +145,9 @@ __global__ void __launch_bounds__(rThreads, 1)
           for (int ti = 0; ti < 3; ++ti)
 #pragma unroll
             for (int kk = 0; kk < rBK / 16; ++kk)
-              mma_bf16(dcol, sw128_kmajor_desc(a0 + (2 - ti) * rATile + kk * 32),
-                       sw128_kmajor_desc(b0 + kk * 32), idesc, (ti | kk) != 0);
+              mma_bf16(dcol, sw128_kmajor_desc(a0 + kk * 32),
+                       sw128_kmajor_desc(b0 + (2 - ti) * rBTile + kk * 32), idesc,
+                       (ti | kk) != 0);
           mma_commit(&empty[stage]);
           mma_commit(&tfull[buf]);
           if (++stage == rNS) {
@@ -161,66 +160,6 @@ __global__ void __launch_bounds__(rThreads, 1)
       const uint64_t t0 = global_ns();
       while (!mbar_try_wait(drain, 0))
         if (global_ns() - t0 > kWaitLimitNs) break;
-    }
-  } else if (warp >= rTransformWarp0) {
-    // ---------------------------------------------------------- transform
-    // Thread j takes the 16-byte chunks j + 192 i (i < 6, below 1024) of the
-    // 128 x 64 tile: rows r = (j >> 3) + 24 i, physical chunk p = j & 7.  The
-    // 128-byte swizzle fills chunk p of row r with the columns of logical
-    // chunk p ^ (r & 7), the same for all of a thread's rows, so a thread
-    // needs the 8 gamma values of one chunk per stage.  hi is written over u;
-    // mid and lo go to the same places of their tiles.
-    const int j = (int)threadIdx.x - rTransformWarp0 * 32;
-    const int p = j & 7, lc = p ^ ((j >> 3) & 7);
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-      const int s = w % splits, mt = w / (splits * nt_n);
-      for (int c = s * cps; c < (s + 1) * cps; ++c) {
-        const float4 g0 = *reinterpret_cast<const float4*>(gamma + c * rBK + 8 * lc);
-        const float4 g1 = *reinterpret_cast<const float4*>(gamma + c * rBK + 8 * lc + 4);
-        const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-        if (!mbar_wait(&raw[stage], phase, status, abort_flag)) {
-          ok = false;
-          break;
-        }
-        uint8_t* st = smem + stage * rStage;
-#pragma unroll 2
-        for (int i = 0; i < 6; ++i) {
-          if (i == 5 && j >= 64) break;  // 1024 chunks: the sixth round has 64
-          const int r = (j >> 3) + 24 * i, t = mt * rBM + r;
-          const float rv = t < Tn ? __ldg(inv_rms + t) : 0.f;  // rows past the end: TMA zeros
-          const int off = r * 128 + p * 16;
-          const uint4 q = *reinterpret_cast<const uint4*>(st + off);
-          const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&q);
-          uint4 oh, om, ol;
-          __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&oh);
-          __nv_bfloat162* mi = reinterpret_cast<__nv_bfloat162*>(&om);
-          __nv_bfloat162* lo = reinterpret_cast<__nv_bfloat162*>(&ol);
-#pragma unroll
-          for (int pr = 0; pr < 4; ++pr) {
-            const float2 uf = __bfloat1622float2(e[pr]);
-            const float x0 = xhat(uf.x, rv, g[2 * pr]), x1 = xhat(uf.y, rv, g[2 * pr + 1]);
-            h[pr] = __floats2bfloat162_rn(x0, x1);
-            const float2 hf = __bfloat1622float2(h[pr]);
-            const float r0 = __fsub_rn(x0, hf.x), r1 = __fsub_rn(x1, hf.y);
-            mi[pr] = __floats2bfloat162_rn(r0, r1);
-            const float2 mf = __bfloat1622float2(mi[pr]);
-            lo[pr] = __floats2bfloat162_rn(__fsub_rn(r0, mf.x), __fsub_rn(r1, mf.y));
-          }
-          *reinterpret_cast<uint4*>(st + off) = oh;
-          *reinterpret_cast<uint4*>(st + rATile + off) = om;
-          *reinterpret_cast<uint4*>(st + 2 * rATile + off) = ol;
-        }
-        // the MMA reads these tiles through the async proxy
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(&full[stage]);
-        if (++stage == rNS) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
     }
   } else {
     // ----------------------------------------------------------- epilogue
@@ -243,14 +182,14 @@ __global__ void __launch_bounds__(rThreads, 1)
         }
         tc_fence_after();
         const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + buf * (uint32_t)rBN + half * 64;
+        float v[4][16];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {  // one load per wait: registers stay under the cap
-          float v[16];
-          tmem_ld16(tb + g * 16, v);
-          tmem_ld_wait();
+        for (int g = 0; g < 4; ++g) tmem_ld16(tb + g * 16, v[g]);
+        tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) acc[g * 16 + j] += v[j];
-        }
+        for (int g = 0; g < 4; ++g)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc[g * 16 + j] += v[g][j];
         tc_fence_before();
         mbar_arrive(&tempty[buf]);
       }
@@ -258,16 +197,17 @@ __global__ void __launch_bounds__(rThreads, 1)
       const int t = mt * rBM + row;
       const int e0 = nt * rBN + half * 64;
       if (t < Tn) {
+        const float r = inv_rms[t];
         float* out = part + ((size_t)s * Tn + t) * E;
         if (e0 + 64 <= E && (E % 4) == 0) {
 #pragma unroll
           for (int j = 0; j < 64; j += 4)
             *reinterpret_cast<float4*>(out + e0 + j) =
-                make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                make_float4(r * acc[j], r * acc[j + 1], r * acc[j + 2], r * acc[j + 3]);
         } else {
 #pragma unroll
           for (int j = 0; j < 64; ++j)
-            if (e0 + j < E) out[e0 + j] = acc[j];
+            if (e0 + j < E) out[e0 + j] = r * acc[j];
         }
       }
     }
@@ -314,12 +254,12 @@ int router_tc_splits(int T, int d, int E, int num_sms) {
   return s;
 }
 
-cudaError_t launch_router_tc(const void* u, const float* inv_rms, const float* gamma,
-                             const void* wr, int T, int d, int E, int splits, float* part,
-                             uint32_t* status, int num_sms, cudaStream_t s) {
+cudaError_t launch_router_tc(const void* u, const float* inv_rms, const void* w3, int T, int d,
+                             int E, int splits, float* part, uint32_t* status, int num_sms,
+                             cudaStream_t s) {
   CUtensorMap ma, mb;
   if (!rmap(&ma, u, (uint64_t)T, (uint64_t)d, rBM) ||
-      !rmap(&mb, wr, (uint64_t)E, (uint64_t)d, rBN))
+      !rmap(&mb, w3, (uint64_t)3 * E, (uint64_t)d, rBN))
     return cudaErrorInvalidValue;
   static bool attr = false;
   if (!attr) {
@@ -330,8 +270,7 @@ cudaError_t launch_router_tc(const void* u, const float* inv_rms, const float* g
   }
   const int items = cdiv(T, rBM) * cdiv(E, rBN) * splits;
   const int grid = items < num_sms ? items : num_sms;
-  k_router_tc<<<grid, rThreads, rSmem, s>>>(ma, mb, inv_rms, gamma, T, d, E, splits, part,
-                                            status);
+  k_router_tc<<<grid, rThreads, rSmem, s>>>(ma, mb, inv_rms, T, d, E, splits, part, status);
   return cudaGetLastError();
 }
 
