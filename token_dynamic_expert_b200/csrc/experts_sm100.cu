@@ -54,13 +54,17 @@ constexpr int kAStage = kBM * kBK * 2;      // 16 KB
 constexpr int kBoxBytes = kBoxN * kBK * 2;  // 8 KB
 constexpr int kMaxStages = 8;
 constexpr int kStageBudget = 200 * 1024;
-constexpr int kXchgBytes = 2 * 2 * 64 * 8 * 4;  // 2 buffers x (gate, up) x 64 rows x 8 floats
-constexpr int kThreads = 192;               // the CTA-pair kernel: 4 epilogue warps
-// The one-CTA kernel (the down GEMM) has 8 epilogue warps, two per TMEM lane
-// quarter taking alternate 16-slot groups: its epilogue (a bf16 store per slot
-// and output column) is the slower side of its pipeline.
+// per epilogue group: 2 buffers x (gate, up) x 64 rows x 8 floats; two groups
+constexpr int kXchgGroupFloats = 2 * 2 * 64 * 8;
+constexpr int kXchgBytes = 2 * kXchgGroupFloats * 4;
+// 8 epilogue warps, two per TMEM lane quarter taking alternate 16-slot groups
+// (in the gate/up epilogue each group of four pairs gate with up values
+// through its own exchange buffers and named barrier): the epilogue (a bf16
+// store per slot and output column) is the slower side of the pipeline.
+// The one-CTA gate/up form keeps 4.
 constexpr int kEpiWarps1 = 8;
 constexpr int kThreads1 = 64 + 32 * kEpiWarps1;
+constexpr int kThreads = kThreads1;  // the CTA-pair kernel
 constexpr uint32_t kTmemCols = 512;         // two accumulators of 256 columns
 constexpr int kSmemBytes = 1024 + kStageBudget + kXchgBytes + 512;
 
@@ -83,8 +87,9 @@ __device__ __forceinline__ void item_of(const int4* __restrict__ tiles, int n_ti
   ti = gs + l % gn;
 }
 
-__device__ __forceinline__ void epilogue_bar() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+// named barrier of one group of four epilogue warps (ids 1 and 2)
+__device__ __forceinline__ void epilogue_bar(int group) {
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + group) : "memory");
 }
 
 template <int MODE>
@@ -271,7 +276,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
           const int off = is_gate ? 8 : 0;
           mine[0] = make_float4(v[off + 0], v[off + 1], v[off + 2], v[off + 3]);
           mine[1] = make_float4(v[off + 4], v[off + 5], v[off + 6], v[off + 7]);
-          epilogue_bar();
+          epilogue_bar(0);
           const float4* other = reinterpret_cast<const float4*>((is_gate ? xu : xg) + r * 8);
           const float4 o0 = other[0], o1 = other[1];
           const float ov[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
@@ -419,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 2 * 128);  // both CTAs' epilogue threads (the leader's copy counts)
+      mbar_init(&tempty[a], 2 * 32 * kEpiWarps1);  // both CTAs' epilogue threads (the leader's copy counts)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -539,7 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ----------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    const int q = warp & 3;           // TMEM lane quarter this warp may read
+    const int grp = (warp - 2) >> 2;  // its group: alternate 16-slot column groups
     int acc = 0;
     uint32_t acc_phase = 0;
     int xb = 0;
@@ -556,17 +562,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = (q & 1) * 32 + lane;
         const int col = it * 128 + (int)rank * 64 + r;
         __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(out);
-        for (int c0 = 0; c0 < n; c0 += 16) {
+        for (int c0 = grp * 16; c0 < n; c0 += 32) {
           float v[16];
           tmem_ld16(tbase + (uint32_t)c0, v);
           tmem_ld_wait();
-          float* xg = xchg + xb * 1024;
+          float* xg = xchg + grp * kXchgGroupFloats + xb * 1024;
           float* xu = xg + 512;
           float4* mine = reinterpret_cast<float4*>((is_gate ? xg : xu) + r * 8);
           const int off = is_gate ? 8 : 0;
           mine[0] = make_float4(v[off + 0], v[off + 1], v[off + 2], v[off + 3]);
           mine[1] = make_float4(v[off + 4], v[off + 5], v[off + 6], v[off + 7]);
-          epilogue_bar();
+          epilogue_bar(grp);
           const float4* other = reinterpret_cast<const float4*>((is_gate ? xu : xg) + r * 8);
           const float4 o0 = other[0], o1 = other[1];
           const float ov[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
@@ -583,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         const int col = it * 256 + (int)rank * kBM + q * 32 + lane;
         __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(out);
-        for (int c0 = 0; c0 < n; c0 += 16) {
+        for (int c0 = grp * 16; c0 < n; c0 += 32) {
           float v[16];
           tmem_ld16(tbase + (uint32_t)c0, v);
           tmem_ld_wait();
