@@ -717,10 +717,10 @@ cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* 
     return cudaErrorInvalidValue;
   cudaError_t e;
   // gate/up on CTA pairs: items of 128 intermediate columns (m % 128 == 0
-  // for bf16 layers).  Down stays on single CTAs: its epilogue (fp32 slot
-  // rows) is heavier and the pair form measured slower there (0.193 vs
-  // 0.209 ms at 4096 tokens, 0% skip), while gate/up gained a little
-  // (0.301 vs 0.296 ms).
+  // for bf16 layers).  Down stays on single CTAs: the pair form measured
+  // slower there, with 8 epilogue warps and bf16 outputs too (0.185 vs
+  // 0.158 ms at 8192 tokens, 256 experts; 0.173 vs 0.156 ms at 4096
+  // tokens, 0% skip).
   if ((e = launch_pair<0>(mg, mu, mx, tiles, n_tiles, max_tiles, L.m, L.d, L.m / 128, L.m, h,
                           L.m, slot_gate, status, num_sms, s)) != cudaSuccess)
     return e;
