@@ -77,6 +77,18 @@ def test_bf16_small_layers_oracle_tables(w):
     assert res["compared_tokens"] >= w.T - 2
 
 
+@pytest.mark.parametrize("E,T,d", [(320, 200, 512), (256, 160, 512), (96, 2000, 256)])
+def test_bf16_many_experts_topk_forms(E, T, d):
+    """The top-k kernel's forms: 257-512 experts (16 logits a lane), 256 experts
+    at a short token count (8 router splits: all of a lane's split loads in
+    flight at once) and 96 experts at a long one (4 splits: the 64-register
+    form), each against the oracle's routing, mask, slot lists and outputs."""
+    w = W("many_experts", T=T, d=d, E=E, m=128, k=8, dtype="bf16", bias=True, skip=0.5,
+          skip_of="slots")
+    res, gpu = _check(w, tables="spread")
+    assert res["compared_tokens"] >= T - 4
+
+
 def test_bf16_expert_with_several_slot_tiles():
     """8 experts, top-2, 1100 tokens: ~275 slots per expert, so every expert
     spans two tiles of ~138 slots."""
