@@ -54,41 +54,95 @@ struct ScanOut {
 
 // Whole-CTA routine (every thread calls it; blockDim.x a multiple of 32 and
 // at least E / 2).  range_cnt [nrange][E] is read with L2-coherent loads
-// (other CTAs' atomics built it).  Thread i takes experts 2i and 2i + 1, so
-// the exclusive scan over experts runs over per-thread pairs.  An expert of
-// n kept slots gets ceil(n / tile_n) tiles of near-equal size (they differ
-// by one slot at most), in slot order.
+// (other CTAs' atomics built it).  With E <= blockDim.x thread i takes expert
+// i and keeps the first kRegRanges of its range counts in registers, so each
+// pass is one round of loads; otherwise thread i takes experts 2i and 2i + 1
+// and the exclusive scan over experts runs over per-thread pairs.  An expert
+// of n kept slots gets ceil(n / tile_n) tiles of near-equal size (they differ
+// by one slot at most), in slot order, each tagged with its index within the
+// expert and the expert's tile count.
+constexpr int kRegRanges = 32;
+
+__device__ __forceinline__ void write_tiles(const ScanOut& o, int e, int off, int cnt, int ntile,
+                                            int toff) {
+  if (ntile <= 0) return;
+  const int each = cnt / ntile, rem = cnt - each * ntile;
+  for (int q = 0; q < ntile; ++q)
+    if (toff + q < o.max_tiles)
+      o.tiles[toff + q] = make_int4(e, off + q * each + min(q, rem), each + (q < rem ? 1 : 0),
+                                    (q << 16) | ntile);
+}
+
 __device__ __forceinline__ void scan_experts(const int32_t* range_cnt, int nrange, int E,
                                              const ScanOut& o) {
   __shared__ int s_warp[32];
   const int t = threadIdx.x;
-  const int e0 = 2 * t;
-  int cnt[2] = {0, 0};
-#pragma unroll 16
-  for (int r = 0; r < nrange; ++r)
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-      if (e0 + j < E) cnt[j] += __ldcg(range_cnt + (size_t)r * E + e0 + j);
   int total, total_tiles;
-  const int off0 = block_excl_scan(cnt[0] + cnt[1], s_warp, &total);
-  int ntile[2];
+  if (E <= (int)blockDim.x) {
+    const bool on = t < E;
+    int rc[kRegRanges];
+    int cnt = 0;
 #pragma unroll
-  for (int j = 0; j < 2; ++j) ntile[j] = e0 + j < E ? (cnt[j] + o.tile_n - 1) / o.tile_n : 0;
-  const int toff0 = block_excl_scan(ntile[0] + ntile[1], s_warp, &total_tiles);
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int e = e0 + j;
-    if (e >= E) continue;
-    const int off = off0 + (j ? cnt[0] : 0), toff = toff0 + (j ? ntile[0] : 0);
-    o.counts[e] = cnt[j];
-    o.offsets[e] = off;
-    if (ntile[j] > 0) {
-      const int each = cnt[j] / ntile[j], rem = cnt[j] - each * ntile[j];
-      for (int q = 0; q < ntile[j]; ++q)
-        if (toff + q < o.max_tiles)
-          o.tiles[toff + q] = make_int4(e, off + q * each + min(q, rem), each + (q < rem ? 1 : 0),
-                                        (q << 16) | ntile[j]);
+    for (int r = 0; r < kRegRanges; ++r) {
+      rc[r] = (on && r < nrange) ? __ldcg(range_cnt + (size_t)r * E + t) : 0;
+      cnt += rc[r];
     }
+    for (int r = kRegRanges; r < nrange; ++r)
+      if (on) cnt += __ldcg(range_cnt + (size_t)r * E + t);
+    const int off = block_excl_scan(cnt, s_warp, &total);
+    const int ntile = on ? (cnt + o.tile_n - 1) / o.tile_n : 0;
+    const int toff = block_excl_scan(ntile, s_warp, &total_tiles);
+    if (on) {
+      o.counts[t] = cnt;
+      o.offsets[t] = off;
+      write_tiles(o, t, off, cnt, ntile, toff);
+      int run = off;
+#pragma unroll
+      for (int r = 0; r < kRegRanges; ++r)
+        if (r < nrange) {
+          o.rbase[(size_t)r * E + t] = run;
+          run += rc[r];
+        }
+      for (int r = kRegRanges; r < nrange; ++r) {
+        const size_t at = (size_t)r * E + t;
+        const int c = __ldcg(range_cnt + at);
+        o.rbase[at] = run;
+        run += c;
+      }
+    }
+  } else {
+    const int e0 = 2 * t;
+    int cnt[2] = {0, 0};
+#pragma unroll 16
+    for (int r = 0; r < nrange; ++r)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        if (e0 + j < E) cnt[j] += __ldcg(range_cnt + (size_t)r * E + e0 + j);
+    const int off0 = block_excl_scan(cnt[0] + cnt[1], s_warp, &total);
+    int ntile[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) ntile[j] = e0 + j < E ? (cnt[j] + o.tile_n - 1) / o.tile_n : 0;
+    const int toff0 = block_excl_scan(ntile[0] + ntile[1], s_warp, &total_tiles);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int e = e0 + j;
+      if (e >= E) continue;
+      const int off = off0 + (j ? cnt[0] : 0);
+      o.counts[e] = cnt[j];
+      o.offsets[e] = off;
+      write_tiles(o, e, off, cnt[j], ntile[j], toff0 + (j ? ntile[0] : 0));
+    }
+    int run[2] = {off0, off0 + cnt[0]};
+#pragma unroll 8
+    for (int r = 0; r < nrange; ++r)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        if (e0 + j < E) {
+          const size_t at = (size_t)r * E + e0 + j;
+          const int c = __ldcg(range_cnt + at);
+          o.rbase[at] = run[j];
+          run[j] += c;
+        }
   }
   if (t == 0) {
     o.offsets[E] = total;
@@ -97,18 +151,6 @@ __device__ __forceinline__ void scan_experts(const int32_t* range_cnt, int nrang
   }
   if (o.tile_done)
     for (int i = t; i < o.max_tiles; i += blockDim.x) o.tile_done[i] = 0u;
-  // range bases
-  int run[2] = {off0, off0 + cnt[0]};
-#pragma unroll 8
-  for (int r = 0; r < nrange; ++r)
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-      if (e0 + j < E) {
-        const size_t at = (size_t)r * E + e0 + j;
-        const int c = __ldcg(range_cnt + at);
-        o.rbase[at] = run[j];
-        run[j] += c;
-      }
 }
 
 }  // namespace ace
