@@ -387,7 +387,8 @@ __device__ __forceinline__ void arrive_on_leader(uint64_t* bar) {
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     k_experts_pair(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                   const __grid_constant__ CUtensorMap tmB, const int4* __restrict__ tiles,
+                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
+                   const int4* __restrict__ tiles,
                    const int32_t* __restrict__ n_tiles_ptr, int max_tiles, int rows_per_expert,
                    int K, int items_per_tile, int out_rows, void* __restrict__ out, int out_ld,
                    const float* __restrict__ slot_gate, uint32_t* status) {
@@ -473,6 +474,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int4 tl = tiles[ti];
         const int half = ((tl.z + 15) & ~15) / 2;
         const int nbox = (half + kBoxN - 1) / kBoxN;
+        // a half of 65-128 rows comes as one box of twice the rows (tmB2): the
+        // same bytes in the same place from half the loads
+        const bool wide = nbox == 2;
         const int brow = tl.y + (int)rank * half;
         for (int kb = 0; kb < ksteps; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, status, abort_flag)) break;
@@ -488,8 +492,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d_pair(sa, &tmA0, kb * kBK,
                              tl.x * rows_per_expert + it * 256 + (int)rank * kBM, lbar, pol_w);
           }
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d_pair(sb + b * kBoxBytes, &tmB, kb * kBK, brow + b * kBoxN, lbar, pol_x);
+          if (wide)
+            tma_load_2d_pair(sb, &tmB2, kb * kBK, brow, lbar, pol_x);
+          else
+            for (int b = 0; b < nbox; ++b)
+              tma_load_2d_pair(sb + b * kBoxBytes, &tmB, kb * kBK, brow + b * kBoxN, lbar, pol_x);
           if (++stage == NS) {
             stage = 0;
             phase ^= 1u;
@@ -675,7 +682,7 @@ cudaError_t set_smem_attr() {
 
 template <int MODE>
 cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
-                        const int4* tiles, const int32_t* n_tiles, int max_tiles,
+                        const CUtensorMap& b2, const int4* tiles, const int32_t* n_tiles, int max_tiles,
                         int rows_per_expert, int K, int items_per_tile, int out_rows, void* out,
                         int out_ld, const float* slot_gate, uint32_t* status, int num_sms,
                         cudaStream_t s) {
@@ -698,7 +705,7 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const CUte
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_experts_pair<MODE>, a0, a1, b, tiles, n_tiles, max_tiles,
+  return cudaLaunchKernelEx(&cfg, k_experts_pair<MODE>, a0, a1, b, b2, tiles, n_tiles, max_tiles,
                             rows_per_expert, K, items_per_tile, out_rows, out, out_ld, slot_gate,
                             status);
 }
@@ -709,10 +716,11 @@ cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* 
                                  void* yslot, const int4* tiles, const int32_t* n_tiles,
                                  int max_tiles, const float* slot_gate, uint32_t* status,
                                  int num_sms, cudaStream_t s, cudaEvent_t ev_mid) {
-  CUtensorMap mg, mu, mx, md, mh;
+  CUtensorMap mg, mu, mx, mx2, md, mh;
   const uint64_t E = (uint64_t)L.E, d = (uint64_t)L.d, m = (uint64_t)L.m;
   if (!make_map(&mg, L.w_gate, E * m, d, 64) || !make_map(&mu, L.w_up, E * m, d, 64) ||
       !make_map(&mx, xp, (uint64_t)cap_slots, d, kBoxN) ||
+      !make_map(&mx2, xp, (uint64_t)cap_slots, d, 2 * kBoxN) ||
       !make_map(&md, L.w_down, E * d, m, kBM) || !make_map(&mh, h, (uint64_t)cap_slots, m, kBoxN))
     return cudaErrorInvalidValue;
   cudaError_t e;
@@ -721,7 +729,7 @@ cudaError_t launch_experts_sm100(const ace_layer& L, int cap_slots, const void* 
   // slower there, with 8 epilogue warps and bf16 outputs too (0.185 vs
   // 0.158 ms at 8192 tokens, 256 experts; 0.173 vs 0.156 ms at 4096
   // tokens, 0% skip).
-  if ((e = launch_pair<0>(mg, mu, mx, tiles, n_tiles, max_tiles, L.m, L.d, L.m / 128, L.m, h,
+  if ((e = launch_pair<0>(mg, mu, mx, mx2, tiles, n_tiles, max_tiles, L.m, L.d, L.m / 128, L.m, h,
                           L.m, slot_gate, status, num_sms, s)) != cudaSuccess)
     return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
