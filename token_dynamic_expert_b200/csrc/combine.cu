@@ -12,7 +12,14 @@
 
 namespace ace {
 
-// T: the storage type of Yslot and y; one 16-byte vector per thread and step
+// Kept slots whose rows one thread loads before it adds any of them
+constexpr int kCombineBatch = 8;
+
+// T: the storage type of Yslot and y; one 16-byte vector per thread and step.
+// Warp 0 first lists the token's kept positions in rank order (a ballot over
+// the k ranks), so a thread issues the loads of up to kCombineBatch rows
+// together and then adds them in rank order: the same sum, in the same order,
+// as one rank at a time.
 template <typename T>
 __global__ void __launch_bounds__(256) k_combine(int Tn, int k, int d,
                                                  const int32_t* __restrict__ slot_of,
@@ -20,28 +27,42 @@ __global__ void __launch_bounds__(256) k_combine(int Tn, int k, int d,
                                                  T* __restrict__ y, uint32_t* status) {
   constexpr int V = 16 / (int)sizeof(T);
   __shared__ int s_pos[kMaxK];
+  __shared__ int s_n;
   const int t = blockIdx.x;
-  if (threadIdx.x < k) {
-    int p = slot_of[(size_t)t * k + threadIdx.x];
-    if (p >= n_rows) {
-      raise_flag(status, ACE_FLAG_BAD_INDEX);
-      p = -1;
+  if (threadIdx.x < 32) {
+    const int r = threadIdx.x;
+    int p = -1;
+    if (r < k) {
+      p = slot_of[(size_t)t * k + r];
+      if (p >= n_rows) {
+        raise_flag(status, ACE_FLAG_BAD_INDEX);
+        p = -1;
+      }
     }
-    s_pos[threadIdx.x] = p;
+    const uint32_t kept = __ballot_sync(0xffffffffu, p >= 0);
+    if (p >= 0) s_pos[__popc(kept & ((1u << r) - 1u))] = p;
+    if (r == 0) s_n = __popc(kept);
   }
   __syncthreads();
+  const int n = s_n;
   const int nv = d / V;
   for (int iv = threadIdx.x; iv < nv; iv += blockDim.x) {
     float acc[V];
 #pragma unroll
     for (int c = 0; c < V; ++c) acc[c] = 0.f;
-    for (int r = 0; r < k; ++r) {
-      const int p = s_pos[r];
-      if (p < 0) continue;
-      const uint4 q = reinterpret_cast<const uint4*>(yslot + (size_t)p * d)[iv];
-      const T* e = reinterpret_cast<const T*>(&q);
+    for (int r0 = 0; r0 < n; r0 += kCombineBatch) {
+      uint4 q[kCombineBatch];
 #pragma unroll
-      for (int c = 0; c < V; ++c) acc[c] += to_f(e[c]);
+      for (int j = 0; j < kCombineBatch; ++j)
+        if (r0 + j < n) q[j] = reinterpret_cast<const uint4*>(yslot + (size_t)s_pos[r0 + j] * d)[iv];
+#pragma unroll
+      for (int j = 0; j < kCombineBatch; ++j) {
+        if (r0 + j < n) {
+          const T* e = reinterpret_cast<const T*>(&q[j]);
+#pragma unroll
+          for (int c = 0; c < V; ++c) acc[c] += to_f(e[c]);
+        }
+      }
     }
     uint4 o;
     T* oe = reinterpret_cast<T*>(&o);

@@ -31,6 +31,28 @@ __global__ void __launch_bounds__(256) k_scatter_gather(
   __shared__ int s_n[kScatterTok];
   const int t0 = blockIdx.x * kScatterTok;
   const int c = t0 / kChunk;
+  // Xp[pos] = x_t: one 16-byte vector of u per thread and step (four in
+  // flight), turned into x and stored to each kept slot of the token.  The
+  // first step's loads do not depend on the positions, so they are issued
+  // before the positions are worked out.
+  constexpr int V = 16 / (int)sizeof(T);
+  const int vpr = d / V;
+  const int total = kScatterTok * vpr;
+  uint4 v[4];
+  float r[4];
+  auto load_step = [&](int q0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int q = q0 + j * (int)blockDim.x;
+      const int tq = q / vpr, w = q - tq * vpr, t = t0 + tq;
+      r[j] = 0.f;
+      if (q < total && t < Tn) {
+        v[j] = reinterpret_cast<const uint4*>(u + (size_t)t * d)[w];
+        r[j] = inv_rms[t];
+      }
+    }
+  };
+  load_step(threadIdx.x);
   if (threadIdx.x < kScatterTok) s_n[threadIdx.x] = 0;
   __syncthreads();
   if ((int)threadIdx.x < kScatterTok * k) {
@@ -66,24 +88,8 @@ __global__ void __launch_bounds__(256) k_scatter_gather(
     }
   }
   __syncthreads();
-  // Xp[pos] = x_t: one 16-byte vector of u per thread and step (four in
-  // flight), turned into x and stored to each kept slot of the token
-  constexpr int V = 16 / (int)sizeof(T);
-  const int vpr = d / V;
-  const int total = kScatterTok * vpr;
   for (int q0 = threadIdx.x; q0 < total; q0 += 4 * blockDim.x) {
-    uint4 v[4];
-    float r[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int q = q0 + j * blockDim.x;
-      const int tq = q / vpr, w = q - tq * vpr, t = t0 + tq;
-      r[j] = 0.f;
-      if (q < total && t < Tn) {
-        v[j] = reinterpret_cast<const uint4*>(u + (size_t)t * d)[w];
-        r[j] = inv_rms[t];
-      }
-    }
+    if (q0 != (int)threadIdx.x) load_step(q0);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int q = q0 + j * blockDim.x;
@@ -92,8 +98,17 @@ __global__ void __launch_bounds__(256) k_scatter_gather(
         const T* e = reinterpret_cast<const T*>(&v[j]);
         uint4 o;
         T* oe = reinterpret_cast<T*>(&o);
+        float gg[V];  // gamma is 16-byte aligned (checked with the layer)
 #pragma unroll
-        for (int cc = 0; cc < V; ++cc) oe[cc] = from_f<T>(xhat(to_f(e[cc]), r[j], gamma[w * V + cc]));
+        for (int h = 0; h < V / 4; ++h) {
+          const float4 g4 = reinterpret_cast<const float4*>(gamma + (size_t)w * V)[h];
+          gg[4 * h] = g4.x;
+          gg[4 * h + 1] = g4.y;
+          gg[4 * h + 2] = g4.z;
+          gg[4 * h + 3] = g4.w;
+        }
+#pragma unroll
+        for (int cc = 0; cc < V; ++cc) oe[cc] = from_f<T>(xhat(to_f(e[cc]), r[j], gg[cc]));
         const int n = s_n[tq];
         for (int i = 0; i < n; ++i) reinterpret_cast<uint4*>(xp + (size_t)s_pos[tq][i] * d)[w] = o;
       }
