@@ -464,9 +464,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
   if (threadIdx.x == 0) {
     sh.abort = 0;
     sh.flags = 0u;
-    volatile const uint32_t* vs = a.sync;
-    sh.epoch = vs[0];
-    sh.fast = vs[1] == (sh.epoch ^ kCleanMark);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sh.full_c[i], 1);
       mbar_init(&sh.empty_c[i], wps_c);  // the slot's warps
@@ -478,6 +475,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
     mbar_init(&sh.in_bar, 1);
     sh.n_c_issued = sh.n_d_issued = sh.n_c_marked = 0;
     fence_barrier_init();
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) sh.tok_mask[e] = 0u;
+  // The launch may begin while the previous kernel of the stream drains
+  // (programmatic stream serialisation): the work above touches shared memory
+  // only, and nothing in global memory is read or written before this wait,
+  // which returns once that kernel has completed and its writes are visible.
+  // The next launch may then be scheduled; its CTAs take an SM only as this
+  // launch's CTAs leave (one CTA fills an SM's shared memory).
+  grid_dependency_wait();
+  if (threadIdx.x == 0) {
+    allow_dependent_launch();
+    volatile const uint32_t* vs = a.sync;
+    sh.epoch = vs[0];
+    sh.fast = vs[1] == (sh.epoch ^ kCleanMark);
     // one round trip for every input of phase A
     mbar_expect_tx(&sh.in_bar, (uint32_t)(NT * d * 2 + d * 4 + n_mine * d * 2));
     bulk_g2s(us, a.u, (uint32_t)(NT * d * 2), &sh.in_bar);
@@ -486,7 +497,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(const DecodeArgs a) {
       bulk_g2s(wrs + (size_t)r * d, a.wr + (size_t)((int)blockIdx.x + G * r) * d,
                (uint32_t)(d * 2), &sh.in_bar);
   }
-  for (int e = threadIdx.x; e < E; e += blockDim.x) sh.tok_mask[e] = 0u;
   stamp(a, 0);
   __syncthreads();  // barrier inits are visible
 
@@ -1068,11 +1078,13 @@ cudaError_t launch_decode(const ace_layer& L, int fusion, const void* u, int T, 
   cfg.blockDim = dim3(kDecThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attrs[1];
+  cudaLaunchAttribute attrs[2];
   attrs[0].id = cudaLaunchAttributeCooperative;
   attrs[0].val.cooperative = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   switch (T) {
     case 1: return launch_nt<1>(cfg, a, smem);
     case 2: return launch_nt<2>(cfg, a, smem);
