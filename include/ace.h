@@ -203,7 +203,10 @@ ACE_API size_t ace_workspace_size(const ace_layer* layer, int max_tokens);
  *   one cooperative kernel whose grid barriers count in 64 bytes of the
  *   workspace's status block; its last CTA writes the status word and
  *   leaves those words zeroed and marked for the next call, so the route
- *   launches nothing before the kernel.
+ *   launches nothing before the kernel.  The kernel may start while the
+ *   previous kernel of the stream is ending (programmatic stream
+ *   serialisation), but it reads and writes no global memory until that
+ *   kernel has completed, so stream order holds for every argument.
  * ---------------------------------------------------------------------- */
 ACE_API ace_status ace_moe_forward(const ace_layer* layer, const void* u, int T,
                            const ace_fwd_opts* opts, void* y, void* ws,
