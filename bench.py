@@ -36,19 +36,24 @@ import workloads  # noqa: E402
 METRIC = "MoE-layer tokens/s (prefill, decode) at skip rate; % of tensor/HBM roofline"
 
 # DRAM traffic (read + write bytes) per launch of the dominant kernel from one ncu
-# capture of that kernel on that workload; reported only while the kernel's source
-# is the revision the counters were taken on.
+# capture of that kernel on that workload at that skip rate; reported only while the
+# kernel's source is the revision the counters were taken on.
 PROFILED_TRAFFIC = {
-    ("prefill_1024", "fused"): ("token_dynamic_expert_b200/csrc/experts_fused_sm100.cu",
-                                "10553744e735", 1227740736),
+    ("prefill_1024", "fused", 0.6): ("token_dynamic_expert_b200/csrc/experts_fused_sm100.cu",
+                                     "10553744e735", 1227740736),
+    # gate/up launch of the 4096-token layer at 0% skip: 1.069221 GB read + 37.43 MB written
+    ("sweep_4096", "gateup", 0.0): ("token_dynamic_expert_b200/csrc/experts_sm100.cu",
+                                    "7f133c65c8f5", 1106649224),
 }
 
 
-def profiled_traffic(workload, kernel):
+def profiled_traffic(workload, kernel, rate):
     import hashlib
-    if (workload, kernel) not in PROFILED_TRAFFIC:
+    key = next((k for k in PROFILED_TRAFFIC
+                if k[:2] == (workload, kernel) and abs(k[2] - rate) < 1e-9), None)
+    if key is None:
         return None
-    path, sha, nbytes = PROFILED_TRAFFIC[(workload, kernel)]
+    path, sha, nbytes = PROFILED_TRAFFIC[key]
     with open(os.path.join(ROOT, path), "rb") as f:
         cur = hashlib.sha1(f.read()).hexdigest()[:12]
     return nbytes if cur == sha else None
@@ -400,7 +405,7 @@ def run_ours(args, w, rate, ws_n, rank, local):
                            "step_ms": spread},
         "roofline": {"bound": "hbm", "achieved": k_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": k_gbs / pk["hbm_gbs"],
-                     "traffic": profiled_traffic(w.name, "fused" if fused else "gateup"),
+                     "traffic": profiled_traffic(w.name, "fused" if fused else "gateup", rate),
                      "kernel": kname, "algorithmic_bytes": k_bytes, "kernel_ms": k_ms,
                      "algorithmic": "touched experts' weights + X in + Y out",
                      "bytes_incl_intermediates": k_bytes_incl,
