@@ -52,3 +52,20 @@ def test_single_rank_needs_no_process_group():
     import bench
     value, slowest = bench.replica_throughput(1, 4, 8, 2.0)
     assert slowest == 2.0 and value == pytest.approx(4 * 8 / 0.002)
+
+
+def test_profiled_traffic_follows_workload_rate_and_source():
+    """The measured DRAM traffic goes only on the line of the workload, kernel
+    and skip rate it was captured on, and only while the kernel's source is
+    the captured revision."""
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    for (wl, kern, rate), (path, sha, nbytes) in bench.PROFILED_TRAFFIC.items():
+        assert nbytes > 0
+        got = bench.profiled_traffic(wl, kern, rate)
+        assert got in (nbytes, None)  # None once the source has changed
+        assert bench.profiled_traffic(wl, kern, rate + 0.25) is None
+        other = "gateup" if kern == "fused" else "fused"
+        assert bench.profiled_traffic(wl, other, rate) is None
+    assert bench.profiled_traffic("decode_bs1", "fused", 0.6) is None
