@@ -105,6 +105,10 @@ def test_rmsnorm_closed_form_and_scale_invariance():
     xbar, x = oracle.rmsnorm(u, gamma, eps_rms=0.0)
     assert np.allclose(xbar, 1.0, rtol=1e-15)           # RMS(u) = 3
     assert np.allclose(x, gamma, rtol=1e-15)
+    # eps sits under the root with the mean square: mean(u^2) = 1, eps = 3
+    xbar, x = oracle.rmsnorm(np.ones((1, d)), gamma, eps_rms=3.0)
+    assert np.allclose(xbar, 0.5, rtol=1e-15)
+    assert np.allclose(x, 0.5 * gamma, rtol=1e-15)
     rng = np.random.default_rng(3)
     u = rng.normal(0, 1, (5, 32))
     xb1, _ = oracle.rmsnorm(u, np.ones(32), eps_rms=0.0)
@@ -223,6 +227,23 @@ def test_gsp_closed_form_scaled_identities():
     spec = oracle.gsp(gamma, wg, wu, wd, spectral=True, iters=50, eps=0.0)
     assert np.allclose(spec["a_tilde"], gd["expected_a_tilde_spectral"], rtol=1e-12)
     assert np.allclose(spec["A"], gd["expected_A"], rtol=1e-12)
+
+
+def test_gsp_closed_form_unequal_views():
+    """Diagonal experts whose two views differ (a^up != a^gate), so the
+    combination of the views and its normalisation are pinned by hand values."""
+    gd = _gold("gsp_diagonal_views.json")
+    diag = lambda rows: np.stack([np.diag(r) for r in rows]).astype(np.float32)
+    wg, wu, wd = diag(gd["w_gate_diag"]), diag(gd["w_up_diag"]), diag(gd["w_down_diag"])
+    gamma = np.ones(wg.shape[1])
+    fro = oracle.gsp(gamma, wg, wu, wd, spectral=False, eps=0.0)
+    assert np.allclose(fro["a_up"], gd["expected_a_up_fro"], rtol=1e-15)
+    assert np.allclose(fro["a_gate"], gd["expected_a_gate_fro"], rtol=1e-15)
+    assert np.allclose(fro["a_tilde"], gd["expected_a_tilde_fro"], rtol=1e-15)
+    assert np.allclose(fro["A"], gd["expected_A_fro"], rtol=1e-14)
+    spec = oracle.gsp(gamma, wg, wu, wd, spectral=True, iters=50, eps=0.0)
+    assert np.allclose(spec["a_tilde"], gd["expected_a_tilde_spectral"], rtol=1e-12)
+    assert np.allclose(spec["A"], gd["expected_A_spectral"], rtol=1e-12)
 
 
 def test_gsp_frobenius_products_match_library_and_gram_identity():
@@ -390,9 +411,17 @@ def test_tau_quantile_skips_exactly_n():
     T, k = 100, 4
     c = rng.uniform(0, 1, (T, k))
     N = T * (k - 1)
+    # slot r of every token routes to expert r with both tables at 1, so the
+    # fused score of a slot is its gate, here c
+    idx = np.tile(np.arange(k, dtype=np.int32), (T, 1))
+    ones = np.ones(k)
     for n in [0, 1, 7, 150, N - 1, N]:
         tau = oracle.tau_quantile(c, n)
         assert int((c[:, 1:] < tau).sum()) == n
+        # the mask's rule with the mapped tau skips exactly those n slots (the
+        # candidate equal to tau is kept)
+        mk = oracle.mask(idx, c, ones, ones, tau)
+        assert int((mk["keep"] == 0).sum()) == n
     assert oracle.n_skip_for(1024, 8, 0.6) == 4915
     assert oracle.n_skip_for(64, 2, 0.5, of="nontop1") == 32
 
