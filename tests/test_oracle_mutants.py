@@ -1,7 +1,10 @@
 """The oracle's pins catch plausible mistakes: each case below plants one
 mistake in a copy of the C oracle (a dropped term, a wrong sign, index or
 operand, a swapped role), builds the copy, points the oracle's front end at it
-and runs the pins of ``test_oracle_pins.py``; at least one pin must fail.
+and runs the pins of ``test_oracle_pins.py``; at least one pin must fail.  The
+two rules written in the Python front end (the slot count a skip rate asks for
+and the quantile mapping to tau) get the same treatment on a rewritten copy of
+the function.
 
 The planted mistakes stay in index range, so a mutant can give wrong numbers
 but never read or write outside its arrays.  Everything runs on the CPU.
@@ -153,6 +156,37 @@ def test_a_planted_mistake_fails_a_pin(name, old, new, first, pins, tmp_path, mo
         try:
             pins[p]()
         except Exception as e:  # an assertion, or numpy refusing the wrong numbers
+            caught = (p, type(e).__name__)
+            break
+    assert caught is not None, f"no pin fails with the planted mistake: {name}"
+
+
+# (name, front-end function, text in it, replacement)
+PY_MUTANTS = [
+    ("tau: one candidate too low", "tau_quantile", "return float(cand[n_skip])",
+     "return float(cand[n_skip - 1])"),
+    ("tau: top-1 slots among the candidates", "tau_quantile", "cand = np.sort(c[:, 1:].reshape(-1))",
+     "cand = np.sort(c.reshape(-1))"),
+    ("slot count: rounded down", "n_skip_for", "int(math.floor(rate * total + 0.5))",
+     "int(math.floor(rate * total))"),
+    ("slot count: the two bases swapped", "n_skip_for",
+     'total = T * k if of == "slots" else T * (k - 1)', 'total = T * (k - 1) if of == "slots" else T * k'),
+]
+
+
+@pytest.mark.parametrize("name,fn,old,new", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_a_planted_mistake_in_the_front_end_fails_a_pin(name, fn, old, new, pins, monkeypatch):
+    src = inspect.getsource(getattr(oracle_front, fn))
+    assert src.count(old) == 1, f"anchor not unique in {fn}: {old!r}"
+    scope = dict(vars(oracle_front))
+    exec(compile(src.replace(old, new), f"<mutant {fn}>", "exec"), scope)
+    monkeypatch.setattr(oracle_front, fn, scope[fn])
+    monkeypatch.setattr(oracle, fn, scope[fn])
+    caught = None
+    for p in sorted(pins):
+        try:
+            pins[p]()
+        except Exception as e:
             caught = (p, type(e).__name__)
             break
     assert caught is not None, f"no pin fails with the planted mistake: {name}"

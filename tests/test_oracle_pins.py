@@ -424,6 +424,9 @@ def test_tau_quantile_skips_exactly_n():
         assert int((mk["keep"] == 0).sum()) == n
     assert oracle.n_skip_for(1024, 8, 0.6) == 4915
     assert oracle.n_skip_for(64, 2, 0.5, of="nontop1") == 32
+    # halves round up: 0.25 of 10 slots asks for 3, 0.5 of 3 non-top-1 slots for 2
+    assert oracle.n_skip_for(10, 1, 0.25) == 3
+    assert oracle.n_skip_for(3, 2, 0.5, of="nontop1") == 2
 
 
 def test_compaction_order_and_bijection():
